@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""LSH attention forward throughput on B200: tokens/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, timed on host cores
+
+A step is one whole forward pass (hash -> sort -> chunked attention ->
+combine) over one batch of the workload, with inputs resident in HBM.  The
+default workload is the long-text shape: batch 1 x 8 heads, L = 65536,
+d_k = 64, bf16, 8 hashes, 1024 buckets, chunks of 64, causal.  Inputs are
+seeded synthetic N(0, 1) data.  L2 is flushed (a 256 MiB write) before every
+timed step; each step is timed with CUDA events on the launching stream.
+
+Multi-GPU: one process per GPU (torchrun), each rank runs the same workload on
+its own GPU -- (batch, head) pairs are independent, so there is no collective
+on the data path ("scaling": "weak"); the time is the max over ranks.
+
+Prints ONE JSON line on rank 0.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import lsh_bucketed_sparse_b200 as lsh  # noqa: E402
+from lsh_bucketed_sparse_b200 import workloads as W  # noqa: E402
+
+METRIC = "LSH-attention fwd tokens/s at L=65536, 8 hashes; % of HBM/tensor roofline"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = {
+    "hash": ["hash_tc.cu", "hash_portable.cu"],
+    "sort": ["sort.cu"],
+    "chunked_attention": ["attn_tc.cu", "attn_portable.cu"],
+    "combine": ["combine.cu"],
+}
+
+
+# ----------------------------------------------------------------- helpers --
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def stage_model(wl):
+    """Algorithmic bytes (HBM) and FLOPs per launch of each stage."""
+    BH, L, d, n_h, half, c = wl.batch * wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, \
+        wl.n_buckets // 2, wl.chunk_len
+    e = 2 if wl.dtype == torch.bfloat16 else 4
+    slots = BH * n_h * L
+    x = BH * L * d * e
+    rot = n_h * d * half * e
+    return {
+        "hash": {"bytes": x + rot + 2 * slots + 4 * BH * L,
+                 "flops": 2.0 * BH * L * d * half * n_h},
+        "sort": {"bytes": 2 * slots + 4 * slots, "flops": 0.0},
+        "chunked_attention": {"bytes": 4 * slots + n_h * 2 * x + n_h * 4 * BH * L
+                              + n_h * (x + 4 * BH * L),
+                              "flops": 4.0 * BH * n_h * L * (2 * c) * d},
+        "combine": {"bytes": n_h * (x + 4 * BH * L) + x + 4 * BH * L, "flops": 0.0},
+    }
+
+
+def source_sha(stage):
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[stage]:
+        with open(os.path.join(ROOT, "lsh_bucketed_sparse_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(stage, workload):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        rec = t[stage]
+        if rec.get("source_sha") != source_sha(stage) or rec.get("workload") != workload:
+            return None
+        return float(rec["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+
+    def summary(self):
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        max_mhz = max(r[1] for r in rows)
+        loaded = [r for r in rows if r[0] >= 0.5 * max_mhz] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4)
+                          if r[2][5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max_mhz,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ distributed --
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------- CPU baseline --
+def oracle_sample(wl, rounds):
+    """Time the oracle (as it stands) on one (batch, head) and ``rounds`` hashing
+    rounds of the workload: hash, sort, chunked attention, combine.  Returns
+    (seconds, tokens-equivalent of the full workload processed)."""
+    import numpy as np
+    from oracle import lsh_oracle as O
+    qk, v, rot = W.make_inputs(wl)
+    x = O.as_f64(qk[0, 0])
+    vv = O.as_f64(v[0, 0])
+    R = O.as_f64(rot[:rounds]) if rot is not None else None
+    t0 = time.perf_counter()
+    b, _ = O.hash_head(x, R, wl.n_buckets)
+    perm, _ = O.sort_head(b)
+    o = np.empty((rounds, wl.seq_len, wl.d_k))
+    lse = np.empty((rounds, wl.seq_len))
+    for r in range(rounds):
+        o[r], lse[r] = O.attend_round(x, vv, perm[r], wl.chunk_len, wl.causal)
+    O.combine_head(o, lse)
+    dt = time.perf_counter() - t0
+    frac = rounds / (wl.n_hashes * wl.batch * wl.heads)  # share of the whole workload
+    return dt, wl.tokens * frac
+
+
+def cpu_threads():
+    try:
+        import numpy  # noqa: F401
+        from threadpoolctl import threadpool_info
+        n = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        n = 1
+    return int(n)
+
+
+def cpu_baseline(wl, rounds):
+    dt, toks = oracle_sample(wl, rounds)
+    return {"value": toks / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"one (batch, head) of {wl.name}, {rounds} of {wl.n_hashes} hashing "
+                      f"rounds, full length: hash, sort, chunked attention, combine in "
+                      f"float64 numpy; {dt:.2f} s, scaled to the whole workload",
+            "seconds": dt, "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args, wl):
+    rank, world, _ = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(wl, 1)
+    times, toks = [], 0.0
+    for _ in range(args.steps):
+        dt, t = oracle_sample(wl, 1)
+        times.append(dt)
+        toks = t
+    total = sum(times)
+    value = toks * args.steps / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": dict(wl.describe(), sample="one (batch, head), one hashing round per step"),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_threads(),
+                             "kind": "oracle",
+                             "sample": "one (batch, head) and one hashing round of the workload "
+                                       "per step, scaled to the whole workload"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------- main --
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=W.HEADLINE.name, choices=list(W.BY_NAME))
+    ap.add_argument("--cpu-rounds", type=int, default=2,
+                    help="hashing rounds of one head the CPU baseline times")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    wl = W.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    rank, world, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    qk_h, v_h, rot_h = W.make_inputs(wl)
+    qk, v = qk_h.to(dev), v_h.to(dev)
+    rot = rot_h.to(dev) if rot_h is not None else None
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype)
+    ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qk)
+    lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
+                             workspace=ws, out=out, lse=lse)
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    lsh.lsh_attn_device_check()
+
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            starts[k].record(stream)
+            step()
+            ends[k].record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    lsh.lsh_attn_device_check()
+    ms_local = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    ms_total = max_over_ranks(ms_local, world)
+    ms_per_step = ms_total / args.steps
+    value = world * wl.tokens * args.steps / (ms_total / 1e3)
+
+    # Per-stage device time: the same kernels through the four stage calls.
+    stage_ms = {k: 0.0 for k in ("hash", "sort", "chunked_attention", "combine")}
+    n_stage = min(args.steps, 10)
+    for it in range(n_stage + 2):
+        flush.fill_(2.0)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+        ev[1].record(stream)
+        perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+        ev[2].record(stream)
+        o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                            n_buckets=wl.n_buckets)
+        ev[3].record(stream)
+        lsh.lsh_attn_combine(o_r, l_r)
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            for j, k in enumerate(stage_ms):
+                stage_ms[k] += ev[j].elapsed_time(ev[j + 1]) / n_stage
+        del b, inv, perm, o_r, l_r
+
+    # End to end through the host-buffer entry point: copies in and out timed.
+    pin = [t.pin_memory() if t is not None else None for t in (qk_h, v_h, rot_h)]
+    out_h = torch.empty_like(qk_h).pin_memory()
+    lse_h = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32).pin_memory()
+    dbuf = torch.empty(lsh.lsh_attn_forward_host_device_bytes(shp), dtype=torch.uint8, device=dev)
+    for _ in range(3):
+        lsh.lsh_attn_forward_host(shp, pin[0], pin[1], pin[2], out_h, lse_h, dbuf)
+    e2e_steps = min(args.steps, 10)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        lsh.lsh_attn_forward_host(shp, pin[0], pin[1], pin[2], out_h, lse_h, dbuf)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
+    h2d = sum(t.numel() * t.element_size() for t in pin if t is not None)
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+
+    # Roofline of the dominant kernel.
+    pk = peaks()
+    model = stage_model(wl)
+    dom = max(stage_ms, key=stage_ms.get)
+    sec = stage_ms[dom] / 1e3
+    m = model[dom]
+    if m["flops"] / (pk["bf16_tflops_sustained"] * 1e12) > m["bytes"] / (pk["hbm_gbs"] * 1e9):
+        achieved, peak, unit, bound = m["flops"] / sec / 1e12, pk["bf16_tflops_sustained"], \
+            "TFLOP/s", "tensor"
+    else:
+        achieved, peak, unit, bound = m["bytes"] / sec / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
+    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+                "frac": achieved / peak, "traffic": traffic_for(dom, wl.name),
+                "peak_source": pk["source"],
+                "algorithmic_bytes": m["bytes"], "algorithmic_flops": m["flops"],
+                "stage_ms": stage_ms}
+    total_bytes = sum(s["bytes"] for s in model.values())
+    total_flops = sum(s["flops"] for s in model.values())
+    t_roof = max(total_bytes / (pk["hbm_gbs"] * 1e9), total_flops / (pk["bf16_tflops"] * 1e12))
+    roofline["pass_roofline_ms"] = t_roof * 1e3
+    roofline["pass_frac"] = t_roof * 1e3 / ms_per_step
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(wl, args.cpu_rounds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
+            "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
+                           parallelism=f"independent (batch, head) problems, 1 per GPU x{world}"),
+            "clocks": clocks.summary(),
+            "e2e": {"value": world * wl.tokens / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms},
+            "gpu_launches": 4 * args.steps,
+            "roofline": roofline,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

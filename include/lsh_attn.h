@@ -1,0 +1,197 @@
+/*
+ * lsh_attn.h -- C ABI of liblsh_attn.so, the B200 (sm_100a) LSH attention
+ * forward pass: shared-QK attention restricted by random-rotation hashing,
+ * as described in "Reformer: The Efficient Transformer" (arXiv 2001.04451v2):
+ *   section 2 "LSH attention"     -- hash h(x) = argmax([xR; -xR]), sort by
+ *                                    bucket, attend within sorted chunks;
+ *   section 2 "Causal masking"    -- positions follow the same permutation,
+ *                                    future positions are masked, a token may
+ *                                    attend to itself only when nothing else
+ *                                    is available;
+ *   section 5 "Shared query-key space" -- one projection serves as query and
+ *                                    key; keys are normalised;
+ *   Appendix A "Multi-round attention" / "Implementation" / "Masking" --
+ *                                    n_hashes independent rounds, each giving
+ *                                    its own output, combined afterwards.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent)
+ *    unless the name ends in _host.  The caller owns every buffer, including
+ *    the workspace; the library never allocates, frees or keeps a pointer
+ *    after a call returns.
+ *  - Every device pointer must be 16-byte aligned.  Tensors are dense,
+ *    row-major, last dimension fastest.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream).  All work is enqueued on it; no call synchronises the host
+ *    except lsh_attn_device_check().
+ *  - Arguments are checked on the host before anything is launched.  A call
+ *    that returns anything but LSH_OK has launched nothing, except
+ *    LSH_ERR_CUDA (a launch or copy failed part-way; lsh_attn_last_error()
+ *    has the CUDA message).
+ *  - Shapes (see lsh_shape): B batch, H heads, L seq_len, d d_k,
+ *    n_h n_hashes, n_b n_buckets, c chunk_len.
+ *  - The library keeps no state between calls except one device word that
+ *    records a kernel's bounded wait running out (see lsh_attn_device_check).
+ */
+#ifndef LSH_ATTN_H_
+#define LSH_ATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define LSH_ATTN_VERSION 1
+
+#if defined(__GNUC__)
+#define LSH_ATTN_API __attribute__((visibility("default")))
+#else
+#define LSH_ATTN_API
+#endif
+
+typedef enum lsh_status {
+  LSH_OK = 0,
+  LSH_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size or flag */
+  LSH_ERR_UNSUPPORTED = 2,     /* valid request this build cannot serve    */
+  LSH_ERR_WORKSPACE = 3,       /* workspace or staging buffer too small     */
+  LSH_ERR_CUDA = 4,            /* a CUDA launch or copy failed              */
+  LSH_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait ran out           */
+} lsh_status;
+
+typedef enum lsh_dtype {
+  LSH_F32 = 0,                 /* float32 qk, v, rotations, out, o_rounds   */
+  LSH_BF16 = 1                 /* bfloat16 qk, v, rotations, out, o_rounds  */
+} lsh_dtype;
+
+/* lsh_shape.flags bits */
+#define LSH_FLAG_PORTABLE 1u   /* use the CUDA-core kernels even where the
+                                  tensor-core (tcgen05) kernels apply; for
+                                  cross-checking the two kernel families   */
+
+typedef struct lsh_shape {
+  int32_t batch;       /* B >= 1                                             */
+  int32_t heads;       /* H >= 1                                             */
+  int32_t seq_len;     /* L >= 1, a multiple of chunk_len, < 2^31 / n_h      */
+  int32_t d_k;         /* d: 8..256, a multiple of 8                         */
+  int32_t n_hashes;    /* n_h >= 1 hashing rounds                            */
+  int32_t n_buckets;   /* n_b: 1, or even with 2 <= n_b <= 32768             */
+  int32_t chunk_len;   /* c >= 1, divides L                                  */
+  int32_t causal;      /* 0 or 1                                             */
+  int32_t dtype;       /* lsh_dtype of the floating-point tensors            */
+  uint32_t flags;      /* LSH_FLAG_* bits, 0 by default                      */
+} lsh_shape;
+
+/* ---------------------------------------------------------------------- *
+ * Stage 1: hash.  Section 2 "LSH attention": h(x) = argmax([xR; -xR]) with
+ * a random projection R per round (Appendix A).
+ *   qk        [B, H, L, d]        dtype, the shared query/key vectors.
+ *   rotations [n_h, d, n_b/2]     dtype, one R per round, shared by all
+ *                                 (b, h); must be NULL when n_b == 1 (every
+ *                                 token then lands in bucket 0).
+ *   buckets   [B, H, n_h, L]      int16 out: the argmax index in [0, n_b);
+ *                                 ties go to the lowest index of [xR; -xR].
+ *                                 Projections are accumulated in float32
+ *                                 (exact bf16 products), so a position whose
+ *                                 top two entries of [xR; -xR] are within
+ *                                 float32 rounding may differ from an exact
+ *                                 evaluation.
+ *   inv_norm  [B, H, L]           float32 out: 1 / ||qk_i||_2, 0 for a zero row
+ *                                 (the key normalisation of section 5).
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, const void* rotations,
+                         int16_t* buckets, float* inv_norm, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Stage 2: sort.  Section 2 / Appendix A "Implementation": per (b, h, round)
+ * the positions ordered by bucket, positions increasing inside a bucket
+ * (a stable sort by bucket, i.e. by the key (round, bucket, position)).
+ *   buckets [B, H, n_h, L]  int16 in, values in [0, n_b).
+ *   perm    [B, H, n_h, L]  int32 out: perm[.., s] = position at sorted slot s.
+ *   undo    [B, H, n_h, L]  int32 out, may be NULL: undo[.., perm[.., s]] = s.
+ *   counts  [B, H, n_h, n_b] int32 out, may be NULL: tokens per bucket.
+ * Bucket ids outside [0, n_b) are undefined behaviour (stage 1 never makes
+ * them); the kernel does not read or write out of bounds for them.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
+                         int32_t* undo, int32_t* counts, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Stage 3: chunked attention of every round, results stored at ORIGINAL
+ * positions (the unsort is folded into the store).  Section 2 "LSH
+ * attention" / "Causal masking"; section 5 "Shared query-key space";
+ * Appendix A "Implementation" / "Masking".  For round r, sorted slot s sits
+ * in chunk k = s / c; its window is chunk k-1 (if k > 0) and chunk k.  The
+ * score of query i and key j is (qk_i . qk_j) * inv_norm_j / sqrt(d); the
+ * score of j == i is replaced by -1e5; with causal, j > i is excluded.
+ *   qk, v       [B, H, L, d]      dtype.
+ *   inv_norm    [B, H, L]         float32 (from stage 1).
+ *   perm        [B, H, n_h, L]    int32 (from stage 2).
+ *   o_rounds    [B, H, n_h, L, d] dtype out: softmax-weighted v per round.
+ *   lse_rounds  [B, H, n_h, L]    float32 out: log-sum-exp of the scores.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,
+                                const float* inv_norm, const int32_t* perm, void* o_rounds,
+                                float* lse_rounds, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Stage 4: combine.  Appendix A "Multi-round attention": each round's output
+ * is combined with weight exp(lse_r - LSE), LSE = logsumexp over rounds.
+ *   o_rounds [B, H, n_h, L, d] dtype; lse_rounds [B, H, n_h, L] float32.
+ *   out      [B, H, L, d] dtype out; lse [B, H, L] float32 out (= LSE).
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_combine(const lsh_shape* shape, const void* o_rounds,
+                            const float* lse_rounds, void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * The whole forward pass (stages 1-4) on one stream, no host sync.
+ * Produces the same out/lse as the four stage calls in sequence.
+ *   workspace: device scratch of at least lsh_attn_forward_workspace_size()
+ *   bytes, 256-byte aligned; its contents on entry do not matter and on
+ *   return are unspecified.  Two calls in flight at once need two workspaces.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_forward_workspace_size(const lsh_shape* shape, size_t* bytes);
+
+LSH_ATTN_API lsh_status lsh_attn_forward(const lsh_shape* shape, const void* qk, const void* v,
+                            const void* rotations, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * The forward pass from HOST buffers: copies qk, v and rotations to the
+ * device, runs lsh_attn_forward, and copies out and lse back, all enqueued on
+ * `stream`.  The caller synchronises `stream` before reading out_host /
+ * lse_host.  Host buffers should be page-locked for the copies to overlap.
+ *   device_buffer: caller-owned device memory of at least
+ *   lsh_attn_forward_host_device_bytes() bytes, 256-byte aligned; it holds the
+ *   device copies of the inputs and outputs plus the workspace.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_forward_host_device_bytes(const lsh_shape* shape, size_t* bytes);
+
+LSH_ATTN_API lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void* qk_host,
+                                 const void* v_host, const void* rotations_host,
+                                 void* out_host, float* lse_host, void* device_buffer,
+                                 size_t device_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Diagnostics.
+ *   lsh_attn_status_string: static text for a status.
+ *   lsh_attn_last_error: detail of the last failing call on this host
+ *   thread (static storage, overwritten by the next failure).
+ *   lsh_attn_device_check: synchronises `stream`, then reads and clears the
+ *   device word that a kernel sets when one of its bounded waits runs out;
+ *   returns LSH_ERR_DEVICE_TIMEOUT if it was set, LSH_ERR_CUDA if the
+ *   synchronisation failed, LSH_OK otherwise.
+ *   lsh_attn_version: LSH_ATTN_VERSION of the built library.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API const char* lsh_attn_status_string(lsh_status status);
+LSH_ATTN_API const char* lsh_attn_last_error(void);
+LSH_ATTN_API lsh_status lsh_attn_device_check(void* stream);
+LSH_ATTN_API int lsh_attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSH_ATTN_H_ */

@@ -1,0 +1,101 @@
+// Stage 4: combine the per-round outputs ("Reformer: The Efficient
+// Transformer", Appendix A "Multi-round attention": every round gives an
+// independently computable output; they are combined after unsorting):
+//   LSE_i = logsumexp_r lse_r,i,   out_i = sum_r exp(lse_r,i - LSE_i) o_r,i.
+//
+// Pure streaming: o_rounds is stored at original positions, so for a fixed
+// round consecutive threads read consecutive 16-byte pieces of consecutive
+// rows (coalesced), and out is written the same way.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lsh {
+namespace {
+
+constexpr int kThreads = 256;
+
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+  static constexpr int N = 4;
+  __device__ static void load(const float* p, float* f) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  }
+  __device__ static void store(float* p, const float* f) {
+    *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
+  }
+};
+template <> struct Vec16<__nv_bfloat16> {
+  static constexpr int N = 8;
+  __device__ static void load(const __nv_bfloat16* p, float* f) {
+    const uint4 u = *reinterpret_cast<const uint4*>(p);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const float2 x = __bfloat1622float2(h[t]);
+      f[2 * t] = x.x; f[2 * t + 1] = x.y;
+    }
+  }
+  __device__ static void store(__nv_bfloat16* p, const float* f) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int t = 0; t < 4; ++t) h[t] = __floats2bfloat162_rn(f[2 * t], f[2 * t + 1]);
+    *reinterpret_cast<uint4*>(p) = u;
+  }
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+combine_kernel(const T* __restrict__ o_rounds, const float* __restrict__ lse_rounds,
+               T* __restrict__ out, float* __restrict__ lse, long long rows, int L, int d,
+               int n_h) {
+  using V = Vec16<T>;
+  const int per_row = d / V::N;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long row = tid / per_row;
+  const int part = (int)(tid % per_row);
+  if (row >= rows) return;
+  const long long bh = row / L, i = row % L;
+  const float* lr = lse_rounds + bh * n_h * (long long)L + i;
+  float m = -INFINITY;
+  for (int r = 0; r < n_h; ++r) m = fmaxf(m, lr[(long long)r * L]);
+  float s = 0.f;
+  for (int r = 0; r < n_h; ++r) s += expf(lr[(long long)r * L] - m);
+  const float LSE = m + logf(s);
+  // exp(lse_r - LSE) evaluated as exp(lse_r - m) / s: the differences to the
+  // maximum stay exact even where |lse| is ~1e5 (a token that saw only itself).
+  const float inv_s = 1.f / s;
+  float acc[V::N];
+#pragma unroll
+  for (int t = 0; t < V::N; ++t) acc[t] = 0.f;
+  for (int r = 0; r < n_h; ++r) {
+    const float w = expf(lr[(long long)r * L] - m) * inv_s;
+    float f[V::N];
+    V::load(o_rounds + ((bh * n_h + r) * (long long)L + i) * d + part * V::N, f);
+#pragma unroll
+    for (int t = 0; t < V::N; ++t) acc[t] = fmaf(w, f[t], acc[t]);
+  }
+  V::store(out + row * d + part * V::N, acc);
+  if (part == 0) lse[row] = LSE;
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const Problem& p, const void* o_rounds, const float* lse_rounds,
+                           void* out, float* lse, cudaStream_t st) {
+  const long long rows = (long long)p.BH() * p.L;
+  const int per_row = p.d / (p.bf16 ? 8 : 4);
+  const long long threads = rows * per_row;
+  const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
+  if (p.bf16)
+    combine_kernel<__nv_bfloat16><<<blocks, kThreads, 0, st>>>(
+        (const __nv_bfloat16*)o_rounds, lse_rounds, (__nv_bfloat16*)out, lse, rows, p.L, p.d,
+        p.n_h);
+  else
+    combine_kernel<float><<<blocks, kThreads, 0, st>>>((const float*)o_rounds, lse_rounds,
+                                                       (float*)out, lse, rows, p.L, p.d, p.n_h);
+  return cudaGetLastError();
+}
+
+}  // namespace lsh

@@ -1,0 +1,51 @@
+// Internal interface between the C ABI layer (lsh_attn_api.cu) and the
+// kernel translation units.  Not installed; the public boundary is
+// include/lsh_attn.h.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lsh {
+
+// Validated copy of lsh_shape with the derived sizes every launcher needs.
+struct Problem {
+  int B, H, L, d, n_h, n_b, c;
+  bool causal;
+  bool bf16;         // element type of qk, v, rotations, out, o_rounds
+  bool portable;     // LSH_FLAG_PORTABLE: CUDA-core kernels only
+  int BH() const { return B * H; }
+  int half() const { return n_b / 2; }  // projections per round, 0 when n_b == 1
+  int n_chunks() const { return L / c; }
+  size_t elem() const { return bf16 ? 2 : 4; }
+};
+
+// Address of the device word that kernels set when a bounded wait runs out.
+// Resolved for the current device (cudaGetSymbolAddress); nullptr on error.
+unsigned int* device_error_word();
+
+// ---- stage 1: hash -------------------------------------------------------
+cudaError_t launch_hash_portable(const Problem& p, const void* qk, const void* rot,
+                                 int16_t* buckets, float* inv_norm, cudaStream_t st);
+bool hash_tc_supported(const Problem& p);
+cudaError_t launch_hash_tc(const Problem& p, const void* qk, const void* rot, int16_t* buckets,
+                           float* inv_norm, cudaStream_t st);
+
+// ---- stage 2: sort -------------------------------------------------------
+cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int32_t* undo,
+                        int32_t* counts, cudaStream_t st);
+
+// ---- stage 3: chunked attention --------------------------------------------
+cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,
+                                 const float* inv_norm, const int32_t* perm, void* o_rounds,
+                                 float* lse_rounds, cudaStream_t st);
+bool attn_tc_supported(const Problem& p);
+cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
+                           const int32_t* perm, void* o_rounds, float* lse_rounds,
+                           cudaStream_t st);
+
+// ---- stage 4: combine ------------------------------------------------------
+cudaError_t launch_combine(const Problem& p, const void* o_rounds, const float* lse_rounds,
+                           void* out, float* lse, cudaStream_t st);
+
+}  // namespace lsh

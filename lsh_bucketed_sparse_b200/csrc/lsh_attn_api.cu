@@ -1,0 +1,349 @@
+// C ABI of liblsh_attn.so (declared in include/lsh_attn.h): argument checks,
+// kernel selection, workspace layout and the host-buffer entry point.  Every
+// step of the computation runs in the kernels of this library; this file
+// only validates and launches.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "internal.h"
+#include "lsh_attn.h"
+
+namespace lsh {
+
+// Set by a kernel whose bounded wait runs out; read and cleared by
+// lsh_attn_device_check().
+__device__ unsigned int g_device_error_word = 0;
+
+namespace {
+
+thread_local char g_last_error[512] = "";
+
+lsh_status fail(lsh_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+lsh_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(LSH_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+std::once_flag g_word_once[kMaxDevices];
+unsigned int* g_word_ptr[kMaxDevices];
+
+lsh_status to_problem(const lsh_shape* s, Problem* p) {
+  if (!s) return fail(LSH_ERR_INVALID_ARG, "shape is NULL");
+  if (s->batch < 1 || s->heads < 1 || s->seq_len < 1)
+    return fail(LSH_ERR_INVALID_ARG, "batch, heads and seq_len must be >= 1");
+  if (s->d_k < 8 || s->d_k > 256 || s->d_k % 8)
+    return fail(LSH_ERR_INVALID_ARG, "d_k=%d: must be a multiple of 8 in [8, 256]", s->d_k);
+  if (s->n_hashes < 1) return fail(LSH_ERR_INVALID_ARG, "n_hashes must be >= 1");
+  if (!(s->n_buckets == 1 || (s->n_buckets >= 2 && s->n_buckets <= 32768 && s->n_buckets % 2 == 0)))
+    return fail(LSH_ERR_INVALID_ARG, "n_buckets=%d: must be 1 or even in [2, 32768]",
+                s->n_buckets);
+  if (s->chunk_len < 1 || s->seq_len % s->chunk_len)
+    return fail(LSH_ERR_INVALID_ARG, "chunk_len=%d must be >= 1 and divide seq_len=%d",
+                s->chunk_len, s->seq_len);
+  if (s->causal != 0 && s->causal != 1) return fail(LSH_ERR_INVALID_ARG, "causal must be 0 or 1");
+  if (s->dtype != LSH_F32 && s->dtype != LSH_BF16)
+    return fail(LSH_ERR_INVALID_ARG, "dtype=%d: must be LSH_F32 or LSH_BF16", s->dtype);
+  if (s->flags & ~LSH_FLAG_PORTABLE) return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
+  const long long bh = (long long)s->batch * s->heads;
+  if (bh > (1LL << 30)) return fail(LSH_ERR_INVALID_ARG, "batch*heads too large");
+  const long long chunks = bh * s->n_hashes * (s->seq_len / s->chunk_len);
+  if (chunks >= (1LL << 31) || (long long)s->n_hashes * s->seq_len >= (1LL << 31))
+    return fail(LSH_ERR_INVALID_ARG, "problem too large for 32-bit grid/slot indices");
+  p->B = s->batch; p->H = s->heads; p->L = s->seq_len; p->d = s->d_k;
+  p->n_h = s->n_hashes; p->n_b = s->n_buckets; p->c = s->chunk_len;
+  p->causal = s->causal != 0; p->bf16 = s->dtype == LSH_BF16;
+  p->portable = (s->flags & LSH_FLAG_PORTABLE) != 0;
+  return LSH_OK;
+}
+
+lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null = false) {
+  if (!ptr) return may_be_null ? LSH_OK : fail(LSH_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(ptr) % 16)
+    return fail(LSH_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return LSH_OK;
+}
+
+#define CHECK(x)                  \
+  do {                            \
+    lsh_status _s = (x);          \
+    if (_s != LSH_OK) return _s;  \
+  } while (0)
+
+lsh_status check_rotations(const Problem& p, const void* rot) {
+  if (p.n_b == 1) {
+    if (rot) return fail(LSH_ERR_INVALID_ARG, "rotations must be NULL when n_buckets == 1");
+    return LSH_OK;
+  }
+  return check_ptr(rot, "rotations");
+}
+
+// ---- stage bodies (arguments already checked) ---------------------------
+lsh_status run_hash(const Problem& p, const void* qk, const void* rot, int16_t* buckets,
+                    float* inv_norm, cudaStream_t st) {
+  cudaError_t e = (!p.portable && hash_tc_supported(p))
+                      ? launch_hash_tc(p, qk, rot, buckets, inv_norm, st)
+                      : launch_hash_portable(p, qk, rot, buckets, inv_norm, st);
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "hash launch");
+}
+
+lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int32_t* undo,
+                    int32_t* counts, cudaStream_t st) {
+  cudaError_t e = launch_sort(p, buckets, perm, undo, counts, st);
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
+}
+
+lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
+                    const int32_t* perm, void* o_r, float* lse_r, cudaStream_t st) {
+  cudaError_t e = (!p.portable && attn_tc_supported(p))
+                      ? launch_attn_tc(p, qk, v, inv_norm, perm, o_r, lse_r, st)
+                      : launch_attn_portable(p, qk, v, inv_norm, perm, o_r, lse_r, st);
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
+}
+
+lsh_status run_combine(const Problem& p, const void* o_r, const float* lse_r, void* out,
+                       float* lse, cudaStream_t st) {
+  cudaError_t e = launch_combine(p, o_r, lse_r, out, lse, st);
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "combine launch");
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace of the fused pass: buckets, inv_norm, perm, o_rounds, lse_rounds.
+struct Workspace {
+  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, total;
+};
+
+Workspace workspace_layout(const Problem& p) {
+  const size_t slots = (size_t)p.BH() * p.n_h * p.L;
+  Workspace w;
+  size_t off = 0;
+  w.buckets = off;    off += align256(slots * sizeof(int16_t));
+  w.inv_norm = off;   off += align256((size_t)p.BH() * p.L * sizeof(float));
+  w.perm = off;       off += align256(slots * sizeof(int32_t));
+  w.o_rounds = off;   off += align256(slots * p.d * p.elem());
+  w.lse_rounds = off; off += align256(slots * sizeof(float));
+  w.total = off;
+  return w;
+}
+
+lsh_status forward_body(const Problem& p, const void* qk, const void* v, const void* rot,
+                        void* out, float* lse, void* ws, cudaStream_t st) {
+  const Workspace w = workspace_layout(p);
+  char* base = static_cast<char*>(ws);
+  int16_t* buckets = reinterpret_cast<int16_t*>(base + w.buckets);
+  float* inv_norm = reinterpret_cast<float*>(base + w.inv_norm);
+  int32_t* perm = reinterpret_cast<int32_t*>(base + w.perm);
+  void* o_r = base + w.o_rounds;
+  float* lse_r = reinterpret_cast<float*>(base + w.lse_rounds);
+  CHECK(run_hash(p, qk, rot, buckets, inv_norm, st));
+  CHECK(run_sort(p, buckets, perm, nullptr, nullptr, st));
+  CHECK(run_attn(p, qk, v, inv_norm, perm, o_r, lse_r, st));
+  CHECK(run_combine(p, o_r, lse_r, out, lse, st));
+  return LSH_OK;
+}
+
+// Device-buffer layout of lsh_attn_forward_host: qk, v, rotations, out, lse, workspace.
+struct HostStaging {
+  size_t qk, v, rot, out, lse, ws, total, in_bytes, rot_bytes, out_bytes, lse_bytes;
+};
+
+HostStaging host_layout(const Problem& p) {
+  HostStaging h;
+  h.in_bytes = (size_t)p.BH() * p.L * p.d * p.elem();
+  h.rot_bytes = p.n_b > 1 ? (size_t)p.n_h * p.d * p.half() * p.elem() : 0;
+  h.out_bytes = h.in_bytes;
+  h.lse_bytes = (size_t)p.BH() * p.L * sizeof(float);
+  size_t off = 0;
+  h.qk = off;  off += align256(h.in_bytes);
+  h.v = off;   off += align256(h.in_bytes);
+  h.rot = off; off += align256(h.rot_bytes);
+  h.out = off; off += align256(h.out_bytes);
+  h.lse = off; off += align256(h.lse_bytes);
+  h.ws = off;  off += workspace_layout(p).total;
+  h.total = off;
+  return h;
+}
+
+}  // namespace
+
+unsigned int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::call_once(g_word_once[dev], [dev] {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_device_error_word) == cudaSuccess)
+      g_word_ptr[dev] = static_cast<unsigned int*>(ptr);
+  });
+  return g_word_ptr[dev];
+}
+
+}  // namespace lsh
+
+using namespace lsh;
+
+extern "C" {
+
+lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, const void* rotations,
+                         int16_t* buckets, float* inv_norm, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(qk, "qk"));
+  CHECK(check_rotations(p, rotations));
+  CHECK(check_ptr(buckets, "buckets"));
+  CHECK(check_ptr(inv_norm, "inv_norm"));
+  return run_hash(p, qk, rotations, buckets, inv_norm, static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
+                         int32_t* undo, int32_t* counts, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(buckets, "buckets"));
+  CHECK(check_ptr(perm, "perm"));
+  CHECK(check_ptr(undo, "undo", true));
+  CHECK(check_ptr(counts, "counts", true));
+  return run_sort(p, buckets, perm, undo, counts, static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,
+                                const float* inv_norm, const int32_t* perm, void* o_rounds,
+                                float* lse_rounds, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(qk, "qk"));
+  CHECK(check_ptr(v, "v"));
+  CHECK(check_ptr(inv_norm, "inv_norm"));
+  CHECK(check_ptr(perm, "perm"));
+  CHECK(check_ptr(o_rounds, "o_rounds"));
+  CHECK(check_ptr(lse_rounds, "lse_rounds"));
+  return run_attn(p, qk, v, inv_norm, perm, o_rounds, lse_rounds,
+                  static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_combine(const lsh_shape* shape, const void* o_rounds,
+                            const float* lse_rounds, void* out, float* lse, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(o_rounds, "o_rounds"));
+  CHECK(check_ptr(lse_rounds, "lse_rounds"));
+  CHECK(check_ptr(out, "out"));
+  CHECK(check_ptr(lse, "lse"));
+  return run_combine(p, o_rounds, lse_rounds, out, lse, static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_forward_workspace_size(const lsh_shape* shape, size_t* bytes) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (!bytes) return fail(LSH_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = workspace_layout(p).total;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_forward(const lsh_shape* shape, const void* qk, const void* v,
+                            const void* rotations, void* out, float* lse, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(qk, "qk"));
+  CHECK(check_ptr(v, "v"));
+  CHECK(check_rotations(p, rotations));
+  CHECK(check_ptr(out, "out"));
+  CHECK(check_ptr(lse, "lse"));
+  CHECK(check_ptr(workspace, "workspace"));
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(LSH_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t need = workspace_layout(p).total;
+  if (workspace_bytes < need)
+    return fail(LSH_ERR_WORKSPACE, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  return forward_body(p, qk, v, rotations, out, lse, workspace,
+                      static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_forward_host_device_bytes(const lsh_shape* shape, size_t* bytes) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (!bytes) return fail(LSH_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = host_layout(p).total;
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void* qk_host,
+                                 const void* v_host, const void* rotations_host,
+                                 void* out_host, float* lse_host, void* device_buffer,
+                                 size_t device_bytes, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (!qk_host || !v_host || !out_host || !lse_host)
+    return fail(LSH_ERR_INVALID_ARG, "a host buffer is NULL");
+  if (p.n_b == 1 && rotations_host)
+    return fail(LSH_ERR_INVALID_ARG, "rotations must be NULL when n_buckets == 1");
+  if (p.n_b > 1 && !rotations_host) return fail(LSH_ERR_INVALID_ARG, "rotations_host is NULL");
+  CHECK(check_ptr(device_buffer, "device_buffer"));
+  if (reinterpret_cast<uintptr_t>(device_buffer) % 256)
+    return fail(LSH_ERR_INVALID_ARG, "device_buffer is not 256-byte aligned");
+  const HostStaging h = host_layout(p);
+  if (device_bytes < h.total)
+    return fail(LSH_ERR_WORKSPACE, "device_buffer of %zu bytes, need %zu", device_bytes, h.total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  char* base = static_cast<char*>(device_buffer);
+  cudaError_t e;
+  // One cudaMemcpyAsync per tensor.
+  if ((e = cudaMemcpyAsync(base + h.qk, qk_host, h.in_bytes, cudaMemcpyHostToDevice, st)))
+    return cuda_fail(e, "copy qk to device");
+  if ((e = cudaMemcpyAsync(base + h.v, v_host, h.in_bytes, cudaMemcpyHostToDevice, st)))
+    return cuda_fail(e, "copy v to device");
+  if (h.rot_bytes &&
+      (e = cudaMemcpyAsync(base + h.rot, rotations_host, h.rot_bytes, cudaMemcpyHostToDevice, st)))
+    return cuda_fail(e, "copy rotations to device");
+  CHECK(forward_body(p, base + h.qk, base + h.v, h.rot_bytes ? base + h.rot : nullptr,
+                     base + h.out, reinterpret_cast<float*>(base + h.lse), base + h.ws, st));
+  if ((e = cudaMemcpyAsync(out_host, base + h.out, h.out_bytes, cudaMemcpyDeviceToHost, st)))
+    return cuda_fail(e, "copy out to host");
+  if ((e = cudaMemcpyAsync(lse_host, base + h.lse, h.lse_bytes, cudaMemcpyDeviceToHost, st)))
+    return cuda_fail(e, "copy lse to host");
+  return LSH_OK;
+}
+
+const char* lsh_attn_status_string(lsh_status status) {
+  switch (status) {
+    case LSH_OK: return "ok";
+    case LSH_ERR_INVALID_ARG: return "invalid argument";
+    case LSH_ERR_UNSUPPORTED: return "unsupported";
+    case LSH_ERR_WORKSPACE: return "workspace too small";
+    case LSH_ERR_CUDA: return "CUDA error";
+    case LSH_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* lsh_attn_last_error(void) { return g_last_error; }
+
+lsh_status lsh_attn_device_check(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  unsigned int* word = device_error_word();
+  if (!word) return fail(LSH_ERR_CUDA, "cannot resolve the device error word");
+  unsigned int v = 0;
+  if ((e = cudaMemcpy(&v, word, sizeof(v), cudaMemcpyDeviceToHost)) != cudaSuccess)
+    return cuda_fail(e, "read device error word");
+  if (v) {
+    const unsigned int zero = 0;
+    if ((e = cudaMemcpy(word, &zero, sizeof(zero), cudaMemcpyHostToDevice)) != cudaSuccess)
+      return cuda_fail(e, "clear device error word");
+    return fail(LSH_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait ran out (code 0x%x)", v);
+  }
+  return LSH_OK;
+}
+
+int lsh_attn_version(void) { return LSH_ATTN_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,107 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host (no GPU needed: validation runs before
+any CUDA call, and nothing here launches a kernel)."""
+
+import ctypes
+
+import pytest
+
+import lsh_bucketed_sparse_b200 as lsh
+from lsh_bucketed_sparse_b200 import build as B
+
+
+@pytest.fixture(scope="module")
+def L():
+    B.build()
+    return lsh.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = lsh.declared_symbols()
+    assert len(names) == 12, names
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.lsh_attn_version() == 1
+
+
+def test_status_strings(L):
+    for code, text in [(0, b"ok"), (1, b"invalid argument"), (3, b"workspace too small"),
+                       (5, b"device wait timed out")]:
+        assert L.lsh_attn_status_string(code) == text
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+STREAM = ctypes.c_void_p(0)
+
+
+def shape(**kw):
+    base = dict(batch=1, heads=2, seq_len=256, d_k=64, n_hashes=2, n_buckets=16, chunk_len=64,
+                causal=1, dtype=lsh.BF16, portable=False)
+    base.update(kw)
+    return lsh.make_shape(base["batch"], base["heads"], base["seq_len"], base["d_k"],
+                          base["n_hashes"], base["n_buckets"], base["chunk_len"], base["causal"],
+                          base["dtype"], base["portable"])
+
+
+def fwd(L, shp, ws_bytes=1 << 40, rot=FAKE, ws=FAKE, qk=FAKE):
+    return L.lsh_attn_forward(ctypes.byref(shp), qk, FAKE, rot, FAKE, FAKE, ws, ws_bytes, STREAM)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(seq_len=250),            # chunk_len does not divide seq_len
+    dict(d_k=60), dict(d_k=264), dict(d_k=0),
+    dict(n_buckets=7), dict(n_buckets=0), dict(n_buckets=65536),
+    dict(n_hashes=0), dict(batch=0), dict(chunk_len=0),
+    dict(dtype=7),
+])
+def test_bad_shape_is_rejected(L, kw):
+    assert fwd(L, shape(**kw)) == 1
+    assert L.lsh_attn_last_error()
+
+
+def test_bad_causal_flag_is_rejected(L):
+    shp = shape()
+    shp.causal = 2
+    assert fwd(L, shp) == 1
+
+
+def test_bad_pointers_are_rejected(L):
+    assert fwd(L, shape(), qk=None) == 1
+    assert fwd(L, shape(), qk=MISALIGNED) == 1
+    assert fwd(L, shape(), rot=None) == 1                       # n_b > 1 needs rotations
+    assert fwd(L, shape(n_buckets=1), rot=FAKE) == 1            # n_b == 1 forbids them
+    assert fwd(L, shape(), ws=ctypes.c_void_p((1 << 20) + 16)) == 1  # not 256-aligned
+    assert b"aligned" in L.lsh_attn_last_error()
+
+
+def test_workspace_size_and_too_small(L):
+    shp = shape()
+    need = lsh.lsh_attn_forward_workspace_size(shp)
+    slots = 1 * 2 * 2 * 256
+    assert need >= slots * (2 + 4 + 64 * 2 + 4) + 2 * 256 * 4
+    assert fwd(L, shp, ws_bytes=need - 1) == 3
+    assert lsh.lsh_attn_forward_host_device_bytes(shp) > need
+
+
+def test_unknown_flag_rejected(L):
+    shp = shape()
+    shp.flags = 4
+    assert fwd(L, shp) == 1
+
+
+def test_stage_calls_validate(L):
+    shp = shape()
+    assert L.lsh_attn_hash(ctypes.byref(shp), FAKE, FAKE, None, FAKE, STREAM) == 1
+    assert L.lsh_attn_sort(ctypes.byref(shp), FAKE, None, None, None, STREAM) == 1
+    assert L.lsh_attn_chunked_fwd(ctypes.byref(shp), FAKE, FAKE, FAKE, MISALIGNED, FAKE, FAKE,
+                                  STREAM) == 1
+    assert L.lsh_attn_combine(ctypes.byref(shp), FAKE, FAKE, FAKE, None, STREAM) == 1
+    assert L.lsh_attn_hash(None, FAKE, FAKE, FAKE, FAKE, STREAM) == 1
+
+
+def test_binding_fails_loudly_without_gpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        lsh.lsh_attn_forward(torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16),
+                             torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16), None, 1, 1, 64, True)

@@ -1,0 +1,222 @@
+"""CUDA path against the fp64 oracle, through the C ABI (needs an sm_100a GPU).
+
+Every stage is compared on seeded inputs: bucket ids exactly except near
+ties (reported), sort outputs bit for bit from the GPU's bucket ids, and the
+floating-point outputs within the tolerances in ``parity.py``.  The fused
+``lsh_attn_forward`` must equal the four stage calls bit for bit.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import lsh_bucketed_sparse_b200 as lsh
+from lsh_bucketed_sparse_b200 import workloads as W
+from oracle import lsh_oracle as O
+
+import parity as P
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+def _stages(wl, qk, v, rot, portable=False):
+    """Run the four stage calls and the fused call on the GPU."""
+    qk_d, v_d = qk.to(DEV), v.to(DEV)
+    rot_d = None if rot is None else rot.to(DEV)
+    buckets, inv_norm = lsh.lsh_attn_hash(qk_d, rot_d, wl.n_buckets, wl.n_hashes,
+                                          portable=portable)
+    perm, undo, counts = lsh.lsh_attn_sort(buckets, wl.n_buckets, want_counts=True)
+    o_r, lse_r = lsh.lsh_attn_chunked_fwd(qk_d, v_d, inv_norm, perm, wl.chunk_len, wl.causal,
+                                          n_buckets=wl.n_buckets, portable=portable)
+    out, lse = lsh.lsh_attn_combine(o_r, lse_r)
+    f_out, f_lse = lsh.lsh_attn_forward(qk_d, v_d, rot_d, wl.n_hashes, wl.n_buckets,
+                                        wl.chunk_len, wl.causal, portable=portable)
+    lsh.lsh_attn_device_check()
+    return dict(buckets=buckets, inv_norm=inv_norm, perm=perm, undo=undo, counts=counts,
+                o_rounds=o_r, lse_rounds=lse_r, out=out, lse=lse, f_out=f_out, f_lse=f_lse)
+
+
+def _full_check(wl, portable=False, qk_override=None):
+    qk, v, rot = W.make_inputs(wl)
+    if qk_override is not None:
+        qk = qk_override(qk)
+    g = _stages(wl, qk, v, rot, portable)
+    bf16 = wl.dtype == torch.bfloat16
+    report = {}
+    # hash
+    if wl.n_buckets > 1:
+        ob, margins = O.hash_all(qk, rot, wl.n_buckets)
+        report["buckets"] = P.check_buckets(g["buckets"], ob, margins)
+    else:
+        assert (g["buckets"] == 0).all()
+    xn = P.np64(qk)
+    norms = np.sqrt((xn * xn).sum(-1))
+    inv = np.where(norms > 0, 1.0 / np.where(norms > 0, norms, 1.0), 0.0)
+    np.testing.assert_allclose(P.np64(g["inv_norm"]), inv, rtol=2e-6, atol=0)
+    # everything downstream from the GPU's own bucket ids
+    res = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal,
+                    buckets=g["buckets"].cpu().numpy().astype(np.int64))
+    np.testing.assert_array_equal(g["perm"].cpu().numpy(), res["perm"])
+    np.testing.assert_array_equal(g["undo"].cpu().numpy(), res["undo"])
+    counts = np.stack([np.stack([np.stack([np.bincount(res["buckets"][b, h, r],
+                                                       minlength=wl.n_buckets)
+                                           for r in range(wl.n_hashes)])
+                                 for h in range(wl.heads)]) for b in range(wl.batch)])
+    np.testing.assert_array_equal(g["counts"].cpu().numpy(), counts)
+    report["o_rounds"] = P.check_float(g["o_rounds"], res["o_rounds"], bf16, "o_rounds", 3)
+    report["lse_rounds"] = P.check_lse(g["lse_rounds"], res["lse_rounds"], bf16, "lse_rounds")
+    report["out"] = P.check_float(g["out"], res["out"], bf16, "out")
+    report["lse"] = P.check_lse(g["lse"], res["lse"], bf16, "lse")
+    # the fused pass is the same kernels in the same order
+    assert torch.equal(g["f_out"], g["out"]) and torch.equal(g["f_lse"], g["lse"])
+    return report, g
+
+
+# Workloads small enough for the whole oracle, spanning several hash tiles
+# (128 rows), several chunks, a ragged hash tile and the edge cases.
+SMALL = [
+    W.small("bf16-causal-ragged", heads=2, seq_len=1088, n_hashes=3, n_buckets=32),
+    W.small("bf16-noncausal-d128", heads=2, seq_len=1024, d_k=128, n_hashes=2, n_buckets=64,
+            chunk_len=128, causal=False),
+    W.small("f32-causal", heads=2, seq_len=512, n_hashes=2, n_buckets=16, dtype=torch.float32),
+    W.small("bf16-one-chunk", heads=1, seq_len=64, n_hashes=2, n_buckets=8),
+    W.small("bf16-two-buckets", heads=2, seq_len=512, n_hashes=4, n_buckets=2),
+    W.small("bf16-c32-d32", heads=3, seq_len=768, d_k=32, n_hashes=2, n_buckets=12,
+            chunk_len=32),
+    W.small("bf16-clustered", heads=2, seq_len=2048, n_hashes=2, n_buckets=64, clustered=True,
+            n_clusters=16, causal=False),
+]
+
+
+@pytest.mark.parametrize("wl", SMALL, ids=[w.name for w in SMALL])
+@pytest.mark.parametrize("portable", [False, True], ids=["fast", "portable"])
+def test_small_workloads(wl, portable):
+    report, _ = _full_check(wl, portable)
+    print(wl.name, report)
+
+
+@pytest.mark.parametrize("idx", [0, 1, 2, 4])
+def test_named_workloads_full_size(idx):
+    wl = W.WORKLOADS[idx]
+    report, _ = _full_check(wl)
+    print(wl.name, report)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_full_attention_limit_on_gpu(causal):
+    # one bucket, one chunk over the whole sequence: plain shared-QK attention
+    wl = W.small("one-bucket", heads=2, seq_len=256, n_hashes=2, n_buckets=1, chunk_len=256,
+                 causal=causal, dtype=torch.float32)
+    report, g = _full_check(wl)
+    qk, v, _ = W.make_inputs(wl)
+    for h in range(2):
+        x = P.np64(qk[0, h])
+        kh = O.normalised_keys(x)
+        s = x @ kh.T / math.sqrt(wl.d_k)
+        np.fill_diagonal(s, O.SELF_SCORE)
+        if causal:
+            s = np.where(np.triu(np.ones_like(s, bool), 1), -np.inf, s)
+        p = np.exp(s - s.max(1, keepdims=True))
+        ref = (p / p.sum(1, keepdims=True)) @ P.np64(v[0, h])
+        assert np.abs(P.np64(g["out"][0, h]) - ref).max() < 1e-4
+
+
+def test_first_causal_token_outputs_its_value():
+    wl = W.small("first-token", heads=2, seq_len=512, n_hashes=4, n_buckets=16)
+    qk, v, rot = W.make_inputs(wl)
+    g = _stages(wl, qk, v, rot)
+    assert torch.equal(g["out"][:, :, 0].cpu(), v[:, :, 0])
+    assert (g["lse_rounds"][:, :, :, 0] == -1e5).all()
+
+
+def test_zero_rows_and_scaled_rows():
+    wl = W.small("zero-rows", heads=1, seq_len=256, n_hashes=2, n_buckets=16, causal=False)
+
+    def plant(qk):
+        qk = qk.clone()
+        qk[0, 0, 5] = 0
+        qk[0, 0, 77] = 0
+        qk[0, 0, 100] = qk[0, 0, 99] * 4  # exact rescale: same bucket in every round
+        return qk
+
+    report, g = _full_check(wl, qk_override=plant)
+    b = g["buckets"][0, 0]
+    assert (b[:, 5] == 0).all() and (b[:, 77] == 0).all()
+    assert torch.equal(b[:, 100], b[:, 99])
+    assert g["inv_norm"][0, 0, 5] == 0
+
+
+def test_deterministic():
+    wl = W.small("det", heads=2, seq_len=1024, n_hashes=2, n_buckets=32)
+    qk, v, rot = [t.to(DEV) if t is not None else None for t in W.make_inputs(wl)]
+    a = lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal)
+    b = lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal)
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_host_buffer_entry_point_matches():
+    wl = W.small("host", heads=2, seq_len=512, n_hashes=2, n_buckets=16)
+    qk, v, rot = W.make_inputs(wl)
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype)
+    dev = torch.empty(lsh.lsh_attn_forward_host_device_bytes(shp), dtype=torch.uint8,
+                      device=DEV)
+    qk_h, v_h, rot_h = qk.pin_memory(), v.pin_memory(), rot.pin_memory()
+    out_h = torch.empty_like(qk_h).pin_memory()
+    lse_h = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32).pin_memory()
+    lsh.lsh_attn_forward_host(shp, qk_h, v_h, rot_h, out_h, lse_h, dev)
+    torch.cuda.current_stream().synchronize()
+    ref_out, ref_lse = lsh.lsh_attn_forward(qk.to(DEV), v.to(DEV), rot.to(DEV), wl.n_hashes,
+                                            wl.n_buckets, wl.chunk_len, wl.causal)
+    assert torch.equal(out_h, ref_out.cpu()) and torch.equal(lse_h, ref_lse.cpu())
+
+
+def test_headline_workload_sampled():
+    """L = 65536, 8 hashes, 1024 buckets (the long-text shape) at full size, in the
+    configuration the benchmark times: buckets of one head in full and sampled
+    rows of the others against the oracle, the sort bit for bit everywhere, and
+    sampled tokens' per-round and combined outputs recomputed one by one."""
+    wl = W.HEADLINE
+    qk, v, rot = W.make_inputs(wl)
+    g = _stages(wl, qk, v, rot)
+    bf16 = True
+    gb = g["buckets"].cpu().numpy().astype(np.int64)
+    x64, v64, rot64 = P.np64(qk), P.np64(v), P.np64(rot)
+    rng = np.random.default_rng(0)
+    # hash: head 0 in full, 512 random rows of every other head
+    ob, om = O.hash_head(x64[0, 0], rot64, wl.n_buckets)
+    rep = P.check_buckets(gb[0, 0], ob, om)
+    for h in range(1, wl.heads):
+        rows = rng.choice(wl.seq_len, 512, replace=False)
+        ob, om = O.hash_head(x64[0, h, rows], rot64, wl.n_buckets)
+        P.check_buckets(gb[0, h][:, rows], ob, om)
+    print("headline buckets head 0:", rep)
+    # sort: every segment, bit for bit from the GPU's buckets
+    gp, gu = g["perm"].cpu().numpy(), g["undo"].cpu().numpy()
+    for h in range(wl.heads):
+        perm, undo = O.sort_head(gb[0, h])
+        np.testing.assert_array_equal(gp[0, h], perm)
+        np.testing.assert_array_equal(gu[0, h], undo)
+    # attention + combine at sampled tokens (including the first, causal edge)
+    go_r, gl_r = g["o_rounds"], g["lse_rounds"]
+    for h in range(wl.heads):
+        toks = np.concatenate([[0, 1, wl.seq_len - 1], rng.choice(wl.seq_len, 61, replace=False)])
+        o_or, o_lr, o_out, o_lse = [], [], [], []
+        for i in toks:
+            o, l = O.token_rounds(x64[0, h], v64[0, h], gp[0, h], gu[0, h], wl.chunk_len,
+                                  wl.causal, int(i))
+            out_i, lse_i = O.combine_head(o[:, None], l[:, None])
+            o_or.append(o); o_lr.append(l); o_out.append(out_i[0]); o_lse.append(lse_i[0])
+        t = torch.as_tensor(toks, device=DEV)
+        P.check_float(go_r[0, h][:, t].transpose(0, 1)[None, None].cpu(),
+                      np.array(o_or)[None, None], bf16, "o_rounds(sampled)")
+        P.check_lse(gl_r[0, h][:, t].transpose(0, 1).cpu(), np.array(o_lr), bf16,
+                    "lse_rounds(sampled)")
+        P.check_float(g["f_out"][0, h][t][None, None].cpu(), np.array(o_out)[None, None], bf16,
+                      "out(sampled)")
+        P.check_lse(g["f_lse"][0, h][t].cpu(), np.array(o_lse), bf16, "lse(sampled)")
+    assert torch.equal(g["f_out"], g["out"]) and torch.equal(g["f_lse"], g["lse"])
