@@ -175,6 +175,37 @@ LSH_ATTN_API lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void
                                  size_t device_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- *
+ * The forward pass without any device allocation or caller workspace.
+ * (The paper has no counterpart: this is a deployment aid of this library.)
+ *
+ * For callers that cannot allocate device memory: a plugin inside a host
+ * framework that owns all device memory through its own pool and hands the
+ * plugin only its input and output buffers, or a latency-critical path that
+ * must not call cudaMalloc because it can synchronise the whole device and
+ * take an unpredictable time.  Same arguments and results as
+ * lsh_attn_forward, minus the workspace: the intermediates live in a scratch
+ * array of LSH_ATTN_NOALLOC_SCRATCH_BYTES built into the library.
+ *  - The scratch occupies that much device memory on every GPU where this
+ *    call has run, from the first call there until the process exits.
+ *  - The first call on a device resolves the scratch's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - Problems whose workspace (lsh_attn_forward_workspace_size) exceeds
+ *    LSH_ATTN_NOALLOC_SCRATCH_BYTES are rejected with LSH_ERR_WORKSPACE
+ *    before anything is launched.
+ *  - Every call on a device shares the one scratch and leaves its contents
+ *    behind; nothing in it needs to start at zero.  Calls that overlap on
+ *    the GPU (different streams, or different host threads, without ordering
+ *    between them) race on the scratch and give wrong results: order them.
+ *  - Calls no cudaMalloc, cudaFree or any other allocating routine.
+ * ---------------------------------------------------------------------- */
+#define LSH_ATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+LSH_ATTN_API lsh_status lsh_attn_forward_noalloc(const lsh_shape* shape, const void* qk,
+                                                 const void* v, const void* rotations,
+                                                 void* out, float* lse, void* stream);
+
+/* ---------------------------------------------------------------------- *
  * Diagnostics.
  *   lsh_attn_status_string: static text for a status.
  *   lsh_attn_last_error: detail of the last failing call on this host

@@ -23,7 +23,8 @@ __all__ = [
     "LshError", "Shape", "lib", "make_shape", "lsh_attn_hash", "lsh_attn_sort",
     "lsh_attn_chunked_fwd", "lsh_attn_combine", "lsh_attn_forward",
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
-    "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "LIB_PATH", "HEADER_PATH",
+    "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
+    "LIB_PATH", "HEADER_PATH", "NOALLOC_SCRATCH_BYTES",
     "F32", "BF16", "FLAG_PORTABLE",
 ]
 
@@ -33,6 +34,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "lsh_attn.h")
 
 F32, BF16 = 0, 1
 FLAG_PORTABLE = 1
+NOALLOC_SCRATCH_BYTES = 64 << 20  # LSH_ATTN_NOALLOC_SCRATCH_BYTES
 STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED",
           3: "LSH_ERR_WORKSPACE", 4: "LSH_ERR_CUDA", 5: "LSH_ERR_DEVICE_TIMEOUT"}
 
@@ -64,6 +66,7 @@ _SIGS = {
     "lsh_attn_forward": [_SHP, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "lsh_attn_forward_host_device_bytes": [_SHP, ctypes.POINTER(_SZ)],
     "lsh_attn_forward_host": [_SHP, _P, _P, _P, _P, _P, _P, _SZ, _P],
+    "lsh_attn_forward_noalloc": [_SHP, _P, _P, _P, _P, _P, _P],
     "lsh_attn_status_string": [ctypes.c_int],
     "lsh_attn_last_error": [],
     "lsh_attn_device_check": [_P],
@@ -251,6 +254,31 @@ def lsh_attn_forward_host(shape: Shape, qk_host, v_host, rot_host, out_host, lse
         ctypes.byref(shape), _ptr(qk_host), _ptr(v_host), _ptr(rot_host), _ptr(out_host),
         _ptr(lse_host), _ptr(device_buffer), ctypes.c_size_t(device_buffer.numel()),
         _stream(stream)))
+
+
+def lsh_attn_forward_noalloc(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *,
+                             out=None, lse=None, portable=False, stream=None):
+    """The fused pass with no workspace and no device allocation inside the
+    library: for callers that are handed only input and output buffers (a
+    plugin whose host framework owns all device memory) or that must not call
+    cudaMalloc on a latency-critical path.  The intermediates live in a
+    64 MiB scratch array inside the library, shared by every call on the
+    device, so calls must not overlap on the GPU; larger problems raise
+    LshError(LSH_ERR_WORKSPACE).  (This Python wrapper still allocates ``out``
+    and ``lse`` with torch when they are not passed in.)"""
+    _cuda(qk, "qk")
+    _cuda(v, "v", qk.dtype)
+    if rotations is not None:
+        _cuda(rotations, "rotations", qk.dtype)
+    B, H, L, d = qk.shape
+    shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable)
+    if out is None:
+        out = torch.empty_like(qk)
+    if lse is None:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
+    _check(lib().lsh_attn_forward_noalloc(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(rotations),
+                                          _ptr(out), _ptr(lse), _stream(stream)))
+    return out, lse
 
 
 def lsh_attn_device_check(stream=None):

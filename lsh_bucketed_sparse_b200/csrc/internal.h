@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "lsh_attn.h"
+
 namespace lsh {
 
 // Validated copy of lsh_shape with the derived sizes every launcher needs.
@@ -19,6 +21,25 @@ struct Problem {
   int n_chunks() const { return L / c; }
   size_t elem() const { return bf16 ? 2 : 4; }
 };
+
+// ---- shared by the C ABI entry points (lsh_attn_api.cu) ------------------
+// Record a failure message for lsh_attn_last_error() and return `st`.
+lsh_status fail(lsh_status st, const char* fmt, ...);
+lsh_status cuda_fail(cudaError_t e, const char* what);
+// Validate the public shape into a Problem.
+lsh_status to_problem(const lsh_shape* s, Problem* p);
+// NULL (unless may_be_null) or not 16-byte aligned -> LSH_ERR_INVALID_ARG.
+lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null = false);
+// rotations must be NULL exactly when n_buckets == 1.
+lsh_status check_rotations(const Problem& p, const void* rot);
+// Byte offsets of the fused pass's intermediates inside its workspace.
+struct Workspace {
+  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, total;
+};
+Workspace workspace_layout(const Problem& p);
+// Stages 1-4 into a checked workspace of workspace_layout(p).total bytes.
+lsh_status forward_body(const Problem& p, const void* qk, const void* v, const void* rot,
+                        void* out, float* lse, void* ws, cudaStream_t st);
 
 // Address of the device word that kernels set when a bounded wait runs out.
 // Resolved for the current device (cudaGetSymbolAddress); nullptr on error.

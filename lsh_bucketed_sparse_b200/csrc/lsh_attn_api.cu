@@ -17,8 +17,8 @@ namespace lsh {
 __device__ unsigned int g_device_error_word = 0;
 
 namespace {
-
 thread_local char g_last_error[512] = "";
+}  // namespace
 
 lsh_status fail(lsh_status st, const char* fmt, ...) {
   va_list ap;
@@ -32,9 +32,13 @@ lsh_status cuda_fail(cudaError_t e, const char* what) {
   return fail(LSH_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
+namespace {
+
 constexpr int kMaxDevices = 64;
 std::once_flag g_word_once[kMaxDevices];
 unsigned int* g_word_ptr[kMaxDevices];
+
+}  // namespace
 
 lsh_status to_problem(const lsh_shape* s, Problem* p) {
   if (!s) return fail(LSH_ERR_INVALID_ARG, "shape is NULL");
@@ -65,18 +69,22 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   return LSH_OK;
 }
 
-lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null = false) {
+lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null) {
   if (!ptr) return may_be_null ? LSH_OK : fail(LSH_ERR_INVALID_ARG, "%s is NULL", name);
   if (reinterpret_cast<uintptr_t>(ptr) % 16)
     return fail(LSH_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
   return LSH_OK;
 }
 
+namespace {
+
 #define CHECK(x)                  \
   do {                            \
     lsh_status _s = (x);          \
     if (_s != LSH_OK) return _s;  \
   } while (0)
+
+}  // namespace
 
 lsh_status check_rotations(const Problem& p, const void* rot) {
   if (p.n_b == 1) {
@@ -85,6 +93,8 @@ lsh_status check_rotations(const Problem& p, const void* rot) {
   }
   return check_ptr(rot, "rotations");
 }
+
+namespace {
 
 // ---- stage bodies (arguments already checked) ---------------------------
 lsh_status run_hash(const Problem& p, const void* qk, const void* rot, int16_t* buckets,
@@ -117,10 +127,7 @@ lsh_status run_combine(const Problem& p, const void* o_r, const float* lse_r, vo
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace of the fused pass: buckets, inv_norm, perm, o_rounds, lse_rounds.
-struct Workspace {
-  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, total;
-};
+}  // namespace
 
 Workspace workspace_layout(const Problem& p) {
   const size_t slots = (size_t)p.BH() * p.n_h * p.L;
@@ -150,6 +157,8 @@ lsh_status forward_body(const Problem& p, const void* qk, const void* v, const v
   CHECK(run_combine(p, o_r, lse_r, out, lse, st));
   return LSH_OK;
 }
+
+namespace {
 
 // Device-buffer layout of lsh_attn_forward_host: qk, v, rotations, out, lse, workspace.
 struct HostStaging {

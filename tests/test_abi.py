@@ -18,7 +18,8 @@ def L():
 
 def test_exports_every_declared_symbol(L):
     names = lsh.declared_symbols()
-    assert len(names) == 12, names
+    assert {"lsh_attn_hash", "lsh_attn_sort", "lsh_attn_chunked_fwd", "lsh_attn_combine",
+            "lsh_attn_forward", "lsh_attn_forward_workspace_size"} <= set(names), names
     for n in names:
         assert hasattr(L, n), n
     assert L.lsh_attn_version() == 1
