@@ -257,6 +257,53 @@ def run_reference(args, wl):
     return 0
 
 
+def run_one_stage(args, wl):
+    """Time one stage of the pass by itself on GPU 0 (inputs prepared by the
+    earlier stages outside the timed loop).  Used to profile a single kernel."""
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    qk_h, v_h, rot_h = W.make_inputs(wl)
+    qk, v = qk_h.to(dev), v_h.to(dev)
+    rot = rot_h.to(dev) if rot_h is not None else None
+    b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+    perm = o_r = l_r = None
+    if args.only_stage in ("sort", "chunked_attention", "combine"):
+        perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+    if args.only_stage in ("chunked_attention", "combine"):
+        o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                            n_buckets=wl.n_buckets)
+    if args.only_stage != "chunked_attention":
+        del v
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    calls = {
+        "hash": lambda: lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes),
+        "sort": lambda: lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False),
+        "chunked_attention": lambda: lsh.lsh_attn_chunked_fwd(
+            qk, v, inv, perm, wl.chunk_len, wl.causal, n_buckets=wl.n_buckets),
+        "combine": lambda: lsh.lsh_attn_combine(o_r, l_r),
+    }
+    fn = calls[args.only_stage]
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        fn()
+    ms = 0.0
+    for k in range(args.steps):
+        flush.fill_(float(k))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms += e0.elapsed_time(e1)
+    lsh.lsh_attn_device_check()
+    m = stage_model(wl)[args.only_stage]
+    sec = ms / args.steps / 1e3
+    print(json.dumps({"stage": args.only_stage, "workload": wl.name, "ms": sec * 1e3,
+                      "GB/s": m["bytes"] / sec / 1e9, "TFLOP/s": m["flops"] / sec / 1e12}),
+          flush=True)
+    return 0
+
+
 # ----------------------------------------------------------------- main --
 def main(argv=None):
     ap = argparse.ArgumentParser()
@@ -268,10 +315,14 @@ def main(argv=None):
     ap.add_argument("--cpu-rounds", type=int, default=2,
                     help="hashing rounds of one head the CPU baseline times")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only-stage", choices=["hash", "sort", "chunked_attention", "combine"],
+                    help="time one stage call alone (for profiling); prints its own JSON line")
     args = ap.parse_args(argv)
     wl = W.BY_NAME[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
+    if args.only_stage:
+        return run_one_stage(args, wl)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

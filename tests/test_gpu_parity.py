@@ -89,6 +89,14 @@ SMALL = [
             chunk_len=32),
     W.small("bf16-clustered", heads=2, seq_len=2048, n_hashes=2, n_buckets=64, clustered=True,
             n_clusters=16, causal=False),
+    # shapes that take the tensor-core hash: several rounds per MMA piece and a
+    # ragged last tile; one round split over two pieces; d = 128 with a
+    # 384-column round; 96-column rounds packed two per piece
+    W.small("tc-hash-ragged", heads=2, seq_len=1088, n_hashes=3, n_buckets=64),
+    W.small("tc-hash-wide", heads=2, seq_len=1024, n_hashes=2, n_buckets=1024),
+    W.small("tc-hash-d128-p384", heads=2, seq_len=512, d_k=128, n_hashes=2, n_buckets=768,
+            chunk_len=128, causal=False),
+    W.small("tc-hash-p96", heads=3, seq_len=768, n_hashes=4, n_buckets=192),
 ]
 
 
@@ -126,7 +134,7 @@ def test_full_attention_limit_on_gpu(causal):
 
 
 def test_first_causal_token_outputs_its_value():
-    wl = W.small("first-token", heads=2, seq_len=512, n_hashes=4, n_buckets=16)
+    wl = W.small("first-token", heads=2, seq_len=512, n_hashes=4, n_buckets=64)
     qk, v, rot = W.make_inputs(wl)
     g = _stages(wl, qk, v, rot)
     assert torch.equal(g["out"][:, :, 0].cpu(), v[:, :, 0])
@@ -134,7 +142,7 @@ def test_first_causal_token_outputs_its_value():
 
 
 def test_zero_rows_and_scaled_rows():
-    wl = W.small("zero-rows", heads=1, seq_len=256, n_hashes=2, n_buckets=16, causal=False)
+    wl = W.small("zero-rows", heads=1, seq_len=256, n_hashes=2, n_buckets=64, causal=False)
 
     def plant(qk):
         qk = qk.clone()
@@ -151,7 +159,7 @@ def test_zero_rows_and_scaled_rows():
 
 
 def test_deterministic():
-    wl = W.small("det", heads=2, seq_len=1024, n_hashes=2, n_buckets=32)
+    wl = W.small("det", heads=2, seq_len=1024, n_hashes=2, n_buckets=64)
     qk, v, rot = [t.to(DEV) if t is not None else None for t in W.make_inputs(wl)]
     a = lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal)
     b = lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal)
