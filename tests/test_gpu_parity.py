@@ -97,6 +97,14 @@ SMALL = [
     W.small("tc-hash-d128-p384", heads=2, seq_len=512, d_k=128, n_hashes=2, n_buckets=768,
             chunk_len=128, causal=False),
     W.small("tc-hash-p96", heads=3, seq_len=768, n_hashes=4, n_buckets=192),
+    # the four tensor-core attention specialisations (chunk, d_k)
+    W.small("tc-attn-c64-d128", heads=2, seq_len=1472, d_k=128, n_hashes=2, n_buckets=64),
+    W.small("tc-attn-c128-d64-causal", heads=2, seq_len=1408, n_hashes=3, n_buckets=64,
+            chunk_len=128),
+    W.small("tc-attn-c128-d128-causal", heads=1, seq_len=2048, d_k=128, n_hashes=2,
+            n_buckets=128, chunk_len=128),
+    W.small("tc-attn-c64-d64-noncausal", batch=2, heads=2, seq_len=1536, n_hashes=2,
+            n_buckets=128, causal=False),
 ]
 
 
