@@ -12,25 +12,30 @@
 // query rows (chunk 2s) see key columns [0, 128) and the last 64 (chunk
 // 2s+1) see [64, 192); with c = 128 every row sees all 256 columns.
 //
-// Data flow per step (warp-specialised, 6 warps):
-//   warp 0      producer: reads perm for the next 128 slots, gathers their
-//               qk and v rows with cp.async into a ring of shared-memory
-//               blocks (128B-swizzled operand layout), and stores each
-//               row's position, key scale (1/||x|| * log2 e / sqrt(d)) and
-//               query reference ||x|| * log2 e / sqrt(d);
+// Data flow per step (warp-specialised, 11 warps):
+//   warp 0      qk producer: reads perm for the next 128 slots and gathers
+//               their qk rows with TMA (tile::gather4, four rows per lane
+//               and instruction) into a ring of shared-memory blocks in the
+//               128B-swizzled operand layout, and stores each row's
+//               position, key scale (1/||x|| * log2 e / sqrt(d)) and query
+//               reference ||x|| * log2 e / sqrt(d);
+//   warp 10     v producer: the same gathers from v, so that keys never wait
+//               for values;
 //   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two MMAs per
 //               k-step: look-back keys and current keys live in different
 //               blocks), then O = P V with P from shared memory;
-//   warps 2..5  softmax: one query row per thread, straight from TMEM.
-//               Keys are unit-normalised, so q . k_hat / sqrt(d) never
-//               exceeds ||q|| / sqrt(d): that bound is the exponent's
-//               reference (p = 2^(s' - ref) <= 1) and no row maximum is
-//               needed; a row whose sum underflows is redone with its exact
-//               maximum.  Masks: window, causal (key position > query
-//               position), self (the key j == i is left out and a row with
-//               no other key outputs v_i with lse -1e5, the value the -1e5
-//               self score gives).  Then O / l and lse go to the row's
-//               original position.
+//   warps 2..9  softmax: two warps per TMEM lane quadrant (32 query rows),
+//               each taking alternate 32-key chunks of the row, straight
+//               from TMEM.  Keys are unit-normalised, so q . k_hat / sqrt(d)
+//               never exceeds ||q|| / sqrt(d): that bound is the exponent's
+//               reference (p = 2^(s' - ref) <= 1), so no row maximum is
+//               needed and the two warps only add their partial sums; a row
+//               whose sum underflows is redone with its exact maximum.
+//               Masks: window, causal (key position > query position), self
+//               (the key j == i is left out and a row with no other key
+//               outputs v_i with lse -1e5, the value the -1e5 self score
+//               gives).  Then O / l (each warp half of the columns) and lse
+//               go to the row's original position.
 #include <algorithm>
 #include <climits>
 
@@ -44,8 +49,9 @@ namespace {
 using namespace sm100;
 
 constexpr int kQ = 128;             // queries per step = rows per block = MMA M
-constexpr int kSoftWarps = 4;
-constexpr int kThreads = (2 + kSoftWarps) * 32;
+constexpr int kSoftWarps = 8;
+constexpr int kThreads = (3 + kSoftWarps) * 32;   // qk producer, MMA, softmax, v producer
+constexpr int kVWarp = 2 + kSoftWarps;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -81,7 +87,7 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, p, pos, ksc, qref, bars, misc, total;
+  uint32_t qk, v, p, pos, ksc, qref, xch, bars, misc, total;
 };
 
 template <int C, int D>
@@ -95,24 +101,13 @@ __host__ __device__ inline Layout layout(int slots, int pbufs) {
   l.pos = off;  off += slots * kQ * 4;
   l.ksc = off;  off += slots * kQ * 4;
   l.qref = off; off += slots * kQ * 4;
-  l.bars = off; off += (6 * slots + 4 * 2 + 2 * 2 + 2) * 8;
+  l.xch = off;  off += (2 * 2 + 2 + 2) * kQ * 4;   // partial sums [2][2], maxima [2], redo sums [2]
+  l.bars = off; off += (4 * slots + 6 * 2 + 2 + 4 + 1) * 8;
   l.misc = off; off += 16;
   l.total = off;
   return l;
 }
 
-__device__ __forceinline__ void cp_async_16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
-               "r"(valid ? 16 : 0)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
@@ -143,6 +138,23 @@ struct Unit {
   int bh, r, s0, s1;
 };
 
+// Positions of sorted slots sl .. sl+3 (INT_MAX past the end of the segment).
+__device__ __forceinline__ void load_positions(const int32_t* perm, int sl, int L, int* pos) {
+  if (sl + 3 < L) {
+    const int4 v = *reinterpret_cast<const int4*>(perm + sl);
+    pos[0] = v.x; pos[1] = v.y; pos[2] = v.z; pos[3] = v.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pos[k] = sl + k < L ? perm[sl + k] : INT_MAX;
+  }
+}
+
+// Row of the [B*H*L, d] view that holds position `pos`; a row past the end
+// of the tensor for a missing position, which the gather fills with zeros.
+__device__ __forceinline__ int gather_row(int rowbase, int pos) {
+  return pos == INT_MAX ? INT_MAX : rowbase + pos;
+}
+
 __device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
   Unit x;
   const int strip = (int)(u % p.n_strips);
@@ -155,7 +167,9 @@ __device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
 }
 
 template <int C, int D>
-__global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
+               const Params p) {
   using K = Cfg<C, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -173,13 +187,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
   uint64_t* v_full = bars + NS;
   uint64_t* qk_empty = bars + 2 * NS;
   uint64_t* v_empty = bars + 3 * NS;
-  uint64_t* s_full = bars + 6 * NS;   // [2]
+  uint64_t* s_full = bars + 4 * NS;   // [2]
   uint64_t* s_free = s_full + 2;      // [2]
   uint64_t* o_full = s_free + 2;      // [2]
   uint64_t* o_free = o_full + 2;      // [2]
   uint64_t* p_full = o_free + 2;      // [2]
   uint64_t* p_empty = p_full + 2;     // [2]
-  uint64_t* done = p_empty + 2;       // [1]
+  uint64_t* xbar = p_empty + 2;       // [2] partial-sum exchange, all softmax warps
+  uint64_t* rbar = xbar + 2;          // [4] redo exchange, the two warps of a quadrant
+  uint64_t* done = rbar + 4;          // [1]
+  float* xl = reinterpret_cast<float*>(smem + Ly.xch);   // [2 buf][2 half][kQ]
+  float* xm = xl + 4 * kQ;                               // [2 half][kQ]
+  float* xl2 = xm + 2 * kQ;                              // [2 half][kQ]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
 
@@ -188,6 +207,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(&qk_full[s], 32);
       mbar_init(&v_full[s], 32);
+      // released by the MMA (keys used) and the softmax warps (metadata used)
       mbar_init(&qk_empty[s], 1 + kSoftWarps);
       mbar_init(&v_empty[s], 1);
     }
@@ -198,7 +218,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
       mbar_init(&o_free[b], kSoftWarps);
       mbar_init(&p_full[b], kSoftWarps);
       mbar_init(&p_empty[b], 1);
+      mbar_init(&xbar[b], kSoftWarps);
     }
+    for (int q = 0; q < 4; ++q) mbar_init(&rbar[q], 2);
     mbar_init(done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -214,67 +236,39 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
   const long long u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (warp == 0) {
-    // ================================================================ producer
-    constexpr int RPI = 32 / K::kCpr;        // rows per warp instruction
-    const int sub = lane / K::kCpr, kc = lane % K::kCpr;
+    // ================================================================ qk producer
+    // Lane l owns rows 4l .. 4l+3 of every block.
     long long li = 0;  // load index (blocks loaded so far)
     bool ok = true;
+    if (lane == 0) tma_prefetch_desc(&qmap);
     for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
       const Unit U = unit_of(p, u);
       const int32_t* perm = p.perm + ((size_t)U.bh * p.n_h + U.r) * p.L;
-      const __nv_bfloat16* qk = p.qk + (size_t)U.bh * p.L * D;
-      const __nv_bfloat16* vv = p.v + (size_t)U.bh * p.L * D;
       const float* invn = p.inv_norm + (size_t)U.bh * p.L;
+      const int rowbase = U.bh * p.L;
       for (int b = (U.s0 > 0 ? U.s0 - 1 : U.s0); b < U.s1; ++b, ++li) {
         const int slot = (int)(li % NS);
         const uint32_t ph = (uint32_t)((li / NS) & 1);
-        if (!mbar_wait(&qk_empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
         int pos[4];
+        load_positions(perm, b * kQ + 4 * lane, p.L, pos);
+        if (!mbar_wait(&qk_empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) mbar_expect_tx(&qk_full[slot], K::kTile);
+        __syncwarp();
+        uint8_t* dst = qk_s + (size_t)slot * K::kTile + lane * 512;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_gather4(dst + h * K::kHalf, &qmap, &qk_full[slot], h * 64,
+                      gather_row(rowbase, pos[0]), gather_row(rowbase, pos[1]),
+                      gather_row(rowbase, pos[2]), gather_row(rowbase, pos[3]));
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int row = lane + 32 * k;
-          const int sl = b * kQ + row;
-          const bool valid = sl < p.L;
-          const int ps = valid ? perm[sl] : INT_MAX;
-          pos[k] = ps;
-          const float in = valid ? invn[ps] : 0.f;
-          pos_s[slot * kQ + row] = ps;
+          const int row = 4 * lane + k;
+          const float in = pos[k] != INT_MAX ? invn[pos[k]] : 0.f;
+          pos_s[slot * kQ + row] = pos[k];
           ksc_s[slot * kQ + row] = in * p.ksc;
           qref_s[slot * kQ + row] = in > 0.f ? p.ksc / in : 0.f;
         }
-        const uint32_t qk_dst = smem_u32(qk_s + (size_t)slot * K::kTile);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          for (int it = 0; it < 32 / RPI; ++it) {
-            const int row = k * 32 + it * RPI + sub;
-            const int ps = __shfl_sync(0xffffffffu, pos[k], row & 31);
-            const bool valid = ps != INT_MAX;
-            const __nv_bfloat16* src = qk + (size_t)(valid ? ps : 0) * D + kc * 8;
-            const uint32_t dst = qk_dst + (kc / 8) * K::kHalf + sw128_offset(row, (kc % 8) * 8);
-            cp_async_16(dst, src, valid);
-          }
-        }
-        cp_async_commit();
-        if (!mbar_wait(&v_empty[slot], ph ^ 1, abort_flag)) { ok = false; cp_async_wait<0>(); break; }
-        const uint32_t v_dst = smem_u32(v_s + (size_t)slot * K::kTile);
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          for (int it = 0; it < 32 / RPI; ++it) {
-            const int row = k * 32 + it * RPI + sub;
-            const int ps = __shfl_sync(0xffffffffu, pos[k], row & 31);
-            const bool valid = ps != INT_MAX;
-            const __nv_bfloat16* src = vv + (size_t)(valid ? ps : 0) * D + kc * 8;
-            const uint32_t dst = v_dst + (kc / 8) * K::kHalf + sw128_offset(row, (kc % 8) * 8);
-            cp_async_16(dst, src, valid);
-          }
-        }
-        cp_async_commit();
-        cp_async_wait<1>();
-        fence_proxy_async_smem();
         mbar_arrive(&qk_full[slot]);
-        cp_async_wait<0>();
-        fence_proxy_async_smem();
-        mbar_arrive(&v_full[slot]);
       }
     }
     if (!ok) {
@@ -289,64 +283,82 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
       const uint32_t idesc_prev = idesc_bf16_f32(kQ, C);
       const uint32_t idesc_cur = idesc_bf16_f32(kQ, kQ);
       const uint32_t idesc_pv = idesc_bf16_f32_bmn(kQ, D);
+      // Block load index of step s of a unit whose first block has index `first`.
+      auto cur_index = [](const Unit& U, long long first, int s) {
+        return first + (s - U.s0) + (U.s0 > 0 ? 1 : 0);
+      };
+      // S(s) = Q K^T into the step's TMEM buffer.
+      auto issue_qk = [&](const Unit& U, long long first, int s, long long ts) -> bool {
+        const long long ci = cur_index(U, first, s), pi = ci - 1;
+        const bool has_prev = s > 0;
+        const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
+        const int buf = (int)(ts % K::kNbuf);
+        const uint32_t bph = (uint32_t)((ts / K::kNbuf) & 1);
+        if (!mbar_wait(&s_free[buf], bph ^ 1, abort_flag)) return false;
+        if (!mbar_wait(&qk_full[cs], (uint32_t)((ci / NS) & 1), abort_flag)) return false;
+        if (has_prev && s == U.s0 &&
+            !mbar_wait(&qk_full[ps], (uint32_t)((pi / NS) & 1), abort_flag))
+          return false;
+        tc_fence_after_sync();
+        const uint32_t s_tmem = tmem_base + buf * K::kBufCols;
+        const uint32_t qa = smem_u32(qk_s + (size_t)cs * K::kTile);
+        const uint32_t pa = smem_u32(qk_s + (size_t)ps * K::kTile) + (kQ - C) * 128;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t koff = (uint32_t)(kk >> 2) * K::kHalf + (uint32_t)(kk & 3) * 32;
+          const uint64_t a = sdesc_kmajor_sw128(qa + koff);
+          if (has_prev)
+            mma_bf16_ss(s_tmem, a, sdesc_kmajor_sw128(pa + koff), idesc_prev, kk > 0);
+          mma_bf16_ss(s_tmem + C, a, sdesc_kmajor_sw128(qa + koff), idesc_cur, kk > 0);
+        }
+        mma_commit(&s_full[buf]);
+        if (has_prev) mma_commit(&qk_empty[ps]);
+        if (s == U.s1 - 1) mma_commit(&qk_empty[cs]);
+        return true;
+      };
+      // O(s) = P(s) V once the softmax has written P(s).
+      auto issue_pv = [&](const Unit& U, long long first, int s, long long ts) -> bool {
+        const long long ci = cur_index(U, first, s), pi = ci - 1;
+        const bool has_prev = s > 0;
+        const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
+        const int buf = (int)(ts % K::kNbuf);
+        const uint32_t bph = (uint32_t)((ts / K::kNbuf) & 1);
+        const int pb = (int)(ts % NP);
+        if (!mbar_wait(&p_full[pb], (uint32_t)((ts / NP) & 1), abort_flag)) return false;
+        if (!mbar_wait(&o_free[buf], bph ^ 1, abort_flag)) return false;
+        if (!mbar_wait(&v_full[cs], (uint32_t)((ci / NS) & 1), abort_flag)) return false;
+        if (has_prev && s == U.s0 &&
+            !mbar_wait(&v_full[ps], (uint32_t)((pi / NS) & 1), abort_flag))
+          return false;
+        tc_fence_after_sync();
+        const uint32_t o_tmem = tmem_base + buf * K::kBufCols + K::kNk;
+        const uint32_t pbase = smem_u32(p_s + (size_t)pb * K::kPBytes);
+        const uint32_t vcur = smem_u32(v_s + (size_t)cs * K::kTile);
+        const uint32_t vprev = smem_u32(v_s + (size_t)ps * K::kTile) + (kQ - C) * 128;
+        bool acc = false;
+        for (int kk = has_prev ? 0 : C / 16; kk < K::kNk / 16; ++kk) {
+          const uint64_t a = sdesc_kmajor_sw128(pbase + (kk >> 2) * (kQ * 128) + (kk & 3) * 32);
+          const int key = kk * 16;  // key column of this k-step
+          const uint32_t vb = key < C ? vprev + key * 128 : vcur + (key - C) * 128;
+          mma_bf16_ss(o_tmem, a, sdesc_mnmajor_sw128(vb, K::kHalf, 1024), idesc_pv,
+                      acc ? 1u : 0u);
+          acc = true;
+        }
+        mma_commit(&o_full[buf]);
+        mma_commit(&p_empty[pb]);
+        if (has_prev) mma_commit(&v_empty[ps]);
+        if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
+        return true;
+      };
       for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
         const Unit U = unit_of(p, u);
-        const bool lookback0 = U.s0 > 0;
         const long long first = li;
-        li += (U.s1 - U.s0) + (lookback0 ? 1 : 0);
+        li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
+        // S of the next step is computed while the softmax works on this one.
+        if (!issue_qk(U, first, U.s0, t)) { ok = false; break; }
+        issued = true;
         for (int s = U.s0; s < U.s1; ++s, ++t) {
-          const long long ci = first + (s - U.s0) + (lookback0 ? 1 : 0);  // current block
-          const long long pi = ci - 1;                                    // look-back block
-          const bool has_prev = s > 0;
-          const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
-          const uint32_t cph = (uint32_t)((ci / NS) & 1), pph = (uint32_t)((pi / NS) & 1);
-          const int buf = (int)(t % K::kNbuf);
-          const uint32_t bph = (uint32_t)((t / K::kNbuf) & 1);
-          const int pb = (int)(t % NP);
-          const uint32_t pbph = (uint32_t)((t / NP) & 1);
-          const uint32_t s_tmem = tmem_base + buf * K::kBufCols;
-          const uint32_t o_tmem = s_tmem + K::kNk;
-          // ---- S = Q K^T
-          if (!mbar_wait(&s_free[buf], bph ^ 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&qk_full[cs], cph, abort_flag)) { ok = false; break; }
-          if (has_prev && s == U.s0 && !mbar_wait(&qk_full[ps], pph, abort_flag)) { ok = false; break; }
-          tc_fence_after_sync();
-          const uint32_t qa = smem_u32(qk_s + (size_t)cs * K::kTile);
-          const uint32_t pa = smem_u32(qk_s + (size_t)ps * K::kTile) + (kQ - C) * 128;
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t koff = (uint32_t)(kk >> 2) * K::kHalf + (uint32_t)(kk & 3) * 32;
-            const uint64_t a = sdesc_kmajor_sw128(qa + koff);
-            if (has_prev)
-              mma_bf16_ss(s_tmem, a, sdesc_kmajor_sw128(pa + koff), idesc_prev, kk > 0);
-            mma_bf16_ss(s_tmem + C, a, sdesc_kmajor_sw128(qa + koff), idesc_cur, kk > 0);
-          }
-          issued = true;
-          mma_commit(&s_full[buf]);
-          if (has_prev) mma_commit(&qk_empty[ps]);
-          if (s == U.s1 - 1) mma_commit(&qk_empty[cs]);
-          // ---- O = P V
-          if (!mbar_wait(&p_full[pb], pbph, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&o_free[buf], bph ^ 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&v_full[cs], cph, abort_flag)) { ok = false; break; }
-          if (has_prev && s == U.s0 && !mbar_wait(&v_full[ps], pph, abort_flag)) { ok = false; break; }
-          tc_fence_after_sync();
-          const uint32_t pbase = smem_u32(p_s + (size_t)pb * K::kPBytes);
-          const uint32_t vcur = smem_u32(v_s + (size_t)cs * K::kTile);
-          const uint32_t vprev = smem_u32(v_s + (size_t)ps * K::kTile) + (kQ - C) * 128;
-          bool acc = false;
-          for (int kk = has_prev ? 0 : C / 16; kk < K::kNk / 16; ++kk) {
-            const uint64_t a =
-                sdesc_kmajor_sw128(pbase + (kk >> 2) * (kQ * 128) + (kk & 3) * 32);
-            const int key = kk * 16;  // key column of this k-step
-            const uint32_t vb = key < C ? vprev + key * 128 : vcur + (key - C) * 128;
-            const uint64_t b = sdesc_mnmajor_sw128(vb, K::kHalf, 1024);
-            mma_bf16_ss(o_tmem, a, b, idesc_pv, acc ? 1u : 0u);
-            acc = true;
-          }
-          mma_commit(&o_full[buf]);
-          mma_commit(&p_empty[pb]);
-          if (has_prev) mma_commit(&v_empty[ps]);
-          if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
+          if (s + 1 < U.s1 && !issue_qk(U, first, s + 1, t + 1)) { ok = false; break; }
+          if (!issue_pv(U, first, s, t)) { ok = false; break; }
         }
       }
       if (!ok) {
@@ -361,15 +373,48 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
         }
       }
     }
+  } else if (warp == kVWarp) {
+    // ================================================================ v producer
+    long long li = 0;
+    bool ok = true;
+    if (lane == 0) tma_prefetch_desc(&vmap);
+    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
+      const Unit U = unit_of(p, u);
+      const int32_t* perm = p.perm + ((size_t)U.bh * p.n_h + U.r) * p.L;
+      const int rowbase = U.bh * p.L;
+      for (int b = (U.s0 > 0 ? U.s0 - 1 : U.s0); b < U.s1; ++b, ++li) {
+        const int slot = (int)(li % NS);
+        const uint32_t ph = (uint32_t)((li / NS) & 1);
+        int pos[4];
+        load_positions(perm, b * kQ + 4 * lane, p.L, pos);
+        if (!mbar_wait(&v_empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
+        if (lane == 0) mbar_expect_tx(&v_full[slot], K::kTile);
+        __syncwarp();
+        uint8_t* dst = v_s + (size_t)slot * K::kTile + lane * 512;
+#pragma unroll
+        for (int h = 0; h < D / 64; ++h)
+          tma_gather4(dst + h * K::kHalf, &vmap, &v_full[slot], h * 64,
+                      gather_row(rowbase, pos[0]), gather_row(rowbase, pos[1]),
+                      gather_row(rowbase, pos[2]), gather_row(rowbase, pos[3]));
+        mbar_arrive(&v_full[slot]);
+      }
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.err, kErrWaitProducer);
+      *abort_flag = 1;
+    }
   } else {
     // ================================================================ softmax
+    const int sw = warp - 2;
     const int quad = warp & 3;
+    const int half = sw >> 2;        // which alternate 32-key chunks this warp takes
     const int m = quad * 32 + lane;  // query row in the step
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     // window columns of this row: c = 64 -> [0,128) or [64,192); c = 128 -> [0,256)
     const int win_lo = (C == 64 && quad >= 2) ? 64 : 0;
     const int win_hi = (C == 64 && quad < 2) ? 128 : K::kNk;
     long long li = 0, t = 0;
+    uint32_t rph = 0;  // phase of this quadrant's redo barrier
     bool ok = true;
     for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
       const Unit U = unit_of(p, u);
@@ -402,39 +447,37 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
         const float qref = qref_s[cs * kQ + m];
         const int qlim = p.causal ? qpos : INT_MAX - 1;
         const int lo = has_prev ? win_lo : max(win_lo, C);
-        // Key metadata: column j < C is look-back row (128 - C + j) of block
-        // ps, column j >= C is row (j - C) of block cs.
-        auto kmeta = [&](int j, int& kp, float& ks) {
-          const int idx = j < C ? ps * kQ + (kQ - C) + j : cs * kQ + (j - C);
-          kp = pos_s[idx];
-          ks = ksc_s[idx];
-        };
+        // metadata row of key column j0 (a multiple of 32, all in one block)
+        auto kbase = [&](int j0) { return j0 < C ? ps * kQ + (kQ - C) + j0 : cs * kQ + (j0 - C); };
         if (!mbar_wait(&p_empty[pb], pbph ^ 1, abort_flag)) { ok = false; break; }
         uint8_t* prow = p_s + (size_t)pb * K::kPBytes;
         float l = 0.f;
         bool any = false;
-        for (int j0 = 0; j0 < K::kNk; j0 += 32) {
+        for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
           uint32_t pk[16];
           if (j0 >= lo && j0 < win_hi) {
             uint32_t sv[32];
             __syncwarp();
             tmem_ld_32x32b_x32(s_tmem + j0, sv);
             tmem_ld_wait(sv);
+            const int kb = kbase(j0);
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
-              float pr[2];
+            for (int e = 0; e < 32; e += 4) {
+              const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
+              const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
+              const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+              const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+              float pr[4];
 #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                int kp;
-                float ks;
-                kmeta(j0 + e + h, kp, ks);
-                const bool valid = kp <= qlim && kp != qpos;
+              for (int h = 0; h < 4; ++h) {
+                const bool valid = kpa[h] <= qlim && kpa[h] != qpos;
                 any |= valid;
-                const float x = fmaf(__uint_as_float(sv[e + h]), ks, -qref);
+                const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
                 pr[h] = valid ? ex2(x) : 0.f;
                 l += pr[h];
               }
               pk[e / 2] = pack_bf16(pr[0], pr[1]);
+              pk[e / 2 + 1] = pack_bf16(pr[2], pr[3]);
             }
           } else {
 #pragma unroll
@@ -448,50 +491,76 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
                 make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
           }
         }
-        // Underflow: redo the row with its exact maximum as the reference.
-        float ref2 = qref;
-        const bool redo = any && !(l >= kTinySum);
+        // The two warps of the quadrant add their partial sums (any key seen is
+        // carried as l >= 0, none as -1).
+        const int xb = (int)(t & 1);
+        xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xbar[xb]);
+        if (!mbar_wait(&xbar[xb], (uint32_t)((t >> 1) & 1), abort_flag)) { ok = false; break; }
+        const float lo_part = xl[(xb * 2 + (half ^ 1)) * kQ + m];
+        any = any || lo_part >= 0.f;
+        float lt = l + fmaxf(lo_part, 0.f);
+        float ref = qref;
+        // Underflow of every term: redo the row with its exact maximum.
+        const bool redo = any && !(lt >= kTinySum);
         if (__any_sync(0xffffffffu, redo)) {
           float mx = -INFINITY;
-          for (int j0 = lo & ~31; j0 < win_hi; j0 += 32) {
+          for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
+            if (j0 < lo || j0 >= win_hi) continue;
             uint32_t sv[32];
             __syncwarp();
             tmem_ld_32x32b_x32(s_tmem + j0, sv);
             tmem_ld_wait(sv);
+            const int kb = kbase(j0);
             for (int e = 0; e < 32; ++e) {
-              int kp;
-              float ks;
-              kmeta(j0 + e, kp, ks);
-              if (j0 + e >= lo && kp <= qlim && kp != qpos)
-                mx = fmaxf(mx, __uint_as_float(sv[e]) * ks);
+              const int kp = pos_s[kb + e];
+              if (kp <= qlim && kp != qpos)
+                mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
             }
           }
-          if (redo) { ref2 = mx; l = 0.f; }
-          for (int j0 = lo & ~31; j0 < win_hi; j0 += 32) {
+          xm[half * kQ + m] = mx;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&rbar[quad]);
+          if (!mbar_wait(&rbar[quad], rph, abort_flag)) { ok = false; break; }
+          rph ^= 1;
+          const float gmax = fmaxf(mx, xm[(half ^ 1) * kQ + m]);
+          float l2 = 0.f;
+          for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
+            if (j0 < lo || j0 >= win_hi) continue;
             uint32_t sv[32];
             __syncwarp();
             tmem_ld_32x32b_x32(s_tmem + j0, sv);
             tmem_ld_wait(sv);
-            if (redo) {
-              uint8_t* base = prow + (j0 / 64) * (kQ * 128);
-              for (int e = 0; e < 32; e += 8) {
-                uint32_t w[4];
-                for (int h = 0; h < 8; h += 2) {
-                  float pr[2];
-                  for (int g = 0; g < 2; ++g) {
-                    int kp;
-                    float ks;
-                    kmeta(j0 + e + h + g, kp, ks);
-                    const bool valid = j0 + e + h + g >= lo && kp <= qlim && kp != qpos;
-                    pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ks, -ref2)) : 0.f;
-                    l += pr[g];
-                  }
-                  w[h / 2] = pack_bf16(pr[0], pr[1]);
+            if (!redo) continue;
+            const int kb = kbase(j0);
+            uint8_t* base = prow + (j0 / 64) * (kQ * 128);
+            for (int e = 0; e < 32; e += 8) {
+              uint32_t w[4];
+              for (int h = 0; h < 8; h += 2) {
+                float pr[2];
+                for (int g = 0; g < 2; ++g) {
+                  const int kp = pos_s[kb + e + h + g];
+                  const bool valid = kp <= qlim && kp != qpos;
+                  pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ksc_s[kb + e + h + g],
+                                           -gmax))
+                                : 0.f;
+                  l2 += pr[g];
                 }
-                *reinterpret_cast<uint4*>(base + sw128_offset(m, (j0 % 64) + e)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                w[h / 2] = pack_bf16(pr[0], pr[1]);
               }
+              *reinterpret_cast<uint4*>(base + sw128_offset(m, (j0 % 64) + e)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
             }
+          }
+          xl2[half * kQ + m] = l2;
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&rbar[quad]);
+          if (!mbar_wait(&rbar[quad], rph, abort_flag)) { ok = false; break; }
+          rph ^= 1;
+          if (redo) {
+            lt = l2 + xl2[(half ^ 1) * kQ + m];
+            ref = gmax;
           }
         }
         tc_fence_before_sync();
@@ -500,14 +569,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
         if (lane == 0) {
           mbar_arrive(&s_free[buf]);
           mbar_arrive(&p_full[pb]);
+          // the look-back block's metadata is not needed again, nor this
+          // block's at the strip's last step (qpos and qref are in registers)
+          if (has_prev) mbar_arrive(&qk_empty[ps]);
+          if (s == U.s1 - 1) mbar_arrive(&qk_empty[cs]);
         }
-        // ---- O / l to the row's original position
+        // ---- O / l to the row's original position: this warp's half of the columns
         if (!mbar_wait(&o_full[buf], bph, abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
-        const float inv_l = any ? 1.f / l : 0.f;
+        const float inv_l = any ? 1.f / lt : 0.f;
         __nv_bfloat16* orow = o_out + (size_t)(q_valid ? qpos : 0) * D;
 #pragma unroll
-        for (int d0 = 0; d0 < D; d0 += 32) {
+        for (int d0 = half * (D / 2); d0 < (half + 1) * (D / 2); d0 += 32) {
           uint32_t ov[32];
           __syncwarp();
           tmem_ld_32x32b_x32(o_tmem + d0, ov);
@@ -536,15 +609,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
             }
           }
         }
-        if (q_valid)
-          lse_out[qpos] = any ? (redo ? ref2 * kLn2 : qref * kLn2) + logf(l) : kSelfScore;
+        if (q_valid && half == 0) lse_out[qpos] = any ? ref * kLn2 + logf(lt) : kSelfScore;
         tc_fence_before_sync();
         __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&o_free[buf]);
-          if (has_prev) mbar_arrive(&qk_empty[ps]);
-          if (s == U.s1 - 1) mbar_arrive(&qk_empty[cs]);
-        }
+        if (lane == 0) mbar_arrive(&o_free[buf]);
       }
     }
     if (!ok) {
@@ -552,7 +620,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_tc_kernel(const Params p) {
       *abort_flag = 1;
     }
   }
-
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -577,7 +644,8 @@ bool plan(const Problem& pr, int* slots, int* pbufs, size_t* smem) {
 }  // namespace
 
 bool attn_tc_supported(const Problem& p) {
-  return p.bf16 && (p.d == 64 || p.d == 128) && (p.c == 64 || p.c == 128);
+  return p.bf16 && (p.d == 64 || p.d == 128) && (p.c == 64 || p.c == 128) &&
+         (long long)p.BH() * p.L < (1LL << 31) - 1 && sm100::tensor_map_encoder() != nullptr;
 }
 
 template <int C, int D>
@@ -609,11 +677,28 @@ static cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v,
   p.n_strips = (p.steps + strip - 1) / strip;
   p.n_units = segs * p.n_strips;
   p.ksc = kLog2e / sqrtf((float)pr.d);
+  auto encode = tensor_map_encoder();
+  if (!encode) return cudaErrorNotSupported;
+  // [B*H*L, d] views of qk and v: boxes of one row of 64 elements (128 B),
+  // 128B swizzle, rows outside the tensor read as zeros.
+  CUtensorMap maps[2];
+  const void* bases[2] = {qk, v};
+  for (int k = 0; k < 2; ++k) {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pr.BH() * pr.L};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 1};
+    const cuuint32_t estr[2] = {1, 1};
+    if (encode(&maps[k], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(bases[k]), dims,
+               strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+        CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+  }
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<C, D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  attn_tc_kernel<C, D><<<grid, kThreads, smem, st>>>(p);
+  attn_tc_kernel<C, D><<<grid, kThreads, smem, st>>>(maps[0], maps[1], p);
   return cudaGetLastError();
 }
 

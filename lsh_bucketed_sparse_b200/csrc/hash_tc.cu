@@ -24,8 +24,6 @@
 // Argmax order: larger |p| first; among equal |p| the smaller index of
 // [xR; -xR] (p_j >= 0 gives index j, else n_b/2 + j), i.e. the lowest index
 // among maximal entries.
-#include <cudaTypedefs.h>
-
 #include <algorithm>
 #include <climits>
 #include <mutex>
@@ -354,20 +352,6 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
 }
 
 // ---------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static std::once_flag once;
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  std::call_once(once, [] {
-    void* ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000,
-                                         cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  });
-  return fn;
-}
-
 struct Plan {
   int gr, n_groups, G, piece_w, n_pieces, stages;
   size_t smem;
@@ -414,14 +398,14 @@ bool make_plan(const Problem& pr, Plan* out) {
 bool hash_tc_supported(const Problem& p) {
   Plan plan;
   return p.bf16 && (p.d == 64 || p.d == 128) && p.n_b >= 2 && make_plan(p, &plan) &&
-         encode_fn() != nullptr;
+         tensor_map_encoder() != nullptr;
 }
 
 cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, int16_t* buckets,
                            float* inv_norm, cudaStream_t st) {
   Plan plan;
   if (!make_plan(pr, &plan)) return cudaErrorNotSupported;
-  auto encode = encode_fn();
+  auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;

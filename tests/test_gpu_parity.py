@@ -166,6 +166,18 @@ def test_zero_rows_and_scaled_rows():
     assert g["inv_norm"][0, 0, 5] == 0
 
 
+@pytest.mark.parametrize("chunk,d", [(64, 64), (128, 128)])
+def test_large_norms_take_the_exact_max_path(chunk, d):
+    # qk x 256 (exact in bf16): ||q|| / sqrt(d) is far above every actual
+    # score, so exponents measured from that bound underflow and the kernel
+    # must redo those rows with their exact maximum.
+    wl = W.small(f"large-norm-{chunk}-{d}", heads=2, seq_len=1024, d_k=d, n_hashes=2,
+                 n_buckets=64, chunk_len=chunk, causal=True)
+    report, g = _full_check(wl, qk_override=lambda qk: qk * 256)
+    assert torch.isfinite(g["out"].float()).all()
+    print(wl.name, report)
+
+
 def test_deterministic():
     wl = W.small("det", heads=2, seq_len=1024, n_hashes=2, n_buckets=64)
     qk, v, rot = [t.to(DEV) if t is not None else None for t in W.make_inputs(wl)]
