@@ -4,26 +4,30 @@
 // section 5 "Shared query-key space"; Appendix A "Implementation" and
 // "Masking"), for bf16 inputs with d_k in {64, 128} and chunks of 64 or 128.
 //
-// A CTA walks a strip of consecutive 128-slot "steps" of one (b*h, round)
-// segment in sorted order.  Step s has the queries of sorted slots
+// A CTA walks strips of consecutive 128-slot "steps" of (b*h, round)
+// segments in sorted order.  Step s has the queries of sorted slots
 // [128 s, 128 s + 128) and the keys of slots [128 s - c, 128 s + 128): the
 // previous c slots (look-back, none for s = 0) and the queries themselves.
 // A query in chunk k sees key chunks k-1 and k; with c = 64 the first 64
 // query rows (chunk 2s) see key columns [0, 128) and the last 64 (chunk
-// 2s+1) see [64, 192); with c = 128 every row sees all 256 columns.
+// 2s+1) see [64, 192); with c = 128 every row sees all 256 columns.  The
+// 128 slots of a step form a "block"; block s is the query block of step s
+// and the look-back block of step s+1.
 //
-// Data flow per step (warp-specialised, 11 warps):
-//   warp 0      qk producer: reads perm for the next 128 slots and gathers
-//               their qk rows with TMA (tile::gather4, four rows per lane
-//               and instruction) into a ring of shared-memory blocks in the
-//               128B-swizzled operand layout, and stores each row's
-//               position, key scale (1/||x|| * log2 e / sqrt(d)) and query
-//               reference ||x|| * log2 e / sqrt(d);
-//   warp 10     v producer: the same gathers from v, so that keys never wait
-//               for values;
+// Warp roles (11 warps):
+//   warp 0      qk producer: per block, gathers the qk rows named by perm
+//               with TMA (tile::gather4, four rows per lane and instruction)
+//               into a ring of shared-memory tiles in the 128B-swizzled
+//               operand layout, and writes each row's position, key scale
+//               (1/||x|| * log2 e / sqrt(d)) and query reference
+//               (||x|| * log2 e / sqrt(d)) into a metadata ring.  Positions
+//               and norms are loaded two blocks ahead.
+//   warp 10     v producer: the same gathers from v into their own ring, so
+//               keys never wait for values.
 //   warp 1      MMA issuer (one thread): S = Q K^T into TMEM (two MMAs per
 //               k-step: look-back keys and current keys live in different
-//               blocks), then O = P V with P from shared memory;
+//               tiles), issued one step ahead; then O = P V with P from
+//               shared memory and V as an MN-major operand.
 //   warps 2..9  softmax: two warps per TMEM lane quadrant (32 query rows),
 //               each taking alternate 32-key chunks of the row, straight
 //               from TMEM.  Keys are unit-normalised, so q . k_hat / sqrt(d)
@@ -34,8 +38,12 @@
 //               Masks: window, causal (key position > query position), self
 //               (the key j == i is left out and a row with no other key
 //               outputs v_i with lse -1e5, the value the -1e5 self score
-//               gives).  Then O / l (each warp half of the columns) and lse
-//               go to the row's original position.
+//               gives).  The softmax of step s+1 runs before the output of
+//               step s, so P V overlaps it.  For the output the two warps of
+//               a quadrant split its 32 rows: each stages its 16 rows of
+//               O / l in a private shared-memory region and writes them to
+//               the rows' original positions with TMA (tile::scatter4, four
+//               full rows per instruction); lse goes out directly.
 #include <algorithm>
 #include <climits>
 
@@ -50,9 +58,10 @@ using namespace sm100;
 
 constexpr int kQ = 128;             // queries per step = rows per block = MMA M
 constexpr int kSoftWarps = 8;
-constexpr int kThreads = (3 + kSoftWarps) * 32;   // qk producer, MMA, softmax, v producer
 constexpr int kVWarp = 2 + kSoftWarps;
+constexpr int kThreads = (3 + kSoftWarps) * 32;   // qk producer, MMA, softmax, v producer
 constexpr int kSmemLimit = 227 * 1024;
+constexpr int kMetaSlots = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // A row whose sum of 2^(s' - ref) falls below this is redone with its exact max.
@@ -66,14 +75,12 @@ struct Cfg {
   static constexpr int kPBytes = kQ * kNk * 2;     // P (bf16) of one step
   static constexpr int kNbuf = (kNk + D) * 2 <= 512 ? 2 : 1;
   static constexpr int kBufCols = kNbuf == 2 ? 256 : 512;
-  static constexpr int kCpr = D / 8;               // 16-byte chunks per row
 };
 
 struct Params {
-  const __nv_bfloat16* qk;
-  const __nv_bfloat16* v;
-  const float* inv_norm;
   const int32_t* perm;
+  const float* inv_norm;
+  const __nv_bfloat16* v;
   __nv_bfloat16* o_rounds;
   float* lse_rounds;
   unsigned int* err;
@@ -82,36 +89,41 @@ struct Params {
   int strip;          // steps per unit
   int n_strips;
   long long n_units;
-  int slots, pbufs;   // ring depth, P buffers
+  int nq, nv, np;     // qk tiles, v tiles, P buffers
+  int stage_o;        // O leaves through a shared-memory tile and TMA scatter4
   float ksc;          // log2 e / sqrt(d)
 };
 
 struct Layout {
-  uint32_t qk, v, p, pos, ksc, qref, xch, bars, misc, total;
+  uint32_t qk, v, p, ost, pos, ksc, qref, xch, bars, misc, total;
 };
 
+__host__ __device__ inline uint32_t n_barriers(int nq, int nv) {
+  return 2 * nq + 2 * nv + 2 * kMetaSlots + 2 * 8 + 4 + 1;
+}
+
 template <int C, int D>
-__host__ __device__ inline Layout layout(int slots, int pbufs) {
+__host__ __device__ inline Layout layout(int nq, int nv, int np, int stage_o) {
   using K = Cfg<C, D>;
   Layout l;
   uint32_t off = 0;
-  l.qk = off;   off += slots * K::kTile;
-  l.v = off;    off += slots * K::kTile;
-  l.p = off;    off += pbufs * K::kPBytes;
-  l.pos = off;  off += slots * kQ * 4;
-  l.ksc = off;  off += slots * kQ * 4;
-  l.qref = off; off += slots * kQ * 4;
+  l.qk = off;   off += nq * K::kTile;
+  l.v = off;    off += nv * K::kTile;
+  l.p = off;    off += np * K::kPBytes;
+  l.ost = off;  off += stage_o ? K::kTile : 0;     // staged O: 16 rows per softmax warp
+  l.pos = off;  off += kMetaSlots * kQ * 4;
+  l.ksc = off;  off += kMetaSlots * kQ * 4;
+  l.qref = off; off += kMetaSlots * kQ * 4;
   l.xch = off;  off += (2 * 2 + 2 + 2) * kQ * 4;   // partial sums [2][2], maxima [2], redo sums [2]
-  l.bars = off; off += (4 * slots + 6 * 2 + 2 + 4 + 1) * 8;
+  l.bars = off; off += n_barriers(nq, nv) * 8;
   l.misc = off; off += 16;
   l.total = off;
   return l;
 }
 
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -134,26 +146,10 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
+// A strip of steps [s0, s1) of segment (bh, r).
 struct Unit {
   int bh, r, s0, s1;
 };
-
-// Positions of sorted slots sl .. sl+3 (INT_MAX past the end of the segment).
-__device__ __forceinline__ void load_positions(const int32_t* perm, int sl, int L, int* pos) {
-  if (sl + 3 < L) {
-    const int4 v = *reinterpret_cast<const int4*>(perm + sl);
-    pos[0] = v.x; pos[1] = v.y; pos[2] = v.z; pos[3] = v.w;
-  } else {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) pos[k] = sl + k < L ? perm[sl + k] : INT_MAX;
-  }
-}
-
-// Row of the [B*H*L, d] view that holds position `pos`; a row past the end
-// of the tensor for a missing position, which the gather fills with zeros.
-__device__ __forceinline__ int gather_row(int rowbase, int pos) {
-  return pos == INT_MAX ? INT_MAX : rowbase + pos;
-}
 
 __device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
   Unit x;
@@ -166,50 +162,118 @@ __device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
   return x;
 }
 
+// The CTA's sequence of blocks to load: for each of its units, the look-back
+// block (if s0 > 0) and then blocks s0 .. s1-1.
+struct Cursor {
+  long long u;
+  Unit U;
+  int b;
+  bool valid;
+};
+
+__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, long long u) {
+  c.u = u;
+  c.valid = u < p.n_units;
+  if (c.valid) {
+    c.U = unit_of(p, u);
+    c.b = c.U.s0 > 0 ? c.U.s0 - 1 : c.U.s0;
+  }
+}
+
+__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, long long u_step) {
+  if (!c.valid) return;
+  if (++c.b >= c.U.s1) cursor_start(c, p, c.u + u_step);
+}
+
+// Positions of sorted slots sl .. sl+3 of a segment (INT_MAX past its end).
+__device__ __forceinline__ void load_positions(const int32_t* perm, int sl, int L, int* pos) {
+  if (sl + 3 < L) {
+    const int4 v = *reinterpret_cast<const int4*>(perm + sl);
+    pos[0] = v.x; pos[1] = v.y; pos[2] = v.z; pos[3] = v.w;
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pos[k] = sl + k < L ? perm[sl + k] : INT_MAX;
+  }
+}
+
+// Positions of the 4 rows lane 4l .. 4l+3 owns in the cursor's block.
+__device__ __forceinline__ void cursor_positions(const Cursor& c, const Params& p, int lane,
+                                                 int* pos) {
+  if (!c.valid) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) pos[k] = INT_MAX;
+    return;
+  }
+  const int32_t* perm = p.perm + ((size_t)c.U.bh * p.n_h + c.U.r) * p.L;
+  load_positions(perm, c.b * kQ + 4 * lane, p.L, pos);
+}
+
+// Row of the [B*H*L, d] view that holds position `pos`; a row past the end
+// of the tensor for a missing position, which the gather fills with zeros.
+__device__ __forceinline__ int gather_row(int rowbase, int pos) {
+  return pos == INT_MAX ? INT_MAX : rowbase + pos;
+}
+
+// What the softmax keeps of a row between its P pass and its output.
+struct RowState {
+  int qpos;     // original position (INT_MAX: no such query)
+  bool any;     // some key other than itself was visible
+  float lt;     // sum of 2^(s' - ref) over the row
+  float ref;    // exponent reference, log2 units
+};
+
 template <int C, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
-               const Params p) {
+               const __grid_constant__ CUtensorMap omap, const Params p) {
   using K = Cfg<C, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const Layout Ly = layout<C, D>(p.slots, p.pbufs);
+  const int NQ = p.nq, NV = p.nv, NP = p.np, NM = kMetaSlots;
+  const Layout Ly = layout<C, D>(NQ, NV, NP, p.stage_o);
+  uint8_t* ost_s = smem + Ly.ost;
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
   uint8_t* p_s = smem + Ly.p;
   int* pos_s = reinterpret_cast<int*>(smem + Ly.pos);
   float* ksc_s = reinterpret_cast<float*>(smem + Ly.ksc);
   float* qref_s = reinterpret_cast<float*>(smem + Ly.qref);
+  float* xl = reinterpret_cast<float*>(smem + Ly.xch);  // [2 buf][2 half][kQ]
+  float* xm = xl + 4 * kQ;                              // [2 half][kQ]
+  float* xl2 = xm + 2 * kQ;                             // [2 half][kQ]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bars);
-  const int NS = p.slots, NP = p.pbufs;
-  uint64_t* qk_full = bars;
-  uint64_t* v_full = bars + NS;
-  uint64_t* qk_empty = bars + 2 * NS;
-  uint64_t* v_empty = bars + 3 * NS;
-  uint64_t* s_full = bars + 4 * NS;   // [2]
-  uint64_t* s_free = s_full + 2;      // [2]
-  uint64_t* o_full = s_free + 2;      // [2]
-  uint64_t* o_free = o_full + 2;      // [2]
-  uint64_t* p_full = o_free + 2;      // [2]
-  uint64_t* p_empty = p_full + 2;     // [2]
-  uint64_t* xbar = p_empty + 2;       // [2] partial-sum exchange, all softmax warps
-  uint64_t* rbar = xbar + 2;          // [4] redo exchange, the two warps of a quadrant
-  uint64_t* done = rbar + 4;          // [1]
-  float* xl = reinterpret_cast<float*>(smem + Ly.xch);   // [2 buf][2 half][kQ]
-  float* xm = xl + 4 * kQ;                               // [2 half][kQ]
-  float* xl2 = xm + 2 * kQ;                              // [2 half][kQ]
+  uint64_t* qk_full = bars;              // [NQ] TMA bytes + 32 producer lanes
+  uint64_t* qk_empty = qk_full + NQ;     // [NQ] MMA: keys consumed
+  uint64_t* v_full = qk_empty + NQ;      // [NV] TMA bytes + 32 producer lanes
+  uint64_t* v_empty = v_full + NV;       // [NV] MMA: values consumed
+  uint64_t* m_full = v_empty + NV;       // [NM] metadata written (32 lanes)
+  uint64_t* m_empty = m_full + NM;       // [NM] metadata consumed (softmax warps)
+  uint64_t* s_full = m_empty + NM;       // [2] S in TMEM
+  uint64_t* s_free = s_full + 2;         // [2] S read
+  uint64_t* o_full = s_free + 2;         // [2] O in TMEM
+  uint64_t* o_free = o_full + 2;         // [2] O read
+  uint64_t* p_full = o_free + 2;         // [2] P written
+  uint64_t* p_empty = p_full + 2;        // [2] P consumed
+  uint64_t* xbar = p_empty + 2;          // [2] partial-sum exchange, all softmax warps
+  uint64_t* rbar = xbar + 2;             // [4] redo exchange, the two warps of a quadrant
+  uint64_t* done = rbar + 4;             // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NQ; ++s) {
       mbar_init(&qk_full[s], 32);
+      mbar_init(&qk_empty[s], 1);
+    }
+    for (int s = 0; s < NV; ++s) {
       mbar_init(&v_full[s], 32);
-      // released by the MMA (keys used) and the softmax warps (metadata used)
-      mbar_init(&qk_empty[s], 1 + kSoftWarps);
       mbar_init(&v_empty[s], 1);
+    }
+    for (int s = 0; s < NM; ++s) {
+      mbar_init(&m_full[s], 32);
+      mbar_init(&m_empty[s], kSoftWarps);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
@@ -237,39 +301,98 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
   if (warp == 0) {
     // ================================================================ qk producer
-    // Lane l owns rows 4l .. 4l+3 of every block.
-    long long li = 0;  // load index (blocks loaded so far)
-    bool ok = true;
+    // Lane l owns rows 4l .. 4l+3 of every block.  Positions are loaded two
+    // blocks ahead and norms one block ahead, so neither waits in line.
     if (lane == 0) tma_prefetch_desc(&qmap);
-    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
-      const Unit U = unit_of(p, u);
-      const int32_t* perm = p.perm + ((size_t)U.bh * p.n_h + U.r) * p.L;
-      const float* invn = p.inv_norm + (size_t)U.bh * p.L;
-      const int rowbase = U.bh * p.L;
-      for (int b = (U.s0 > 0 ? U.s0 - 1 : U.s0); b < U.s1; ++b, ++li) {
-        const int slot = (int)(li % NS);
-        const uint32_t ph = (uint32_t)((li / NS) & 1);
-        int pos[4];
-        load_positions(perm, b * kQ + 4 * lane, p.L, pos);
-        if (!mbar_wait(&qk_empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) mbar_expect_tx(&qk_full[slot], K::kTile);
-        __syncwarp();
-        uint8_t* dst = qk_s + (size_t)slot * K::kTile + lane * 512;
+    Cursor c0, c1, c2;
+    cursor_start(c0, p, u_begin);
+    c1 = c0;
+    cursor_next(c1, p, u_step);
+    c2 = c1;
+    cursor_next(c2, p, u_step);
+    int pos0[4], pos1[4];
+    float in0[4];
+    cursor_positions(c0, p, lane, pos0);
+    cursor_positions(c1, p, lane, pos1);
 #pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_gather4(dst + h * K::kHalf, &qmap, &qk_full[slot], h * 64,
-                      gather_row(rowbase, pos[0]), gather_row(rowbase, pos[1]),
-                      gather_row(rowbase, pos[2]), gather_row(rowbase, pos[3]));
+    for (int k = 0; k < 4; ++k)
+      in0[k] = pos0[k] != INT_MAX ? p.inv_norm[(size_t)c0.U.bh * p.L + pos0[k]] : 0.f;
+    long long li = 0;
+    bool ok = true;
+    for (; ok && c0.valid; ++li) {
+      // prefetch for the next two blocks
+      int pos2[4];
+      float in1[4];
+      cursor_positions(c2, p, lane, pos2);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int row = 4 * lane + k;
-          const float in = pos[k] != INT_MAX ? invn[pos[k]] : 0.f;
-          pos_s[slot * kQ + row] = pos[k];
-          ksc_s[slot * kQ + row] = in * p.ksc;
-          qref_s[slot * kQ + row] = in > 0.f ? p.ksc / in : 0.f;
-        }
-        mbar_arrive(&qk_full[slot]);
+      for (int k = 0; k < 4; ++k)
+        in1[k] = (c1.valid && pos1[k] != INT_MAX)
+                     ? p.inv_norm[(size_t)c1.U.bh * p.L + pos1[k]] : 0.f;
+      const int qs = (int)(li % NQ), ms = (int)(li % NM);
+      if (!mbar_wait(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (lane == 0) mbar_expect_tx(&qk_full[qs], K::kTile);
+      __syncwarp();
+      const int rowbase = c0.U.bh * p.L;
+      uint8_t* dst = qk_s + (size_t)qs * K::kTile + lane * 512;
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_gather4(dst + h * K::kHalf, &qmap, &qk_full[qs], h * 64, gather_row(rowbase, pos0[0]),
+                    gather_row(rowbase, pos0[1]), gather_row(rowbase, pos0[2]),
+                    gather_row(rowbase, pos0[3]));
+      mbar_arrive(&qk_full[qs]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int row = ms * kQ + 4 * lane + k;
+        pos_s[row] = pos0[k];
+        ksc_s[row] = in0[k] * p.ksc;
+        qref_s[row] = in0[k] > 0.f ? p.ksc / in0[k] : 0.f;
       }
+      mbar_arrive(&m_full[ms]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        pos0[k] = pos1[k];
+        pos1[k] = pos2[k];
+        in0[k] = in1[k];
+      }
+      c0 = c1;
+      c1 = c2;
+      cursor_next(c2, p, u_step);
+    }
+    if (!ok) {
+      if (lane == 0) atomicOr(p.err, kErrWaitProducer);
+      *abort_flag = 1;
+    }
+  } else if (warp == kVWarp) {
+    // ================================================================ v producer
+    if (lane == 0) tma_prefetch_desc(&vmap);
+    Cursor c0, c1;
+    cursor_start(c0, p, u_begin);
+    c1 = c0;
+    cursor_next(c1, p, u_step);
+    int pos0[4];
+    cursor_positions(c0, p, lane, pos0);
+    long long li = 0;
+    bool ok = true;
+    for (; ok && c0.valid; ++li) {
+      int pos1[4];
+      cursor_positions(c1, p, lane, pos1);
+      const int vs = (int)(li % NV);
+      if (!mbar_wait(&v_empty[vs], (uint32_t)(((li / NV) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (lane == 0) mbar_expect_tx(&v_full[vs], K::kTile);
+      __syncwarp();
+      const int rowbase = c0.U.bh * p.L;
+      uint8_t* dst = v_s + (size_t)vs * K::kTile + lane * 512;
+#pragma unroll
+      for (int h = 0; h < D / 64; ++h)
+        tma_gather4(dst + h * K::kHalf, &vmap, &v_full[vs], h * 64, gather_row(rowbase, pos0[0]),
+                    gather_row(rowbase, pos0[1]), gather_row(rowbase, pos0[2]),
+                    gather_row(rowbase, pos0[3]));
+      mbar_arrive(&v_full[vs]);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) pos0[k] = pos1[k];
+      c0 = c1;
+      cursor_next(c1, p, u_step);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitProducer);
@@ -283,21 +406,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const uint32_t idesc_prev = idesc_bf16_f32(kQ, C);
       const uint32_t idesc_cur = idesc_bf16_f32(kQ, kQ);
       const uint32_t idesc_pv = idesc_bf16_f32_bmn(kQ, D);
-      // Block load index of step s of a unit whose first block has index `first`.
-      auto cur_index = [](const Unit& U, long long first, int s) {
-        return first + (s - U.s0) + (U.s0 > 0 ? 1 : 0);
-      };
-      // S(s) = Q K^T into the step's TMEM buffer.
+      // S(s) = Q K^T into the step's TMEM buffer (ts = the step's counter).
       auto issue_qk = [&](const Unit& U, long long first, int s, long long ts) -> bool {
-        const long long ci = cur_index(U, first, s), pi = ci - 1;
+        const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
         const bool has_prev = s > 0;
-        const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
+        const int cs = (int)(ci % NQ), ps = (int)(((pi % NQ) + NQ) % NQ);
         const int buf = (int)(ts % K::kNbuf);
-        const uint32_t bph = (uint32_t)((ts / K::kNbuf) & 1);
-        if (!mbar_wait(&s_free[buf], bph ^ 1, abort_flag)) return false;
-        if (!mbar_wait(&qk_full[cs], (uint32_t)((ci / NS) & 1), abort_flag)) return false;
+        if (!mbar_wait(&s_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
+          return false;
+        if (!mbar_wait(&qk_full[cs], (uint32_t)((ci / NQ) & 1), abort_flag)) return false;
         if (has_prev && s == U.s0 &&
-            !mbar_wait(&qk_full[ps], (uint32_t)((pi / NS) & 1), abort_flag))
+            !mbar_wait(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t s_tmem = tmem_base + buf * K::kBufCols;
@@ -317,17 +436,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       };
       // O(s) = P(s) V once the softmax has written P(s).
       auto issue_pv = [&](const Unit& U, long long first, int s, long long ts) -> bool {
-        const long long ci = cur_index(U, first, s), pi = ci - 1;
+        const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
         const bool has_prev = s > 0;
-        const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
+        const int cs = (int)(ci % NV), ps = (int)(((pi % NV) + NV) % NV);
         const int buf = (int)(ts % K::kNbuf);
-        const uint32_t bph = (uint32_t)((ts / K::kNbuf) & 1);
         const int pb = (int)(ts % NP);
         if (!mbar_wait(&p_full[pb], (uint32_t)((ts / NP) & 1), abort_flag)) return false;
-        if (!mbar_wait(&o_free[buf], bph ^ 1, abort_flag)) return false;
-        if (!mbar_wait(&v_full[cs], (uint32_t)((ci / NS) & 1), abort_flag)) return false;
+        if (!mbar_wait(&o_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
+          return false;
+        if (!mbar_wait(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
         if (has_prev && s == U.s0 &&
-            !mbar_wait(&v_full[ps], (uint32_t)((pi / NS) & 1), abort_flag))
+            !mbar_wait(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_base + buf * K::kBufCols + K::kNk;
@@ -373,36 +492,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         }
       }
     }
-  } else if (warp == kVWarp) {
-    // ================================================================ v producer
-    long long li = 0;
-    bool ok = true;
-    if (lane == 0) tma_prefetch_desc(&vmap);
-    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
-      const Unit U = unit_of(p, u);
-      const int32_t* perm = p.perm + ((size_t)U.bh * p.n_h + U.r) * p.L;
-      const int rowbase = U.bh * p.L;
-      for (int b = (U.s0 > 0 ? U.s0 - 1 : U.s0); b < U.s1; ++b, ++li) {
-        const int slot = (int)(li % NS);
-        const uint32_t ph = (uint32_t)((li / NS) & 1);
-        int pos[4];
-        load_positions(perm, b * kQ + 4 * lane, p.L, pos);
-        if (!mbar_wait(&v_empty[slot], ph ^ 1, abort_flag)) { ok = false; break; }
-        if (lane == 0) mbar_expect_tx(&v_full[slot], K::kTile);
-        __syncwarp();
-        uint8_t* dst = v_s + (size_t)slot * K::kTile + lane * 512;
-#pragma unroll
-        for (int h = 0; h < D / 64; ++h)
-          tma_gather4(dst + h * K::kHalf, &vmap, &v_full[slot], h * 64,
-                      gather_row(rowbase, pos[0]), gather_row(rowbase, pos[1]),
-                      gather_row(rowbase, pos[2]), gather_row(rowbase, pos[3]));
-        mbar_arrive(&v_full[slot]);
-      }
-    }
-    if (!ok) {
-      if (lane == 0) atomicOr(p.err, kErrWaitProducer);
-      *abort_flag = 1;
-    }
   } else {
     // ================================================================ softmax
     const int sw = warp - 2;
@@ -413,251 +502,304 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     // window columns of this row: c = 64 -> [0,128) or [64,192); c = 128 -> [0,256)
     const int win_lo = (C == 64 && quad >= 2) ? 64 : 0;
     const int win_hi = (C == 64 && quad < 2) ? 128 : K::kNk;
-    long long li = 0, t = 0;
     uint32_t rph = 0;  // phase of this quadrant's redo barrier
     bool ok = true;
-    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
-      const Unit U = unit_of(p, u);
-      const bool lookback0 = U.s0 > 0;
-      const long long first = li;
-      li += (U.s1 - U.s0) + (lookback0 ? 1 : 0);
-      __nv_bfloat16* o_out = p.o_rounds + ((size_t)U.bh * p.n_h + U.r) * p.L * D;
-      float* lse_out = p.lse_rounds + ((size_t)U.bh * p.n_h + U.r) * p.L;
-      const __nv_bfloat16* vsrc = p.v + (size_t)U.bh * p.L * D;
-      for (int s = U.s0; s < U.s1; ++s, ++t) {
-        const long long ci = first + (s - U.s0) + (lookback0 ? 1 : 0);
-        const long long pi = ci - 1;
-        const bool has_prev = s > 0;
-        const int cs = (int)(ci % NS), ps = (int)(((pi % NS) + NS) % NS);
-        const uint32_t cph = (uint32_t)((ci / NS) & 1);
-        const int buf = (int)(t % K::kNbuf);
-        const uint32_t bph = (uint32_t)((t / K::kNbuf) & 1);
-        const int pb = (int)(t % NP);
-        const uint32_t pbph = (uint32_t)((t / NP) & 1);
-        const uint32_t s_tmem = tmem_base + lane_off + buf * K::kBufCols;
-        const uint32_t o_tmem = s_tmem + K::kNk;
-        // Metadata of this step's blocks is published with qk_full.
-        if (!mbar_wait(&qk_full[cs], cph, abort_flag)) { ok = false; break; }
-        if (has_prev && s == U.s0 &&
-            !mbar_wait(&qk_full[ps], (uint32_t)((pi / NS) & 1), abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&s_full[buf], bph, abort_flag)) { ok = false; break; }
-        tc_fence_after_sync();
-        const int qpos = pos_s[cs * kQ + m];
-        const bool q_valid = qpos != INT_MAX;
-        const float qref = qref_s[cs * kQ + m];
-        const int qlim = p.causal ? qpos : INT_MAX - 1;
-        const int lo = has_prev ? win_lo : max(win_lo, C);
-        // metadata row of key column j0 (a multiple of 32, all in one block)
-        auto kbase = [&](int j0) { return j0 < C ? ps * kQ + (kQ - C) + j0 : cs * kQ + (j0 - C); };
-        if (!mbar_wait(&p_empty[pb], pbph ^ 1, abort_flag)) { ok = false; break; }
-        uint8_t* prow = p_s + (size_t)pb * K::kPBytes;
-        float l = 0.f;
-        bool any = false;
-        for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
-          uint32_t pk[16];
-          if (j0 >= lo && j0 < win_hi) {
-            uint32_t sv[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(s_tmem + j0, sv);
-            tmem_ld_wait(sv);
-            const int kb = kbase(j0);
+
+    // P pass of step s (step counter ts): S from TMEM -> P (bf16) in shared
+    // memory; returns the row's state for its output.
+    auto p_pass = [&](const Unit& U, long long first, int s, long long ts, RowState& st) -> bool {
+      const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
+      const bool has_prev = s > 0;
+      const int cs = (int)(ci % NM), ps = (int)(((pi % NM) + NM) % NM);
+      const int buf = (int)(ts % K::kNbuf);
+      const int pb = (int)(ts % NP);
+      const uint32_t s_tmem = tmem_base + lane_off + buf * K::kBufCols;
+      if (!mbar_wait(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
+      if (has_prev && s == U.s0 &&
+          !mbar_wait(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
+        return false;
+      if (!mbar_wait(&s_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
+      tc_fence_after_sync();
+      const int qpos = pos_s[cs * kQ + m];
+      const float qref = qref_s[cs * kQ + m];
+      const int qlim = p.causal ? qpos : INT_MAX - 1;
+      const int lo = has_prev ? win_lo : max(win_lo, C);
+      // metadata row of key column j0 (a multiple of 32, all in one block)
+      auto kbase = [&](int j0) { return j0 < C ? ps * kQ + (kQ - C) + j0 : cs * kQ + (j0 - C); };
+      if (!mbar_wait(&p_empty[pb], (uint32_t)(((ts / NP) & 1) ^ 1), abort_flag)) return false;
+      uint8_t* prow = p_s + (size_t)pb * K::kPBytes;
+      bool any = false;
+      float la[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
+        uint32_t pk[16];
+        if (j0 >= lo && j0 < win_hi) {
+          uint32_t sv[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(s_tmem + j0, sv);
+          tmem_ld_wait(sv);
+          const int kb = kbase(j0);
 #pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
-              const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
-              const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
-              const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
-              float pr[4];
+          for (int e = 0; e < 32; e += 4) {
+            const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
+            const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
+            const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+            const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+            float pr[4];
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const bool valid = kpa[h] <= qlim && kpa[h] != qpos;
-                any |= valid;
-                const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
-                pr[h] = valid ? ex2(x) : 0.f;
-                l += pr[h];
-              }
-              pk[e / 2] = pack_bf16(pr[0], pr[1]);
-              pk[e / 2 + 1] = pack_bf16(pr[2], pr[3]);
+            for (int h = 0; h < 4; ++h) {
+              const bool valid = kpa[h] <= qlim && kpa[h] != qpos;
+              any |= valid;
+              const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
+              pr[h] = valid ? ex2(x) : 0.f;
+              la[h] += pr[h];
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            pk[e / 2] = pack_bf16(pr[0], pr[1]);
+            pk[e / 2 + 1] = pack_bf16(pr[2], pr[3]);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
+        }
+        uint8_t* base = prow + (j0 / 64) * (kQ * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k = (j0 % 64) + q * 8;
+          *reinterpret_cast<uint4*>(base + sw128_offset(m, k)) =
+              make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+      }
+      const float l = (la[0] + la[1]) + (la[2] + la[3]);
+      // The two warps of the quadrant add their partial sums (a row that saw
+      // no key is carried as -1).
+      const int xb = (int)(ts & 1);
+      xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&xbar[xb]);
+      if (!mbar_wait(&xbar[xb], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
+      const float other = xl[(xb * 2 + (half ^ 1)) * kQ + m];
+      any = any || other >= 0.f;
+      float lt = l + fmaxf(other, 0.f);
+      float ref = qref;
+      // Every term underflowed against the bound: redo the row against its
+      // exact maximum.
+      const bool need = any && !(lt >= kTinySum);
+      if (__any_sync(0xffffffffu, need)) {
+        float mx = -INFINITY;
+        for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
+          if (j0 < lo || j0 >= win_hi) continue;
+          uint32_t sv[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(s_tmem + j0, sv);
+          tmem_ld_wait(sv);
+          const int kb = kbase(j0);
+          for (int e = 0; e < 32; ++e) {
+            const int kp = pos_s[kb + e];
+            if (kp <= qlim && kp != qpos) mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
+          }
+        }
+        xm[half * kQ + m] = mx;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rbar[quad]);
+        if (!mbar_wait(&rbar[quad], rph, abort_flag)) return false;
+        rph ^= 1;
+        const float gmax = fmaxf(mx, xm[(half ^ 1) * kQ + m]);
+        const bool redo = need;
+        float l2 = 0.f;
+        for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
+          if (j0 < lo || j0 >= win_hi) continue;
+          uint32_t sv[32];
+          __syncwarp();
+          tmem_ld_32x32b_x32(s_tmem + j0, sv);
+          tmem_ld_wait(sv);
+          if (!redo) continue;
+          const int kb = kbase(j0);
           uint8_t* base = prow + (j0 / 64) * (kQ * 128);
+          for (int e = 0; e < 32; e += 8) {
+            uint32_t w[4];
+            for (int h = 0; h < 8; h += 2) {
+              float pr[2];
+              for (int g = 0; g < 2; ++g) {
+                const int kp = pos_s[kb + e + h + g];
+                const bool valid = kp <= qlim && kp != qpos;
+                pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ksc_s[kb + e + h + g],
+                                         -gmax))
+                              : 0.f;
+                l2 += pr[g];
+              }
+              w[h / 2] = pack_bf16(pr[0], pr[1]);
+            }
+            *reinterpret_cast<uint4*>(base + sw128_offset(m, (j0 % 64) + e)) =
+                make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        xl2[half * kQ + m] = l2;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&rbar[quad]);
+        if (!mbar_wait(&rbar[quad], rph, abort_flag)) return false;
+        rph ^= 1;
+        if (redo) {
+          lt = l2 + xl2[(half ^ 1) * kQ + m];
+          ref = gmax;
+        }
+      }
+      tc_fence_before_sync();
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&s_free[buf]);
+        mbar_arrive(&p_full[pb]);
+        // metadata of the look-back block is not needed again, nor this
+        // block's at the strip's last step (the row's state is in registers)
+        if (has_prev) mbar_arrive(&m_empty[ps]);
+        if (s == U.s1 - 1) mbar_arrive(&m_empty[cs]);
+      }
+      st.qpos = qpos;
+      st.any = any;
+      st.lt = lt;
+      st.ref = ref;
+      return true;
+    };
+
+    // Output of step s: this warp takes rows lane 16*half .. 16*half+15 of
+    // its quadrant, all D columns: O / l and lse.  When every query of the
+    // step exists and there is room, the rows are staged in this warp's own
+    // 16-row region (128B-swizzled, like the operand tiles) and lane 0
+    // writes them with TMA scatter4; otherwise each lane stores its row.
+    const bool mine = (lane >> 4) == half;
+    uint8_t* my_ost = ost_s + (size_t)sw * (16 * D * 2);
+    bool st_pending = false;  // lane 0: a scatter from my_ost may still be reading it
+    auto o_pass = [&](const Unit& U, long long ts, int s, const RowState& st) -> bool {
+      const int buf = (int)(ts % K::kNbuf);
+      const uint32_t o_tmem = tmem_base + lane_off + buf * K::kBufCols + K::kNk;
+      const bool stage = p.stage_o && (s + 1) * kQ <= p.L;  // every query of the step exists
+      if (!mbar_wait(&o_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
+      tc_fence_after_sync();
+      if (stage && lane == 0 && st_pending) bulk_wait_read_all();
+      __syncwarp();
+      const bool q_valid = st.qpos != INT_MAX;
+      const size_t seg_row = ((size_t)U.bh * p.n_h + U.r) * p.L;
+      const float inv_l = st.any ? 1.f / st.lt : 0.f;
+      __nv_bfloat16* orow = p.o_rounds + (seg_row + (q_valid ? st.qpos : 0)) * D;
+      const __nv_bfloat16* vrow = p.v + ((size_t)U.bh * p.L + (q_valid ? st.qpos : 0)) * D;
+      const int r16 = lane & 15;
+#pragma unroll
+      for (int d0 = 0; d0 < D; d0 += 32) {
+        uint32_t ov[32];
+        __syncwarp();
+        tmem_ld_32x32b_x32(o_tmem + d0, ov);
+        tmem_ld_wait(ov);
+        if (!mine || !q_valid) continue;
+        uint4 w[4];
+        if (st.any) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int k = (j0 % 64) + q * 8;
-            *reinterpret_cast<uint4*>(base + sw128_offset(m, k)) =
-                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+            w[q].x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv_l,
+                               __uint_as_float(ov[8 * q + 1]) * inv_l);
+            w[q].y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv_l,
+                               __uint_as_float(ov[8 * q + 3]) * inv_l);
+            w[q].z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv_l,
+                               __uint_as_float(ov[8 * q + 5]) * inv_l);
+            w[q].w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv_l,
+                               __uint_as_float(ov[8 * q + 7]) * inv_l);
           }
+        } else {
+          // nothing but itself to attend to: the -1e5 self score makes it v_i
+#pragma unroll
+          for (int q = 0; q < 4; ++q) w[q] = reinterpret_cast<const uint4*>(vrow + d0)[q];
         }
-        // The two warps of the quadrant add their partial sums (any key seen is
-        // carried as l >= 0, none as -1).
-        const int xb = (int)(t & 1);
-        xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&xbar[xb]);
-        if (!mbar_wait(&xbar[xb], (uint32_t)((t >> 1) & 1), abort_flag)) { ok = false; break; }
-        const float lo_part = xl[(xb * 2 + (half ^ 1)) * kQ + m];
-        any = any || lo_part >= 0.f;
-        float lt = l + fmaxf(lo_part, 0.f);
-        float ref = qref;
-        // Underflow of every term: redo the row with its exact maximum.
-        const bool redo = any && !(lt >= kTinySum);
-        if (__any_sync(0xffffffffu, redo)) {
-          float mx = -INFINITY;
-          for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
-            if (j0 < lo || j0 >= win_hi) continue;
-            uint32_t sv[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(s_tmem + j0, sv);
-            tmem_ld_wait(sv);
-            const int kb = kbase(j0);
-            for (int e = 0; e < 32; ++e) {
-              const int kp = pos_s[kb + e];
-              if (kp <= qlim && kp != qpos)
-                mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
-            }
-          }
-          xm[half * kQ + m] = mx;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&rbar[quad]);
-          if (!mbar_wait(&rbar[quad], rph, abort_flag)) { ok = false; break; }
-          rph ^= 1;
-          const float gmax = fmaxf(mx, xm[(half ^ 1) * kQ + m]);
-          float l2 = 0.f;
-          for (int j0 = half * 32; j0 < K::kNk; j0 += 64) {
-            if (j0 < lo || j0 >= win_hi) continue;
-            uint32_t sv[32];
-            __syncwarp();
-            tmem_ld_32x32b_x32(s_tmem + j0, sv);
-            tmem_ld_wait(sv);
-            if (!redo) continue;
-            const int kb = kbase(j0);
-            uint8_t* base = prow + (j0 / 64) * (kQ * 128);
-            for (int e = 0; e < 32; e += 8) {
-              uint32_t w[4];
-              for (int h = 0; h < 8; h += 2) {
-                float pr[2];
-                for (int g = 0; g < 2; ++g) {
-                  const int kp = pos_s[kb + e + h + g];
-                  const bool valid = kp <= qlim && kp != qpos;
-                  pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ksc_s[kb + e + h + g],
-                                           -gmax))
-                                : 0.f;
-                  l2 += pr[g];
-                }
-                w[h / 2] = pack_bf16(pr[0], pr[1]);
-              }
-              *reinterpret_cast<uint4*>(base + sw128_offset(m, (j0 % 64) + e)) =
-                  make_uint4(w[0], w[1], w[2], w[3]);
-            }
-          }
-          xl2[half * kQ + m] = l2;
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&rbar[quad]);
-          if (!mbar_wait(&rbar[quad], rph, abort_flag)) { ok = false; break; }
-          rph ^= 1;
-          if (redo) {
-            lt = l2 + xl2[(half ^ 1) * kQ + m];
-            ref = gmax;
-          }
+        if (stage) {
+          uint8_t* atom = my_ost + (d0 / 64) * (16 * 128);
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4*>(atom + sw128_offset(r16, (d0 % 64) + 8 * q)) = w[q];
+        } else {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
         }
-        tc_fence_before_sync();
-        fence_proxy_async_smem();
-        __syncwarp();
+      }
+      if (mine && q_valid)
+        p.lse_rounds[seg_row + st.qpos] = st.any ? st.ref * kLn2 + logf(st.lt) : kSelfScore;
+      tc_fence_before_sync();
+      if (stage) fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&o_free[buf]);
+      if (stage) {
+        // destination rows of my 16 rows, gathered to lane 0
+        const int dst = (int)(seg_row + st.qpos);
+        int y[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) y[k] = __shfl_sync(0xffffffffu, dst, 16 * half + k);
         if (lane == 0) {
-          mbar_arrive(&s_free[buf]);
-          mbar_arrive(&p_full[pb]);
-          // the look-back block's metadata is not needed again, nor this
-          // block's at the strip's last step (qpos and qref are in registers)
-          if (has_prev) mbar_arrive(&qk_empty[ps]);
-          if (s == U.s1 - 1) mbar_arrive(&qk_empty[cs]);
+#pragma unroll
+          for (int g = 0; g < 4; ++g)
+#pragma unroll
+            for (int h = 0; h < D / 64; ++h)
+              tma_scatter4(&omap, my_ost + h * (16 * 128) + g * 512, h * 64, y[4 * g],
+                           y[4 * g + 1], y[4 * g + 2], y[4 * g + 3]);
+          bulk_commit_group();
+          st_pending = true;
         }
-        // ---- O / l to the row's original position: this warp's half of the columns
-        if (!mbar_wait(&o_full[buf], bph, abort_flag)) { ok = false; break; }
-        tc_fence_after_sync();
-        const float inv_l = any ? 1.f / lt : 0.f;
-        __nv_bfloat16* orow = o_out + (size_t)(q_valid ? qpos : 0) * D;
-#pragma unroll
-        for (int d0 = half * (D / 2); d0 < (half + 1) * (D / 2); d0 += 32) {
-          uint32_t ov[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(o_tmem + d0, ov);
-          tmem_ld_wait(ov);
-          if (q_valid) {
-            if (any) {
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint4 w;
-                w.x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv_l,
-                                __uint_as_float(ov[8 * q + 1]) * inv_l);
-                w.y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv_l,
-                                __uint_as_float(ov[8 * q + 3]) * inv_l);
-                w.z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv_l,
-                                __uint_as_float(ov[8 * q + 5]) * inv_l);
-                w.w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv_l,
-                                __uint_as_float(ov[8 * q + 7]) * inv_l);
-                *reinterpret_cast<uint4*>(orow + d0 + 8 * q) = w;
-              }
-            } else {
-              // nothing but itself to attend to: the -1e5 self score makes it v_i
-              const uint4* vr = reinterpret_cast<const uint4*>(vsrc + (size_t)qpos * D + d0);
-              uint4* dst = reinterpret_cast<uint4*>(orow + d0);
-#pragma unroll
-              for (int q = 0; q < 4; ++q) dst[q] = vr[q];
-            }
-          }
-        }
-        if (q_valid && half == 0) lse_out[qpos] = any ? ref * kLn2 + logf(lt) : kSelfScore;
-        tc_fence_before_sync();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&o_free[buf]);
+      }
+      return true;
+    };
+
+    long long li = 0, t = 0;
+    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
+      const Unit U = unit_of(p, u);
+      const long long first = li;
+      li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
+      RowState cur, next;
+      if (!p_pass(U, first, U.s0, t, cur)) { ok = false; break; }
+      for (int s = U.s0; s < U.s1; ++s, ++t) {
+        if (s + 1 < U.s1 && !p_pass(U, first, s + 1, t + 1, next)) { ok = false; break; }
+        if (!o_pass(U, t, s, cur)) { ok = false; break; }
+        cur = next;
       }
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitEpilogue);
       *abort_flag = 1;
     }
+    if (lane == 0 && st_pending) bulk_wait_all();  // staged stores done before the CTA exits
   }
+
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
+// Ring depths that fit, preferring (in this order) a staged output tile,
+// double-buffered P with at least three key tiles, and key tiles before
+// value tiles; at least two of each.
 template <int C, int D>
-bool plan(const Problem& pr, int* slots, int* pbufs, size_t* smem) {
-  for (int ns = 3; ns >= 2; --ns)
-    for (int np = 2; np >= 1; --np) {
-      const size_t t = layout<C, D>(ns, np).total + 1024;
-      if (t <= (size_t)kSmemLimit) {
-        *slots = ns;
-        *pbufs = np;
-        *smem = std::max<size_t>(t, 116 * 1024);
-        return true;
-      }
+bool plan(int* nq, int* nv, int* np, int* stage_o, size_t* smem) {
+  const size_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
+  for (int so = 1; so >= 0; --so)
+    for (int pb = 2; pb >= 1; --pb) {
+      const size_t fixed = layout<C, D>(0, 0, pb, so).total + n_barriers(6, 6) * 8;
+      if (fixed >= limit) continue;
+      const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
+      if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
+      const int q = std::min(5, (tiles + 1) / 2), v = std::min(5, tiles - q);
+      *nq = q;
+      *nv = v;
+      *np = pb;
+      *stage_o = so;
+      *smem = std::max<size_t>(layout<C, D>(q, v, pb, so).total + 1024, 116 * 1024);
+      return *smem <= (size_t)kSmemLimit;
     }
   return false;
 }
 
-}  // namespace
-
-bool attn_tc_supported(const Problem& p) {
-  return p.bf16 && (p.d == 64 || p.d == 128) && (p.c == 64 || p.c == 128) &&
-         (long long)p.BH() * p.L < (1LL << 31) - 1 && sm100::tensor_map_encoder() != nullptr;
-}
-
 template <int C, int D>
-static cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v,
-                             const float* inv_norm, const int32_t* perm, void* o_rounds,
-                             float* lse_rounds, cudaStream_t st) {
+cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const float* inv_norm,
+                      const int32_t* perm, void* o_rounds, float* lse_rounds, cudaStream_t st) {
   Params p;
   size_t smem = 0;
-  if (!plan<C, D>(pr, &p.slots, &p.pbufs, &smem)) return cudaErrorNotSupported;
+  if (!plan<C, D>(&p.nq, &p.nv, &p.np, &p.stage_o, &smem)) return cudaErrorNotSupported;
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;
-  p.qk = static_cast<const __nv_bfloat16*>(qk);
   p.v = static_cast<const __nv_bfloat16*>(v);
   p.inv_norm = inv_norm;
   p.perm = perm;
@@ -679,12 +821,14 @@ static cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v,
   p.ksc = kLog2e / sqrtf((float)pr.d);
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
-  // [B*H*L, d] views of qk and v: boxes of one row of 64 elements (128 B),
-  // 128B swizzle, rows outside the tensor read as zeros.
-  CUtensorMap maps[2];
-  const void* bases[2] = {qk, v};
-  for (int k = 0; k < 2; ++k) {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)pr.BH() * pr.L};
+  // [B*H*L, d] views of qk and v and the [B*H*n_h*L, d] view of o_rounds:
+  // boxes of one row of 64 elements (128 B), 128B swizzle; gathered rows
+  // outside the tensor read as zeros (stores are only issued for real rows).
+  CUtensorMap maps[3];
+  const void* bases[3] = {qk, v, o_rounds};
+  for (int k = 0; k < 3; ++k) {
+    const cuuint64_t rows = (cuuint64_t)pr.BH() * pr.L * (k == 2 ? pr.n_h : 1);
+    const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
     const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, 1};
     const cuuint32_t estr[2] = {1, 1};
@@ -698,8 +842,16 @@ static cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  attn_tc_kernel<C, D><<<grid, kThreads, smem, st>>>(maps[0], maps[1], p);
+  attn_tc_kernel<C, D><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], p);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attn_tc_supported(const Problem& p) {
+  return p.bf16 && (p.d == 64 || p.d == 128) && (p.c == 64 || p.c == 128) &&
+         (long long)p.BH() * p.n_h * p.L < (1LL << 31) - 1 &&
+         sm100::tensor_map_encoder() != nullptr;
 }
 
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,

@@ -248,3 +248,21 @@ def test_headline_workload_sampled():
                       "out(sampled)")
         P.check_lse(g["f_lse"][0, h][t].cpu(), np.array(o_lse), bf16, "lse(sampled)")
     assert torch.equal(g["f_out"], g["out"]) and torch.equal(g["f_lse"], g["lse"])
+
+
+def test_sharded_ranks_concatenate_to_the_full_pass():
+    # Each "rank" runs the unchanged pass on its own (batch, head) pairs; run
+    # one after another here, they must reproduce the one-call result.
+    from lsh_bucketed_sparse_b200 import sharding
+    wl = W.small("shards", batch=2, heads=3, seq_len=1024, n_hashes=2, n_buckets=64)
+    qk, v, rot = [t.to(DEV) for t in W.make_inputs(wl)]
+    full_out, full_lse = lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets,
+                                              wl.chunk_len, wl.causal)
+    outs, lses = [], []
+    for r in range(4):
+        o, l = sharding.forward_local(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len,
+                                      wl.causal, r, 4)
+        outs.append(o[0])
+        lses.append(l[0])
+    assert torch.equal(torch.cat(outs), full_out.reshape(6, *full_out.shape[2:]))
+    assert torch.equal(torch.cat(lses), full_lse.reshape(6, -1))
