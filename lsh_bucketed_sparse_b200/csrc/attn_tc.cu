@@ -88,9 +88,7 @@ struct Params {
   int steps;          // ceil(L / 128) per segment
   int strip;          // steps per unit
   int n_strips;
-  long long n_units;
-  int nq, nv, np;     // qk tiles, v tiles, P buffers
-  int stage_o;        // O leaves through a shared-memory tile and TMA scatter4
+  int n_units;
   float ksc;          // log2 e / sqrt(d)
 };
 
@@ -98,14 +96,14 @@ struct Layout {
   uint32_t qk, v, p, ost, pos, ksc, qref, xch, bars, misc, total;
 };
 
-__host__ __device__ inline uint32_t n_barriers(int nq, int nv) {
+__host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
   return 2 * nq + 2 * nv + 2 * kMetaSlots + 2 * 8 + 4 + 1;
 }
 
 template <int C, int D>
-__host__ __device__ inline Layout layout(int nq, int nv, int np, int stage_o) {
+__host__ __device__ constexpr Layout layout(int nq, int nv, int np, int stage_o) {
   using K = Cfg<C, D>;
-  Layout l;
+  Layout l{};
   uint32_t off = 0;
   l.qk = off;   off += nq * K::kTile;
   l.v = off;    off += nv * K::kTile;
@@ -151,10 +149,10 @@ struct Unit {
   int bh, r, s0, s1;
 };
 
-__device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
+__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
   Unit x;
-  const int strip = (int)(u % p.n_strips);
-  const long long seg = u / p.n_strips;
+  const int strip = u % p.n_strips;
+  const int seg = u / p.n_strips;
   x.r = (int)(seg % p.n_h);
   x.bh = (int)(seg / p.n_h);
   x.s0 = strip * p.strip;
@@ -165,13 +163,13 @@ __device__ __forceinline__ Unit unit_of(const Params& p, long long u) {
 // The CTA's sequence of blocks to load: for each of its units, the look-back
 // block (if s0 > 0) and then blocks s0 .. s1-1.
 struct Cursor {
-  long long u;
+  int u;
   Unit U;
   int b;
   bool valid;
 };
 
-__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, long long u) {
+__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, int u) {
   c.u = u;
   c.valid = u < p.n_units;
   if (c.valid) {
@@ -180,7 +178,7 @@ __device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, long lo
   }
 }
 
-__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, long long u_step) {
+__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, int u_step) {
   if (!c.valid) return;
   if (++c.b >= c.U.s1) cursor_start(c, p, c.u + u_step);
 }
@@ -222,6 +220,34 @@ struct RowState {
   float ref;    // exponent reference, log2 units
 };
 
+// Ring depths that fit, preferring (in this order) a staged output tile,
+// double-buffered P with at least three key tiles, and key tiles before
+// value tiles; at least two of each.  Fixed per (chunk, d), so the kernel
+// sees the depths as compile-time constants.
+struct Plan {
+  int nq, nv, np, stage_o;
+  uint32_t smem;
+  bool ok;
+};
+
+template <int C, int D>
+__host__ __device__ constexpr Plan make_plan() {
+  constexpr uint32_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
+  for (int so = 1; so >= 0; --so)
+    for (int pb = 2; pb >= 1; --pb) {
+      const uint32_t fixed = layout<C, D>(0, 0, pb, so).total + n_barriers(6, 6) * 8;
+      if (fixed >= limit) continue;
+      const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
+      if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
+      const int q = (tiles + 1) / 2 < 5 ? (tiles + 1) / 2 : 5;
+      const int v = tiles - q < 5 ? tiles - q : 5;
+      uint32_t smem = layout<C, D>(q, v, pb, so).total + 1024;
+      if (smem < 116 * 1024) smem = 116 * 1024;
+      return Plan{q, v, pb, so, smem, smem <= (uint32_t)kSmemLimit};
+    }
+  return Plan{0, 0, 0, 0, 0, false};
+}
+
 template <int C, int D>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
@@ -230,8 +256,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const int NQ = p.nq, NV = p.nv, NP = p.np, NM = kMetaSlots;
-  const Layout Ly = layout<C, D>(NQ, NV, NP, p.stage_o);
+  constexpr Plan PL = make_plan<C, D>();
+  constexpr int NQ = PL.nq, NV = PL.nv, NP = PL.np, NM = kMetaSlots;
+  constexpr bool kStageO = PL.stage_o != 0;
+  constexpr Layout Ly = layout<C, D>(NQ, NV, NP, PL.stage_o);
   uint8_t* ost_s = smem + Ly.ost;
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
@@ -297,7 +325,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const long long u_begin = blockIdx.x, u_step = gridDim.x;
+  const int u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (warp == 0) {
     // ================================================================ qk producer
@@ -317,7 +345,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 #pragma unroll
     for (int k = 0; k < 4; ++k)
       in0[k] = pos0[k] != INT_MAX ? p.inv_norm[(size_t)c0.U.bh * p.L + pos0[k]] : 0.f;
-    long long li = 0;
+    int li = 0;
     bool ok = true;
     for (; ok && c0.valid; ++li) {
       // prefetch for the next two blocks
@@ -372,7 +400,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     cursor_next(c1, p, u_step);
     int pos0[4];
     cursor_positions(c0, p, lane, pos0);
-    long long li = 0;
+    int li = 0;
     bool ok = true;
     for (; ok && c0.valid; ++li) {
       int pos1[4];
@@ -401,14 +429,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   } else if (warp == 1) {
     // ================================================================ MMA issuer
     if (lane == 0) {
-      long long li = 0, t = 0;  // blocks consumed, steps issued
+      int li = 0, t = 0;  // blocks consumed, steps issued
       bool ok = true, issued = false;
       const uint32_t idesc_prev = idesc_bf16_f32(kQ, C);
       const uint32_t idesc_cur = idesc_bf16_f32(kQ, kQ);
       const uint32_t idesc_pv = idesc_bf16_f32_bmn(kQ, D);
       // S(s) = Q K^T into the step's TMEM buffer (ts = the step's counter).
-      auto issue_qk = [&](const Unit& U, long long first, int s, long long ts) -> bool {
-        const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
+      auto issue_qk = [&](const Unit& U, int first, int s, int ts) -> bool {
+        const int ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
         const bool has_prev = s > 0;
         const int cs = (int)(ci % NQ), ps = (int)(((pi % NQ) + NQ) % NQ);
         const int buf = (int)(ts % K::kNbuf);
@@ -435,8 +463,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         return true;
       };
       // O(s) = P(s) V once the softmax has written P(s).
-      auto issue_pv = [&](const Unit& U, long long first, int s, long long ts) -> bool {
-        const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
+      auto issue_pv = [&](const Unit& U, int first, int s, int ts) -> bool {
+        const int ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
         const bool has_prev = s > 0;
         const int cs = (int)(ci % NV), ps = (int)(((pi % NV) + NV) % NV);
         const int buf = (int)(ts % K::kNbuf);
@@ -468,9 +496,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
         return true;
       };
-      for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
+      for (int u = u_begin; ok && u < p.n_units; u += u_step) {
         const Unit U = unit_of(p, u);
-        const long long first = li;
+        const int first = li;
         li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
         // S of the next step is computed while the softmax works on this one.
         if (!issue_qk(U, first, U.s0, t)) { ok = false; break; }
@@ -507,8 +535,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
     // P pass of step s (step counter ts): S from TMEM -> P (bf16) in shared
     // memory; returns the row's state for its output.
-    auto p_pass = [&](const Unit& U, long long first, int s, long long ts, RowState& st) -> bool {
-      const long long ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
+    auto p_pass = [&](const Unit& U, int first, int s, int ts, RowState& st) -> bool {
+      const int ci = first + (s - U.s0) + (U.s0 > 0 ? 1 : 0), pi = ci - 1;
       const bool has_prev = s > 0;
       const int cs = (int)(ci % NM), ps = (int)(((pi % NM) + NM) % NM);
       const int buf = (int)(ts % K::kNbuf);
@@ -668,10 +696,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     const bool mine = (lane >> 4) == half;
     uint8_t* my_ost = ost_s + (size_t)sw * (16 * D * 2);
     bool st_pending = false;  // lane 0: a scatter from my_ost may still be reading it
-    auto o_pass = [&](const Unit& U, long long ts, int s, const RowState& st) -> bool {
+    auto o_pass = [&](const Unit& U, int ts, int s, const RowState& st) -> bool {
       const int buf = (int)(ts % K::kNbuf);
       const uint32_t o_tmem = tmem_base + lane_off + buf * K::kBufCols + K::kNk;
-      const bool stage = p.stage_o && (s + 1) * kQ <= p.L;  // every query of the step exists
+      const bool stage = kStageO && (s + 1) * kQ <= p.L;  // every query of the step exists
       if (!mbar_wait(&o_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
       tc_fence_after_sync();
       if (stage && lane == 0 && st_pending) bulk_wait_read_all();
@@ -743,10 +771,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       return true;
     };
 
-    long long li = 0, t = 0;
-    for (long long u = u_begin; ok && u < p.n_units; u += u_step) {
+    int li = 0, t = 0;
+    for (int u = u_begin; ok && u < p.n_units; u += u_step) {
       const Unit U = unit_of(p, u);
-      const long long first = li;
+      const int first = li;
       li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
       RowState cur, next;
       if (!p_pass(U, first, U.s0, t, cur)) { ok = false; break; }
@@ -769,35 +797,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   if (warp == 1) tmem_dealloc(tmem_base, 512);
 }
 
-// Ring depths that fit, preferring (in this order) a staged output tile,
-// double-buffered P with at least three key tiles, and key tiles before
-// value tiles; at least two of each.
-template <int C, int D>
-bool plan(int* nq, int* nv, int* np, int* stage_o, size_t* smem) {
-  const size_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
-  for (int so = 1; so >= 0; --so)
-    for (int pb = 2; pb >= 1; --pb) {
-      const size_t fixed = layout<C, D>(0, 0, pb, so).total + n_barriers(6, 6) * 8;
-      if (fixed >= limit) continue;
-      const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
-      if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
-      const int q = std::min(5, (tiles + 1) / 2), v = std::min(5, tiles - q);
-      *nq = q;
-      *nv = v;
-      *np = pb;
-      *stage_o = so;
-      *smem = std::max<size_t>(layout<C, D>(q, v, pb, so).total + 1024, 116 * 1024);
-      return *smem <= (size_t)kSmemLimit;
-    }
-  return false;
-}
-
 template <int C, int D>
 cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const float* inv_norm,
                       const int32_t* perm, void* o_rounds, float* lse_rounds, cudaStream_t st) {
+  constexpr Plan PL = make_plan<C, D>();
+  static_assert(PL.ok, "no shared-memory plan for this (chunk, d)");
   Params p;
-  size_t smem = 0;
-  if (!plan<C, D>(&p.nq, &p.nv, &p.np, &p.stage_o, &smem)) return cudaErrorNotSupported;
+  const size_t smem = PL.smem;
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;
   p.v = static_cast<const __nv_bfloat16*>(v);
@@ -817,7 +823,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   strip = std::min(strip, p.steps);
   p.strip = strip;
   p.n_strips = (p.steps + strip - 1) / strip;
-  p.n_units = segs * p.n_strips;
+  p.n_units = (int)(segs * p.n_strips);
   p.ksc = kLog2e / sqrtf((float)pr.d);
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;

@@ -61,7 +61,7 @@ struct Params {
 };
 
 struct Smem {  // offsets inside the 1024-aligned dynamic shared memory
-  uint32_t r, x, bars, xch, misc, total;
+  uint32_t r, x, save, bars, xch, misc, total;
 };
 
 __host__ __device__ inline Smem smem_layout(int n_cols, int d, int stages) {
@@ -69,6 +69,7 @@ __host__ __device__ inline Smem smem_layout(int n_cols, int d, int stages) {
   uint32_t off = 0;
   s.r = off;    off += (uint32_t)n_cols * d * 2;
   s.x = off;    off += (uint32_t)stages * kRows * d * 2;
+  s.save = off; off += kEpiWarps * 32 * kChunk * 4;   // one 128-byte row per epilogue thread
   s.bars = off; off += (uint32_t)(2 * stages + 4 + 4 + 1) * 8;
   s.xch = off;  off += 2 * kRows * 8;
   s.misc = off; off += 16;
@@ -88,6 +89,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
   const Smem L = smem_layout(p.n_cols, p.d, p.stages);
   uint8_t* r_smem = smem + L.r;
   uint8_t* x_smem = smem + L.x;
+  uint8_t* save_smem = smem + L.save;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars);
   uint64_t* x_full = bars;
   uint64_t* x_empty = bars + p.stages;
@@ -221,13 +223,31 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     const int half = ew >> 2;            // which alternate 32-column chunks
     const int row = quad * 32 + lane;    // token row inside the tile
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
+    // This thread's copy of the chunk that holds its row's largest |p| so
+    // far: a private 128-byte row, 16-byte pieces rotated by (lane & 7) so
+    // that neighbouring lanes hit different banks.
+    uint8_t* my_save = save_smem + (size_t)(ew * 32 + lane) * (kChunk * 4);
+    const int sx = lane & 7;
+    auto save_chunk = [&](const uint32_t* u) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        *reinterpret_cast<uint4*>(my_save + ((q ^ sx) << 4)) =
+            make_uint4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+    };
+    auto load_saved = [&](float* sv) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const uint4 w = *reinterpret_cast<const uint4*>(my_save + ((q ^ sx) << 4));
+        sv[4 * q] = __uint_as_float(w.x);
+        sv[4 * q + 1] = __uint_as_float(w.y);
+        sv[4 * q + 2] = __uint_as_float(w.z);
+        sv[4 * q + 3] = __uint_as_float(w.w);
+      }
+    };
     int it = 0, gp = 0, ex = 0;
     bool ok = true;
     float best_a = -1.f;
-    int saved_j0 = 0;
-    float sv[kChunk];
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) sv[t] = 0.f;
+    int best_j0 = 0;
 
     for (int tile = g; ok && tile < p.n_tiles; tile += p.G, ++it) {
       const int bh = tile / p.tiles_per_head, t0 = (tile % p.tiles_per_head) * kRows;
@@ -261,19 +281,19 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
         tc_fence_after_sync();
         const int col0 = pc * p.piece_w;
         const int w = min(p.piece_w, p.n_cols - col0);
+        int rr = col0 / p.P;             // round (within the group) of column col0
+        int j0 = col0 - rr * p.P;        // its column inside the round
+        const uint32_t taddr = lane_addr + (uint32_t)(buf * kPieceMax - col0);
         for (int c = col0; c < col0 + w; c += kChunk) {
-          const int rr = c / p.P, j0 = c % p.P;
-          if (((c / kChunk) & 1) == half) {
+          if (((c >> 5) & 1) == half) {
             uint32_t u[kChunk];
             __syncwarp();
-            tmem_ld_32x32b_x32(lane_addr + (uint32_t)(buf * kPieceMax + (c - col0)), u);
+            tmem_ld_32x32b_x32(taddr + (uint32_t)c, u);
             tmem_ld_wait(u);
-            float v[kChunk];
-#pragma unroll
-            for (int t = 0; t < kChunk; ++t) v[t] = __uint_as_float(u[t]);
             float m[16];
 #pragma unroll
-            for (int t = 0; t < 16; ++t) m[t] = fmaxf(fabsf(v[2 * t]), fabsf(v[2 * t + 1]));
+            for (int t = 0; t < 16; ++t)
+              m[t] = fmaxf(fabsf(__uint_as_float(u[2 * t])), fabsf(__uint_as_float(u[2 * t + 1])));
 #pragma unroll
             for (int t = 0; t < 8; ++t) m[t] = fmaxf(m[t], m[t + 8]);
 #pragma unroll
@@ -283,33 +303,37 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
             if (cm == best_a) {
               // Equal largest |p| in an earlier chunk: a positive entry wins
               // over negative ones, and the earlier chunk wins otherwise.
+              float sv[kChunk];
+              load_saved(sv);
               bool pos_saved = false, pos_new = false;
 #pragma unroll
               for (int t = 0; t < kChunk; ++t) {
                 pos_saved |= (sv[t] == best_a);
-                pos_new |= (v[t] == cm);
+                pos_new |= (__uint_as_float(u[t]) == cm);
               }
               take = !pos_saved && pos_new;
             }
             if (take) {
               best_a = cm;
-              saved_j0 = j0;
-#pragma unroll
-              for (int t = 0; t < kChunk; ++t) sv[t] = v[t];
+              best_j0 = j0;
+              save_chunk(u);
             }
           }
-          if (j0 + kChunk == p.P) {
+          j0 += kChunk;
+          if (j0 == p.P) {
             // End of round r0 + rr: this half's candidate, then the exchange.
             int z = INT_MAX;
-            float a = best_a;
+            const float a = best_a;
             if (best_a >= 0.f) {
+              float sv[kChunk];
+              load_saved(sv);
               int tp = -1, tn = 0;
 #pragma unroll
               for (int t = kChunk - 1; t >= 0; --t) {
                 if (sv[t] == best_a) tp = t;
                 if (sv[t] == -best_a) tn = t;
               }
-              z = tp >= 0 ? saved_j0 + tp : p.P + saved_j0 + tn;
+              z = tp >= 0 ? best_j0 + tp : p.P + best_j0 + tn;
             }
             best_a = -1.f;
             const int xb = ex & 1;
@@ -331,6 +355,8 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
                 p.buckets[((size_t)bh * p.n_h + r0 + rr) * p.L + t0 + row] = (int16_t)z;
             }
             ++ex;
+            j0 = 0;
+            ++rr;
           }
         }
         if (!ok) break;
@@ -362,35 +388,36 @@ bool make_plan(const Problem& pr, Plan* out) {
   const int P = pr.half();
   if (P <= 0 || P % kChunk) return false;
   const int d = pr.d;
-  // rounds per group: the largest divisor of n_h whose rotations fit
-  int gr = 0;
-  for (int k = pr.n_h; k >= 1; --k)
-    if (pr.n_h % k == 0 && (size_t)k * P * d * 2 <= (size_t)kRBudget) { gr = k; break; }
-  if (gr == 0) return false;
-  int piece_w;
-  if (P <= kPieceMax) {
-    const int rpp = std::min(gr, kPieceMax / P);
-    piece_w = rpp * P;
-  } else {
-    const int s = (P + kPieceMax - 1) / kPieceMax;
-    if (P % s || (P / s) % kChunk) return false;
-    piece_w = P / s;
+  // The largest group of rounds (a divisor of n_h) whose rotations, at least
+  // two X stages, the save rows and the barriers fit in shared memory.
+  for (int gr = pr.n_h; gr >= 1; --gr) {
+    if (pr.n_h % gr) continue;
+    if ((size_t)gr * P * d * 2 > (size_t)kRBudget) continue;
+    const int n_cols = gr * P;
+    int piece_w;
+    if (P <= kPieceMax) {
+      piece_w = std::min(gr, kPieceMax / P) * P;
+    } else {
+      const int s = (P + kPieceMax - 1) / kPieceMax;
+      if (P % s || (P / s) % kChunk) return false;
+      piece_w = P / s;
+    }
+    for (int stages = d == 64 ? 4 : 3; stages >= 2; --stages) {
+      const Smem L = smem_layout(n_cols, d, stages);
+      if (L.total + 1024 > (uint32_t)kSmemLimit) continue;
+      out->gr = gr;
+      out->n_groups = pr.n_h / gr;
+      out->G = (int)std::max(1LL, std::min<long long>(148 / out->n_groups, n_tiles));
+      out->piece_w = piece_w;
+      out->n_pieces = (n_cols + piece_w - 1) / piece_w;
+      out->stages = stages;
+      // At least half the SM's shared memory: one CTA per SM, since each CTA
+      // allocates all 512 TMEM columns.
+      out->smem = std::max<size_t>(L.total + 1024, 116 * 1024);
+      return true;
+    }
   }
-  const int n_cols = gr * P;
-  int stages = d == 64 ? 4 : 2;
-  Smem L = smem_layout(n_cols, d, stages);
-  while (stages > 2 && L.total + 1024 > (uint32_t)kSmemLimit) L = smem_layout(n_cols, d, --stages);
-  if (L.total + 1024 > (uint32_t)kSmemLimit) return false;
-  out->gr = gr;
-  out->n_groups = pr.n_h / gr;
-  out->G = (int)std::max(1LL, std::min<long long>(148 / out->n_groups, n_tiles));
-  out->piece_w = piece_w;
-  out->n_pieces = (n_cols + piece_w - 1) / piece_w;
-  out->stages = stages;
-  // At least half the SM's shared memory: one CTA per SM, since each CTA
-  // allocates all 512 TMEM columns.
-  out->smem = std::max<size_t>(L.total + 1024, 116 * 1024);
-  return true;
+  return false;
 }
 
 }  // namespace

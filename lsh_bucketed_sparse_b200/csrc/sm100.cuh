@@ -72,15 +72,31 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Wait until the phase of `bar` with parity `parity` has completed.  Gives up
-// (returns false) when *abort is set by another thread or after
-// kWaitLimitNs; the caller then records an error and leaves its loop.
+// Like mbar_try_wait, but the thread may be suspended (without taking issue
+// slots) until the phase completes or about `suspend_ns` have passed.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity,
+                                                      uint32_t suspend_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(suspend_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Wait until the phase of `bar` with parity `parity` has completed.  Each
+// attempt suspends the thread for up to 0.5 ms, so waiting costs no issue
+// slots.  Gives up (returns false) when *abort is set by another thread or
+// after kWaitLimitNs; the caller then records an error and leaves its loop.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, 500000u)) return true;
     if (*abort) return false;
     if (globaltimer() - t0 > kWaitLimitNs) return false;
   }
