@@ -125,6 +125,15 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+// 16-byte shared-memory store issued only where `pred` holds, without a branch.
+__device__ __forceinline__ void st_shared_if(bool pred, uint32_t addr, uint4 v) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+      "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((uint32_t)pred),
+      "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+      : "memory");
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -710,39 +719,43 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       __nv_bfloat16* orow = p.o_rounds + (seg_row + (q_valid ? st.qpos : 0)) * D;
       const __nv_bfloat16* vrow = p.v + ((size_t)U.bh * p.L + (q_valid ? st.qpos : 0)) * D;
       const int r16 = lane & 15;
+      const bool put = mine && q_valid;
+      // rows with nothing but themselves to attend to (rare) output v_i
+      const bool self_only = put && !st.any;
+      const bool any_self_only = __any_sync(0xffffffffu, self_only);
 #pragma unroll
       for (int d0 = 0; d0 < D; d0 += 32) {
         uint32_t ov[32];
-        __syncwarp();
         tmem_ld_32x32b_x32(o_tmem + d0, ov);
         tmem_ld_wait(ov);
-        if (!mine || !q_valid) continue;
         uint4 w[4];
-        if (st.any) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            w[q].x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv_l,
-                               __uint_as_float(ov[8 * q + 1]) * inv_l);
-            w[q].y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv_l,
-                               __uint_as_float(ov[8 * q + 3]) * inv_l);
-            w[q].z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv_l,
-                               __uint_as_float(ov[8 * q + 5]) * inv_l);
-            w[q].w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv_l,
-                               __uint_as_float(ov[8 * q + 7]) * inv_l);
-          }
-        } else {
+        for (int q = 0; q < 4; ++q) {
+          w[q].x = pack_bf16(__uint_as_float(ov[8 * q + 0]) * inv_l,
+                             __uint_as_float(ov[8 * q + 1]) * inv_l);
+          w[q].y = pack_bf16(__uint_as_float(ov[8 * q + 2]) * inv_l,
+                             __uint_as_float(ov[8 * q + 3]) * inv_l);
+          w[q].z = pack_bf16(__uint_as_float(ov[8 * q + 4]) * inv_l,
+                             __uint_as_float(ov[8 * q + 5]) * inv_l);
+          w[q].w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv_l,
+                             __uint_as_float(ov[8 * q + 7]) * inv_l);
+        }
+        if (any_self_only) {
           // nothing but itself to attend to: the -1e5 self score makes it v_i
 #pragma unroll
-          for (int q = 0; q < 4; ++q) w[q] = reinterpret_cast<const uint4*>(vrow + d0)[q];
+          for (int q = 0; q < 4; ++q) {
+            const uint4 vq = self_only ? reinterpret_cast<const uint4*>(vrow + d0)[q] : w[q];
+            w[q] = vq;
+          }
         }
         if (stage) {
-          uint8_t* atom = my_ost + (d0 / 64) * (16 * 128);
+          const uint32_t atom = smem_u32(my_ost + (d0 / 64) * (16 * 128));
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4*>(atom + sw128_offset(r16, (d0 % 64) + 8 * q)) = w[q];
+          for (int q = 0; q < 4; ++q) st_shared_if(put, atom + sw128_offset(r16, (d0 % 64) + 8 * q), w[q]);
         } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
+          for (int q = 0; q < 4; ++q)
+            if (put) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
         }
       }
       if (mine && q_valid)

@@ -228,11 +228,17 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     // that neighbouring lanes hit different banks.
     uint8_t* my_save = save_smem + (size_t)(ew * 32 + lane) * (kChunk * 4);
     const int sx = lane & 7;
-    auto save_chunk = [&](const uint32_t* u) {
+    // Predicated stores: no branch, so the warp stays converged.
+    auto save_chunk_if = [&](bool take, const uint32_t* u) {
+      const uint32_t base = smem_u32(my_save);
 #pragma unroll
       for (int q = 0; q < 8; ++q)
-        *reinterpret_cast<uint4*>(my_save + ((q ^ sx) << 4)) =
-            make_uint4(u[4 * q], u[4 * q + 1], u[4 * q + 2], u[4 * q + 3]);
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+            "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((uint32_t)take),
+            "r"(base + (uint32_t)((q ^ sx) << 4)), "r"(u[4 * q]), "r"(u[4 * q + 1]),
+            "r"(u[4 * q + 2]), "r"(u[4 * q + 3])
+            : "memory");
     };
     auto load_saved = [&](float* sv) {
 #pragma unroll
@@ -300,9 +306,9 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
             for (int t = 0; t < 4; ++t) m[t] = fmaxf(m[t], m[t + 4]);
             const float cm = fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
             bool take = cm > best_a;
-            if (cm == best_a) {
-              // Equal largest |p| in an earlier chunk: a positive entry wins
-              // over negative ones, and the earlier chunk wins otherwise.
+            if (__any_sync(0xffffffffu, cm == best_a)) {
+              // Equal largest |p| in an earlier chunk (rare): a positive entry
+              // wins over negative ones, and the earlier chunk wins otherwise.
               float sv[kChunk];
               load_saved(sv);
               bool pos_saved = false, pos_new = false;
@@ -311,13 +317,11 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
                 pos_saved |= (sv[t] == best_a);
                 pos_new |= (__uint_as_float(u[t]) == cm);
               }
-              take = !pos_saved && pos_new;
+              if (cm == best_a) take = !pos_saved && pos_new;
             }
-            if (take) {
-              best_a = cm;
-              best_j0 = j0;
-              save_chunk(u);
-            }
+            best_a = take ? cm : best_a;
+            best_j0 = take ? j0 : best_j0;
+            save_chunk_if(take, u);
           }
           j0 += kChunk;
           if (j0 == p.P) {
