@@ -81,6 +81,31 @@ __device__ __forceinline__ bool better(float a, int z, float ba, int bz) {
   return a > ba || (a == ba && z < bz);
 }
 
+// max(a, b, c): one three-input instruction on sm_100.
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// Largest |p| of a 32-column chunk: a depth-4 tree of 17 max instructions.
+__device__ __forceinline__ float chunk_max_abs(const uint32_t* u) {
+  float v[11];
+#pragma unroll
+  for (int t = 0; t < 10; ++t)
+    v[t] = max3f(fabsf(__uint_as_float(u[3 * t])), fabsf(__uint_as_float(u[3 * t + 1])),
+                 fabsf(__uint_as_float(u[3 * t + 2])));
+  v[10] = fmaxf(fabsf(__uint_as_float(u[30])), fabsf(__uint_as_float(u[31])));
+  const float w0 = max3f(v[0], v[1], v[2]), w1 = max3f(v[3], v[4], v[5]);
+  const float w2 = max3f(v[6], v[7], v[8]), w3 = fmaxf(v[9], v[10]);
+  return fmaxf(max3f(w0, w1, w2), w3);
+}
+
+// NP > 0: every piece is NP pairs of 32-column chunks and a round is a whole
+// number of pairs (P % 64 == 0), so each epilogue warp takes one chunk of
+// every pair at fixed positions and loads the next chunk while it reduces the
+// current one.  NP == 0: any P that is a multiple of 32.
+template <int NP>
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -231,14 +256,28 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     // Predicated stores: no branch, so the warp stays converged.
     auto save_chunk_if = [&](bool take, const uint32_t* u) {
       const uint32_t base = smem_u32(my_save);
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
-            "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((uint32_t)take),
-            "r"(base + (uint32_t)((q ^ sx) << 4)), "r"(u[4 * q]), "r"(u[4 * q + 1]),
-            "r"(u[4 * q + 2]), "r"(u[4 * q + 3])
-            : "memory");
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+          "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
+          "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t"
+          "@p st.shared.v4.b32 [%11], {%12, %13, %14, %15};\n\t"
+          "@p st.shared.v4.b32 [%16], {%17, %18, %19, %20};\n\t}" ::"r"((uint32_t)take),
+          "r"(base + (uint32_t)((0 ^ sx) << 4)), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]),
+          "r"(base + (uint32_t)((1 ^ sx) << 4)), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
+          "r"(base + (uint32_t)((2 ^ sx) << 4)), "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]),
+          "r"(base + (uint32_t)((3 ^ sx) << 4)), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+          : "memory");
+      asm volatile(
+          "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+          "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
+          "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t"
+          "@p st.shared.v4.b32 [%11], {%12, %13, %14, %15};\n\t"
+          "@p st.shared.v4.b32 [%16], {%17, %18, %19, %20};\n\t}" ::"r"((uint32_t)take),
+          "r"(base + (uint32_t)((4 ^ sx) << 4)), "r"(u[16]), "r"(u[17]), "r"(u[18]), "r"(u[19]),
+          "r"(base + (uint32_t)((5 ^ sx) << 4)), "r"(u[20]), "r"(u[21]), "r"(u[22]), "r"(u[23]),
+          "r"(base + (uint32_t)((6 ^ sx) << 4)), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]),
+          "r"(base + (uint32_t)((7 ^ sx) << 4)), "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
+          : "memory");
     };
     auto load_saved = [&](float* sv) {
 #pragma unroll
@@ -254,6 +293,67 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     bool ok = true;
     float best_a = -1.f;
     int best_j0 = 0;
+
+    // One 32-column chunk starting at round column j0: keep it when it holds
+    // a larger |p| than every earlier chunk of the round.
+    auto take_chunk = [&](const uint32_t* u, int j0) {
+      const float cm = chunk_max_abs(u);
+      bool take = cm > best_a;
+      if (__any_sync(0xffffffffu, cm == best_a)) {
+        // Equal largest |p| in an earlier chunk (rare): a positive entry
+        // wins over negative ones, and the earlier chunk wins otherwise.
+        float sv[kChunk];
+        load_saved(sv);
+        bool pos_saved = false, pos_new = false;
+#pragma unroll
+        for (int t = 0; t < kChunk; ++t) {
+          pos_saved |= (sv[t] == best_a);
+          pos_new |= (__uint_as_float(u[t]) == cm);
+        }
+        if (cm == best_a) take = !pos_saved && pos_new;
+      }
+      best_a = take ? cm : best_a;
+      best_j0 = take ? j0 : best_j0;
+      save_chunk_if(take, u);
+    };
+
+    // End of round r0 + rr: this half's candidate, then the two halves meet
+    // and half 0 writes the bucket.  Returns false on a wait timeout.
+    auto round_end = [&](int bh, int t0, int rr, bool row_valid) -> bool {
+      int z = INT_MAX;
+      const float a = best_a;
+      if (best_a >= 0.f) {
+        float sv[kChunk];
+        load_saved(sv);
+        int tp = -1, tn = 0;
+#pragma unroll
+        for (int t = kChunk - 1; t >= 0; --t) {
+          if (sv[t] == best_a) tp = t;
+          if (sv[t] == -best_a) tn = t;
+        }
+        z = tp >= 0 ? best_j0 + tp : p.P + best_j0 + tn;
+      }
+      best_a = -1.f;
+      const int xb = ex & 1;
+      const uint32_t par = (ex >> 1) & 1;
+      ++ex;
+      if (half == 1) {
+        if (!mbar_wait(&xc_empty[xb], par ^ 1, abort_flag)) return false;
+        xch_a[xb * kRows + row] = a;
+        xch_z[xb * kRows + row] = z;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xc_full[xb]);
+      } else {
+        if (!mbar_wait(&xc_full[xb], par, abort_flag)) return false;
+        const float oa = xch_a[xb * kRows + row];
+        const int oz = xch_z[xb * kRows + row];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&xc_empty[xb]);
+        if (better(oa, oz, a, z)) z = oz;
+        if (row_valid) p.buckets[((size_t)bh * p.n_h + r0 + rr) * p.L + t0 + row] = (int16_t)z;
+      }
+      return true;
+    };
 
     for (int tile = g; ok && tile < p.n_tiles; tile += p.G, ++it) {
       const int bh = tile / p.tiles_per_head, t0 = (tile % p.tiles_per_head) * kRows;
@@ -281,86 +381,54 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
         __syncwarp();
         if (lane == 0) mbar_arrive(&x_empty[s]);
       }
+      int rr = 0, j0 = 0;  // round (within the group) and column of the next chunk
       for (int pc = 0; pc < p.n_pieces; ++pc, ++gp) {
         const int buf = gp & 1;
         if (!mbar_wait(&t_full[buf], (gp >> 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after_sync();
-        const int col0 = pc * p.piece_w;
-        const int w = min(p.piece_w, p.n_cols - col0);
-        int rr = col0 / p.P;             // round (within the group) of column col0
-        int j0 = col0 - rr * p.P;        // its column inside the round
-        const uint32_t taddr = lane_addr + (uint32_t)(buf * kPieceMax - col0);
-        for (int c = col0; c < col0 + w; c += kChunk) {
-          if (((c >> 5) & 1) == half) {
-            uint32_t u[kChunk];
-            __syncwarp();
-            tmem_ld_32x32b_x32(taddr + (uint32_t)c, u);
-            tmem_ld_wait(u);
-            float m[16];
+        if constexpr (NP > 0) {
+          // My chunk of pair m sits at piece column 64 m + 32 half.
+          const uint32_t taddr = lane_addr + (uint32_t)(buf * kPieceMax + kChunk * half);
+          uint32_t u[2][kChunk];
+          __syncwarp();
+          tmem_ld_32x32b_x32(taddr, u[0]);
+          tmem_ld_wait(u[0]);
 #pragma unroll
-            for (int t = 0; t < 16; ++t)
-              m[t] = fmaxf(fabsf(__uint_as_float(u[2 * t])), fabsf(__uint_as_float(u[2 * t + 1])));
-#pragma unroll
-            for (int t = 0; t < 8; ++t) m[t] = fmaxf(m[t], m[t + 8]);
-#pragma unroll
-            for (int t = 0; t < 4; ++t) m[t] = fmaxf(m[t], m[t + 4]);
-            const float cm = fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
-            bool take = cm > best_a;
-            if (__any_sync(0xffffffffu, cm == best_a)) {
-              // Equal largest |p| in an earlier chunk (rare): a positive entry
-              // wins over negative ones, and the earlier chunk wins otherwise.
-              float sv[kChunk];
-              load_saved(sv);
-              bool pos_saved = false, pos_new = false;
-#pragma unroll
-              for (int t = 0; t < kChunk; ++t) {
-                pos_saved |= (sv[t] == best_a);
-                pos_new |= (__uint_as_float(u[t]) == cm);
-              }
-              if (cm == best_a) take = !pos_saved && pos_new;
+          for (int m = 0; m < NP; ++m) {
+            if (m + 1 < NP) {
+              __syncwarp();
+              tmem_ld_32x32b_x32(taddr + (uint32_t)(2 * kChunk * (m + 1)), u[(m + 1) & 1]);
             }
-            best_a = take ? cm : best_a;
-            best_j0 = take ? j0 : best_j0;
-            save_chunk_if(take, u);
+            if (ok) {
+              take_chunk(u[m & 1], j0 + kChunk * half);
+              j0 += 2 * kChunk;
+              if (j0 == p.P) {
+                ok = round_end(bh, t0, rr, row_valid);
+                j0 = 0;
+                ++rr;
+              }
+            }
+            // the load in flight lands before anything else happens
+            if (m + 1 < NP) tmem_ld_wait(u[(m + 1) & 1]);
           }
-          j0 += kChunk;
-          if (j0 == p.P) {
-            // End of round r0 + rr: this half's candidate, then the exchange.
-            int z = INT_MAX;
-            const float a = best_a;
-            if (best_a >= 0.f) {
-              float sv[kChunk];
-              load_saved(sv);
-              int tp = -1, tn = 0;
-#pragma unroll
-              for (int t = kChunk - 1; t >= 0; --t) {
-                if (sv[t] == best_a) tp = t;
-                if (sv[t] == -best_a) tn = t;
-              }
-              z = tp >= 0 ? best_j0 + tp : p.P + best_j0 + tn;
-            }
-            best_a = -1.f;
-            const int xb = ex & 1;
-            const uint32_t par = (ex >> 1) & 1;
-            if (half == 1) {
-              if (!mbar_wait(&xc_empty[xb], par ^ 1, abort_flag)) { ok = false; break; }
-              xch_a[xb * kRows + row] = a;
-              xch_z[xb * kRows + row] = z;
+        } else {
+          const int col0 = pc * p.piece_w;
+          const int w = min(p.piece_w, p.n_cols - col0);
+          const uint32_t taddr = lane_addr + (uint32_t)(buf * kPieceMax - col0);
+          for (int c = col0; c < col0 + w; c += kChunk) {
+            if (((c >> 5) & 1) == half) {
+              uint32_t u[kChunk];
               __syncwarp();
-              if (lane == 0) mbar_arrive(&xc_full[xb]);
-            } else {
-              if (!mbar_wait(&xc_full[xb], par, abort_flag)) { ok = false; break; }
-              const float oa = xch_a[xb * kRows + row];
-              const int oz = xch_z[xb * kRows + row];
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&xc_empty[xb]);
-              if (better(oa, oz, a, z)) z = oz;
-              if (row_valid)
-                p.buckets[((size_t)bh * p.n_h + r0 + rr) * p.L + t0 + row] = (int16_t)z;
+              tmem_ld_32x32b_x32(taddr + (uint32_t)c, u);
+              tmem_ld_wait(u);
+              take_chunk(u, j0);
             }
-            ++ex;
-            j0 = 0;
-            ++rr;
+            j0 += kChunk;
+            if (j0 == p.P) {
+              if (!round_end(bh, t0, rr, row_valid)) { ok = false; break; }
+              j0 = 0;
+              ++rr;
+            }
           }
         }
         if (!ok) break;
@@ -384,6 +452,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
 // ---------------------------------------------------------------- host side
 struct Plan {
   int gr, n_groups, G, piece_w, n_pieces, stages;
+  int np;  // pairs of chunks per piece for the fixed-position epilogue, 0 = general
   size_t smem;
 };
 
@@ -415,6 +484,9 @@ bool make_plan(const Problem& pr, Plan* out) {
       out->piece_w = piece_w;
       out->n_pieces = (n_cols + piece_w - 1) / piece_w;
       out->stages = stages;
+      out->np = (P % (2 * kChunk) == 0 && piece_w % (2 * kChunk) == 0 && n_cols % piece_w == 0)
+                    ? piece_w / (2 * kChunk)
+                    : 0;
       // At least half the SM's shared memory: one CTA per SM, since each CTA
       // allocates all 512 TMEM columns.
       out->smem = std::max<size_t>(L.total + 1024, 116 * 1024);
@@ -464,10 +536,18 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   p.piece_w = plan.piece_w;
   p.n_pieces = plan.n_pieces;
   p.stages = plan.stages;
-  cudaError_t e = cudaFuncSetAttribute(hash_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)plan.smem);
+  void (*kernel)(const CUtensorMap, const Params);
+  switch (plan.np) {
+    case 1: kernel = hash_tc_kernel<1>; break;
+    case 2: kernel = hash_tc_kernel<2>; break;
+    case 3: kernel = hash_tc_kernel<3>; break;
+    case 4: kernel = hash_tc_kernel<4>; break;
+    default: kernel = hash_tc_kernel<0>; break;
+  }
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
   if (e != cudaSuccess) return e;
-  hash_tc_kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p);
+  kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p);
   return cudaGetLastError();
 }
 

@@ -97,6 +97,8 @@ SMALL = [
     W.small("tc-hash-d128-p384", heads=2, seq_len=512, d_k=128, n_hashes=2, n_buckets=768,
             chunk_len=128, causal=False),
     W.small("tc-hash-p96", heads=3, seq_len=768, n_hashes=4, n_buckets=192),
+    # 64-column rounds, four per 256-column piece, and a ragged last tile
+    W.small("tc-hash-p64", heads=2, seq_len=1088, n_hashes=4, n_buckets=128),
     # the four tensor-core attention specialisations (chunk, d_k)
     W.small("tc-attn-c64-d128", heads=2, seq_len=1472, d_k=128, n_hashes=2, n_buckets=64),
     W.small("tc-attn-c128-d64-causal", heads=2, seq_len=1408, n_hashes=3, n_buckets=64,
@@ -164,6 +166,51 @@ def test_zero_rows_and_scaled_rows():
     assert (b[:, 5] == 0).all() and (b[:, 77] == 0).all()
     assert torch.equal(b[:, 100], b[:, 99])
     assert g["inv_norm"][0, 0, 5] == 0
+
+
+def _planted_tie_rotations(wl, rot):
+    """Rotations whose column j1 = 3 (scaled by 4, so it usually holds the
+    largest |p|) is repeated in a chunk of the same epilogue half, repeated in
+    a chunk of the other half, and negated in a later chunk: every token then
+    has exact |p| ties, which the argmax breaks by the lowest index of
+    [xR; -xR] (a positive entry before any negative one, then the smaller j)."""
+    P_ = wl.n_buckets // 2
+    j1 = 3
+    same = j1 + 64 if P_ > j1 + 64 else 7
+    other = j1 + 32 if P_ > j1 + 32 else 11
+    neg = j1 + 96 if P_ > j1 + 96 else P_ - 5
+    assert len({j1, same, other, neg}) == 4 and max(same, other, neg) < P_
+    rot = rot.clone()
+    rot[:, :, j1] *= 4
+    rot[:, :, same] = rot[:, :, j1]
+    rot[:, :, other] = rot[:, :, j1]
+    rot[:, :, neg] = -rot[:, :, j1]
+    return rot
+
+
+@pytest.mark.parametrize("portable", [False, True], ids=["fast", "portable"])
+@pytest.mark.parametrize("n_buckets", [64, 192, 256, 1024])
+def test_hash_breaks_exact_ties_by_lowest_index(n_buckets, portable):
+    wl = W.small(f"ties-{n_buckets}", heads=2, seq_len=640, n_hashes=2, n_buckets=n_buckets)
+    qk, _, rot = W.make_inputs(wl)
+    rot = _planted_tie_rotations(wl, rot)
+    b, _ = lsh.lsh_attn_hash(qk.to(DEV), rot.to(DEV), wl.n_buckets, wl.n_hashes,
+                             portable=portable)
+    b = b.cpu().numpy().astype(np.int64)
+    x, R = P.np64(qk), P.np64(rot)
+    checked = 0
+    for h in range(wl.heads):
+        for r in range(wl.n_hashes):
+            p = x[0, h] @ R[r]
+            z = np.concatenate([p, -p], axis=1)
+            top = z.max(1, keepdims=True)
+            below = np.where(z < top, z, -np.inf).max(1)
+            clear = (top[:, 0] - below) >= 1e-5      # a clear gap below the tied group
+            want = np.argmax(z, axis=1)               # first maximal index
+            ok = b[0, h, r] == want
+            assert ok[clear].all(), np.nonzero(~ok & clear)[0][:10]
+            checked += int(clear.sum())
+    assert checked > 0.9 * wl.heads * wl.n_hashes * wl.seq_len
 
 
 @pytest.mark.parametrize("chunk,d", [(64, 64), (128, 128)])
