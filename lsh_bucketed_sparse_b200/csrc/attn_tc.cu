@@ -97,7 +97,8 @@ struct Layout {
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
-  return 2 * nq + 2 * nv + 2 * kMetaSlots + 2 * 8 + 4 + 1;
+  // rings; S/O/P full/free pairs (2 x 6); exchange (2 x 4); redo (4); done
+  return 2 * nq + 2 * nv + 2 * kMetaSlots + 12 + 8 + 4 + 1;
 }
 
 template <int C, int D>
@@ -257,7 +258,7 @@ __host__ __device__ constexpr Plan make_plan() {
   return Plan{0, 0, 0, 0, 0, false};
 }
 
-template <int C, int D>
+template <int C, int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
                const __grid_constant__ CUtensorMap omap, const Params p) {
@@ -292,8 +293,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   uint64_t* o_free = o_full + 2;         // [2] O read
   uint64_t* p_full = o_free + 2;         // [2] P written
   uint64_t* p_empty = p_full + 2;        // [2] P consumed
-  uint64_t* xbar = p_empty + 2;          // [2] partial-sum exchange, all softmax warps
-  uint64_t* rbar = xbar + 2;             // [4] redo exchange, the two warps of a quadrant
+  uint64_t* xbar = p_empty + 2;          // [2][4] partial-sum exchange, the two warps of a quadrant
+  uint64_t* rbar = xbar + 8;             // [4] redo exchange, the two warps of a quadrant
   uint64_t* done = rbar + 4;             // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
@@ -319,7 +320,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       mbar_init(&o_free[b], kSoftWarps);
       mbar_init(&p_full[b], kSoftWarps);
       mbar_init(&p_empty[b], 1);
-      mbar_init(&xbar[b], kSoftWarps);
+      for (int q = 0; q < 4; ++q) mbar_init(&xbar[b * 4 + q], 2);
     }
     for (int q = 0; q < 4; ++q) mbar_init(&rbar[q], 2);
     mbar_init(done, 1);
@@ -575,6 +576,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           tmem_ld_32x32b_x32(s_tmem + j0, sv);
           tmem_ld_wait(sv);
           const int kb = kbase(j0);
+          // Causal: a key is visible iff its position is below the query's
+          // (one comparison, which also leaves the query itself out), and
+          // the row sees some key iff the chunk's smallest position does.
+          if (CAUSAL) any |= __reduce_min_sync(0xffffffffu, pos_s[kb + lane]) < qpos;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
@@ -584,8 +589,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             float pr[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
-              const bool valid = kpa[h] <= qlim && kpa[h] != qpos;
-              any |= valid;
+              bool valid;
+              if (CAUSAL) {
+                valid = kpa[h] < qpos;
+              } else {
+                valid = kpa[h] <= qlim && kpa[h] != qpos;
+                any |= valid;
+              }
               const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
               pr[h] = valid ? ex2(x) : 0.f;
               la[h] += pr[h];
@@ -611,8 +621,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int xb = (int)(ts & 1);
       xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
       __syncwarp();
-      if (lane == 0) mbar_arrive(&xbar[xb]);
-      if (!mbar_wait(&xbar[xb], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
+      if (lane == 0) mbar_arrive(&xbar[xb * 4 + quad]);
+      if (!mbar_wait(&xbar[xb * 4 + quad], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
       const float other = xl[(xb * 2 + (half ^ 1)) * kQ + m];
       any = any || other >= 0.f;
       float lt = l + fmaxf(other, 0.f);
@@ -857,11 +867,12 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<C, D>,
+  auto kernel = pr.causal ? attn_tc_kernel<C, D, true> : attn_tc_kernel<C, D, false>;
+  cudaError_t e = cudaFuncSetAttribute(kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  attn_tc_kernel<C, D><<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], p);
+  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], p);
   return cudaGetLastError();
 }
 

@@ -99,6 +99,10 @@ SMALL = [
     W.small("tc-hash-p96", heads=3, seq_len=768, n_hashes=4, n_buckets=192),
     # 64-column rounds, four per 256-column piece, and a ragged last tile
     W.small("tc-hash-p64", heads=2, seq_len=1088, n_hashes=4, n_buckets=128),
+    # rounds of whole 128-column groups: one round per 256-column piece, and
+    # 384-column rounds that end inside a piece
+    W.small("tc-hash-p256", heads=2, seq_len=1088, n_hashes=3, n_buckets=512),
+    W.small("tc-hash-p384", heads=2, seq_len=1088, n_hashes=2, n_buckets=768),
     # the four tensor-core attention specialisations (chunk, d_k)
     W.small("tc-attn-c64-d128", heads=2, seq_len=1472, d_k=128, n_hashes=2, n_buckets=64),
     W.small("tc-attn-c128-d64-causal", heads=2, seq_len=1408, n_hashes=3, n_buckets=64,
