@@ -17,18 +17,22 @@ constexpr int kThreads = 256;
 template <typename T> struct Vec16;
 template <> struct Vec16<float> {
   static constexpr int N = 4;
-  __device__ static void load(const float* p, float* f) {
-    const float4 u = *reinterpret_cast<const float4*>(p);
-    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+  __device__ static uint4 raw(const float* p) { return *reinterpret_cast<const uint4*>(p); }
+  __device__ static void unpack(const uint4& u, float* f) {
+    f[0] = __uint_as_float(u.x); f[1] = __uint_as_float(u.y);
+    f[2] = __uint_as_float(u.z); f[3] = __uint_as_float(u.w);
   }
+  __device__ static void load(const float* p, float* f) { unpack(raw(p), f); }
   __device__ static void store(float* p, const float* f) {
     *reinterpret_cast<float4*>(p) = make_float4(f[0], f[1], f[2], f[3]);
   }
 };
 template <> struct Vec16<__nv_bfloat16> {
   static constexpr int N = 8;
-  __device__ static void load(const __nv_bfloat16* p, float* f) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p);
+  __device__ static uint4 raw(const __nv_bfloat16* p) {
+    return *reinterpret_cast<const uint4*>(p);
+  }
+  __device__ static void unpack(const uint4& u, float* f) {
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
@@ -36,6 +40,7 @@ template <> struct Vec16<__nv_bfloat16> {
       f[2 * t] = x.x; f[2 * t + 1] = x.y;
     }
   }
+  __device__ static void load(const __nv_bfloat16* p, float* f) { unpack(raw(p), f); }
   __device__ static void store(__nv_bfloat16* p, const float* f) {
     uint4 u;
     __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
@@ -45,12 +50,16 @@ template <> struct Vec16<__nv_bfloat16> {
   }
 };
 
-template <typename T>
+// NH > 0: the number of rounds as a compile-time constant, so every round's
+// lse and 16-byte piece are loaded before any is used (all loads in flight
+// at once); NH == 0: any n_h.
+template <typename T, int NH>
 __global__ void __launch_bounds__(kThreads)
 combine_kernel(const T* __restrict__ o_rounds, const float* __restrict__ lse_rounds,
                T* __restrict__ out, float* __restrict__ lse, long long rows, int L, int d,
-               int n_h) {
+               int n_h_rt) {
   using V = Vec16<T>;
+  const int n_h = NH > 0 ? NH : n_h_rt;
   const int per_row = d / V::N;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long row = tid / per_row;
@@ -58,26 +67,73 @@ combine_kernel(const T* __restrict__ o_rounds, const float* __restrict__ lse_rou
   if (row >= rows) return;
   const long long bh = row / L, i = row % L;
   const float* lr = lse_rounds + bh * n_h * (long long)L + i;
-  float m = -INFINITY;
-  for (int r = 0; r < n_h; ++r) m = fmaxf(m, lr[(long long)r * L]);
-  float s = 0.f;
-  for (int r = 0; r < n_h; ++r) s += expf(lr[(long long)r * L] - m);
-  const float LSE = m + logf(s);
-  // exp(lse_r - LSE) evaluated as exp(lse_r - m) / s: the differences to the
-  // maximum stay exact even where |lse| is ~1e5 (a token that saw only itself).
-  const float inv_s = 1.f / s;
+  const T* orow = o_rounds + (bh * n_h * (long long)L + i) * d + part * V::N;
   float acc[V::N];
 #pragma unroll
   for (int t = 0; t < V::N; ++t) acc[t] = 0.f;
-  for (int r = 0; r < n_h; ++r) {
-    const float w = expf(lr[(long long)r * L] - m) * inv_s;
-    float f[V::N];
-    V::load(o_rounds + ((bh * n_h + r) * (long long)L + i) * d + part * V::N, f);
+  float LSE;
+  if constexpr (NH > 0) {
+    float l[NH];
+    uint4 u[NH];
 #pragma unroll
-    for (int t = 0; t < V::N; ++t) acc[t] = fmaf(w, f[t], acc[t]);
+    for (int r = 0; r < NH; ++r) {
+      l[r] = lr[(long long)r * L];
+      u[r] = V::raw(orow + (long long)r * L * d);
+    }
+    float m = l[0];
+#pragma unroll
+    for (int r = 1; r < NH; ++r) m = fmaxf(m, l[r]);
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+      l[r] = expf(l[r] - m);
+      s += l[r];
+    }
+    LSE = m + logf(s);
+    // exp(lse_r - LSE) evaluated as exp(lse_r - m) / s: the differences to
+    // the maximum stay exact even where |lse| is ~1e5 (a token that saw only
+    // itself).
+    const float inv_s = 1.f / s;
+#pragma unroll
+    for (int r = 0; r < NH; ++r) {
+      const float w = l[r] * inv_s;
+      float f[V::N];
+      V::unpack(u[r], f);
+#pragma unroll
+      for (int t = 0; t < V::N; ++t) acc[t] = fmaf(w, f[t], acc[t]);
+    }
+  } else {
+    float m = -INFINITY;
+    for (int r = 0; r < n_h; ++r) m = fmaxf(m, lr[(long long)r * L]);
+    float s = 0.f;
+    for (int r = 0; r < n_h; ++r) s += expf(lr[(long long)r * L] - m);
+    LSE = m + logf(s);
+    const float inv_s = 1.f / s;
+    for (int r = 0; r < n_h; ++r) {
+      const float w = expf(lr[(long long)r * L] - m) * inv_s;
+      float f[V::N];
+      V::load(orow + (long long)r * L * d, f);
+#pragma unroll
+      for (int t = 0; t < V::N; ++t) acc[t] = fmaf(w, f[t], acc[t]);
+    }
   }
   V::store(out + row * d + part * V::N, acc);
   if (part == 0) lse[row] = LSE;
+}
+
+template <typename T>
+void launch_t(const Problem& p, const void* o_rounds, const float* lse_rounds, void* out,
+              float* lse, unsigned blocks, long long rows, cudaStream_t st) {
+  const T* o = static_cast<const T*>(o_rounds);
+  T* y = static_cast<T*>(out);
+  switch (p.n_h) {
+    case 1: combine_kernel<T, 1><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 1); break;
+    case 2: combine_kernel<T, 2><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 2); break;
+    case 4: combine_kernel<T, 4><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 4); break;
+    case 8: combine_kernel<T, 8><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 8); break;
+    default:
+      combine_kernel<T, 0><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, p.n_h);
+  }
 }
 
 }  // namespace
@@ -89,12 +145,9 @@ cudaError_t launch_combine(const Problem& p, const void* o_rounds, const float* 
   const long long threads = rows * per_row;
   const unsigned blocks = (unsigned)((threads + kThreads - 1) / kThreads);
   if (p.bf16)
-    combine_kernel<__nv_bfloat16><<<blocks, kThreads, 0, st>>>(
-        (const __nv_bfloat16*)o_rounds, lse_rounds, (__nv_bfloat16*)out, lse, rows, p.L, p.d,
-        p.n_h);
+    launch_t<__nv_bfloat16>(p, o_rounds, lse_rounds, out, lse, blocks, rows, st);
   else
-    combine_kernel<float><<<blocks, kThreads, 0, st>>>((const float*)o_rounds, lse_rounds,
-                                                       (float*)out, lse, rows, p.L, p.d, p.n_h);
+    launch_t<float>(p, o_rounds, lse_rounds, out, lse, blocks, rows, st);
   return cudaGetLastError();
 }
 

@@ -21,6 +21,7 @@ namespace lsh {
 namespace {
 
 constexpr int kThreads = 1024;
+constexpr int kBatch = 16;  // keys per thread loaded ahead
 constexpr int kMaxSmem = 227 * 1024 - 1024;  // leave room for static shared memory
 
 // Exclusive scan of a[0..n) in place by the whole block; returns nothing.
@@ -74,9 +75,20 @@ sort_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ perm,
 
   for (int t = tid; t < W * n_b; t += blockDim.x) sh[t] = 0;
   __syncthreads();
-  for (int e = tid; e < L; e += blockDim.x) {
-    const int b = keys[e];
-    if ((unsigned)b < (unsigned)n_b) atomicAdd(&sh[(e / len) * n_b + b], 1);
+  // kBatch loads in flight per thread before their counts, so the loop pays
+  // the memory latency once per batch rather than once per key
+  for (int e0 = tid; e0 < L; e0 += kBatch * blockDim.x) {
+    int kb[kBatch];
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int e = e0 + i * blockDim.x;
+      kb[i] = e < L ? (int)keys[e] : -1;
+    }
+#pragma unroll
+    for (int i = 0; i < kBatch; ++i) {
+      const int e = e0 + i * blockDim.x;
+      if ((unsigned)kb[i] < (unsigned)n_b) atomicAdd(&sh[(e / len) * n_b + kb[i]], 1);
+    }
   }
   __syncthreads();
   if (W > 1) {
@@ -103,21 +115,31 @@ sort_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ perm,
   if (warp < W) {
     int32_t* off = sh + (size_t)warp * n_b;
     const int beg = warp * len, end = min(L, beg + len);
-    for (int base = beg; base < end; base += 32) {
-      const int e = base + lane;
-      int b = (e < end) ? (int)keys[e] : -1 - lane;
-      const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
-      const unsigned peers = __match_any_sync(0xffffffffu, b);
-      const int rank = __popc(peers & ((1u << lane) - 1u));
-      int slot = 0;
-      if (valid) slot = off[b] + rank;
-      __syncwarp();
-      if (valid) {
-        P[slot] = e;
-        if (U) U[e] = slot;
-        if (lane == 31 - __clz(peers)) off[b] += __popc(peers);
+    for (int base0 = beg; base0 < end; base0 += 32 * kBatch) {
+      // the next kBatch rows of 32 keys, loaded ahead of their ranking
+      int kb[kBatch];
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int e = base0 + 32 * i + lane;
+        kb[i] = (e < end) ? (int)keys[e] : -1 - lane;
       }
-      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < kBatch; ++i) {
+        const int e = base0 + 32 * i + lane;
+        const int b = kb[i];
+        const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
+        const unsigned peers = __match_any_sync(0xffffffffu, b);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        int slot = 0;
+        if (valid) slot = off[b] + rank;
+        __syncwarp();
+        if (valid) {
+          P[slot] = e;
+          if (U) U[e] = slot;
+          if (lane == 31 - __clz(peers)) off[b] += __popc(peers);
+        }
+        __syncwarp();
+      }
     }
   }
 }
