@@ -40,10 +40,10 @@
 //               outputs v_i with lse -1e5, the value the -1e5 self score
 //               gives).  The softmax of step s+1 runs before the output of
 //               step s, so P V overlaps it.  For the output the two warps of
-//               a quadrant split its 32 rows: each stages its 16 rows of
-//               O / l in a private shared-memory region and writes them to
-//               the rows' original positions with TMA (tile::scatter4, four
-//               full rows per instruction); lse goes out directly.
+//               a quadrant split the D columns: each writes its half of O / l
+//               for the quadrant's 32 rows straight to their original
+//               positions; half 0 writes lse.  Waits spin on the barrier
+//               (no suspend), which keeps the hand-offs between roles short.
 #include <algorithm>
 #include <climits>
 
@@ -93,7 +93,7 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, p, ost, pos, ksc, qref, xch, bars, misc, total;
+  uint32_t qk, v, p, pos, ksc, qref, xch, bars, misc, total;
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
@@ -102,14 +102,13 @@ __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
 }
 
 template <int C, int D>
-__host__ __device__ constexpr Layout layout(int nq, int nv, int np, int stage_o) {
+__host__ __device__ constexpr Layout layout(int nq, int nv, int np) {
   using K = Cfg<C, D>;
   Layout l{};
   uint32_t off = 0;
   l.qk = off;   off += nq * K::kTile;
   l.v = off;    off += nv * K::kTile;
   l.p = off;    off += np * K::kPBytes;
-  l.ost = off;  off += stage_o ? K::kTile : 0;     // staged O: 16 rows per softmax warp
   l.pos = off;  off += kMetaSlots * kQ * 4;
   l.ksc = off;  off += kMetaSlots * kQ * 4;
   l.qref = off; off += kMetaSlots * kQ * 4;
@@ -230,12 +229,12 @@ struct RowState {
   float ref;    // exponent reference, log2 units
 };
 
-// Ring depths that fit, preferring (in this order) a staged output tile,
-// double-buffered P with at least three key tiles, and key tiles before
-// value tiles; at least two of each.  Fixed per (chunk, d), so the kernel
-// sees the depths as compile-time constants.
+// Ring depths that fit, preferring (in this order) double-buffered P with at
+// least three key tiles, and key tiles before value tiles; at least two of
+// each.  Fixed per (chunk, d), so the kernel sees the depths as compile-time
+// constants.
 struct Plan {
-  int nq, nv, np, stage_o;
+  int nq, nv, np;
   uint32_t smem;
   bool ok;
 };
@@ -243,34 +242,31 @@ struct Plan {
 template <int C, int D>
 __host__ __device__ constexpr Plan make_plan() {
   constexpr uint32_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
-  for (int so = 1; so >= 0; --so)
-    for (int pb = 2; pb >= 1; --pb) {
-      const uint32_t fixed = layout<C, D>(0, 0, pb, so).total + n_barriers(6, 6) * 8;
-      if (fixed >= limit) continue;
-      const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
-      if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
-      const int q = (tiles + 1) / 2 < 5 ? (tiles + 1) / 2 : 5;
-      const int v = tiles - q < 5 ? tiles - q : 5;
-      uint32_t smem = layout<C, D>(q, v, pb, so).total + 1024;
-      if (smem < 116 * 1024) smem = 116 * 1024;
-      return Plan{q, v, pb, so, smem, smem <= (uint32_t)kSmemLimit};
-    }
-  return Plan{0, 0, 0, 0, 0, false};
+  for (int pb = 2; pb >= 1; --pb) {
+    const uint32_t fixed = layout<C, D>(0, 0, pb).total + n_barriers(6, 6) * 8;
+    if (fixed >= limit) continue;
+    const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
+    if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
+    const int q = (tiles + 1) / 2 < 5 ? (tiles + 1) / 2 : 5;
+    const int v = tiles - q < 5 ? tiles - q : 5;
+    uint32_t smem = layout<C, D>(q, v, pb).total + 1024;
+    if (smem < 116 * 1024) smem = 116 * 1024;
+    return Plan{q, v, pb, smem, smem <= (uint32_t)kSmemLimit};
+  }
+  return Plan{0, 0, 0, 0, false};
 }
 
 template <int C, int D, bool CAUSAL>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
-               const __grid_constant__ CUtensorMap omap, const Params p) {
+               const Params p) {
   using K = Cfg<C, D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   constexpr Plan PL = make_plan<C, D>();
   constexpr int NQ = PL.nq, NV = PL.nv, NP = PL.np, NM = kMetaSlots;
-  constexpr bool kStageO = PL.stage_o != 0;
-  constexpr Layout Ly = layout<C, D>(NQ, NV, NP, PL.stage_o);
-  uint8_t* ost_s = smem + Ly.ost;
+  constexpr Layout Ly = layout<C, D>(NQ, NV, NP);
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
   uint8_t* p_s = smem + Ly.p;
@@ -367,8 +363,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         in1[k] = (c1.valid && pos1[k] != INT_MAX)
                      ? p.inv_norm[(size_t)c1.U.bh * p.L + pos1[k]] : 0.f;
       const int qs = (int)(li % NQ), ms = (int)(li % NM);
-      if (!mbar_wait(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
-      if (!mbar_wait(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait_spin(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait_spin(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
       if (lane == 0) mbar_expect_tx(&qk_full[qs], K::kTile);
       __syncwarp();
       const int rowbase = c0.U.bh * p.L;
@@ -416,7 +412,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       int pos1[4];
       cursor_positions(c1, p, lane, pos1);
       const int vs = (int)(li % NV);
-      if (!mbar_wait(&v_empty[vs], (uint32_t)(((li / NV) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait_spin(&v_empty[vs], (uint32_t)(((li / NV) & 1) ^ 1), abort_flag)) { ok = false; break; }
       if (lane == 0) mbar_expect_tx(&v_full[vs], K::kTile);
       __syncwarp();
       const int rowbase = c0.U.bh * p.L;
@@ -450,11 +446,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const bool has_prev = s > 0;
         const int cs = (int)(ci % NQ), ps = (int)(((pi % NQ) + NQ) % NQ);
         const int buf = (int)(ts % K::kNbuf);
-        if (!mbar_wait(&s_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
+        if (!mbar_wait_spin(&s_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
           return false;
-        if (!mbar_wait(&qk_full[cs], (uint32_t)((ci / NQ) & 1), abort_flag)) return false;
+        if (!mbar_wait_spin(&qk_full[cs], (uint32_t)((ci / NQ) & 1), abort_flag)) return false;
         if (has_prev && s == U.s0 &&
-            !mbar_wait(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
+            !mbar_wait_spin(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t s_tmem = tmem_base + buf * K::kBufCols;
@@ -479,12 +475,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const int cs = (int)(ci % NV), ps = (int)(((pi % NV) + NV) % NV);
         const int buf = (int)(ts % K::kNbuf);
         const int pb = (int)(ts % NP);
-        if (!mbar_wait(&p_full[pb], (uint32_t)((ts / NP) & 1), abort_flag)) return false;
-        if (!mbar_wait(&o_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
+        if (!mbar_wait_spin(&p_full[pb], (uint32_t)((ts / NP) & 1), abort_flag)) return false;
+        if (!mbar_wait_spin(&o_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
           return false;
-        if (!mbar_wait(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
+        if (!mbar_wait_spin(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
         if (has_prev && s == U.s0 &&
-            !mbar_wait(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
+            !mbar_wait_spin(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_base + buf * K::kBufCols + K::kNk;
@@ -552,11 +548,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int buf = (int)(ts % K::kNbuf);
       const int pb = (int)(ts % NP);
       const uint32_t s_tmem = tmem_base + lane_off + buf * K::kBufCols;
-      if (!mbar_wait(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
+      if (!mbar_wait_spin(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
       if (has_prev && s == U.s0 &&
-          !mbar_wait(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
+          !mbar_wait_spin(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
         return false;
-      if (!mbar_wait(&s_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
+      if (!mbar_wait_spin(&s_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
       tc_fence_after_sync();
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
@@ -564,7 +560,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int lo = has_prev ? win_lo : max(win_lo, C);
       // metadata row of key column j0 (a multiple of 32, all in one block)
       auto kbase = [&](int j0) { return j0 < C ? ps * kQ + (kQ - C) + j0 : cs * kQ + (j0 - C); };
-      if (!mbar_wait(&p_empty[pb], (uint32_t)(((ts / NP) & 1) ^ 1), abort_flag)) return false;
+      if (!mbar_wait_spin(&p_empty[pb], (uint32_t)(((ts / NP) & 1) ^ 1), abort_flag)) return false;
       uint8_t* prow = p_s + (size_t)pb * K::kPBytes;
       bool any = false;
       float la[4] = {0.f, 0.f, 0.f, 0.f};
@@ -622,7 +618,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
       __syncwarp();
       if (lane == 0) mbar_arrive(&xbar[xb * 4 + quad]);
-      if (!mbar_wait(&xbar[xb * 4 + quad], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
+      if (!mbar_wait_spin(&xbar[xb * 4 + quad], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
       const float other = xl[(xb * 2 + (half ^ 1)) * kQ + m];
       any = any || other >= 0.f;
       float lt = l + fmaxf(other, 0.f);
@@ -647,7 +643,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         xm[half * kQ + m] = mx;
         __syncwarp();
         if (lane == 0) mbar_arrive(&rbar[quad]);
-        if (!mbar_wait(&rbar[quad], rph, abort_flag)) return false;
+        if (!mbar_wait_spin(&rbar[quad], rph, abort_flag)) return false;
         rph ^= 1;
         const float gmax = fmaxf(mx, xm[(half ^ 1) * kQ + m]);
         const bool redo = need;
@@ -682,7 +678,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         xl2[half * kQ + m] = l2;
         __syncwarp();
         if (lane == 0) mbar_arrive(&rbar[quad]);
-        if (!mbar_wait(&rbar[quad], rph, abort_flag)) return false;
+        if (!mbar_wait_spin(&rbar[quad], rph, abort_flag)) return false;
         rph ^= 1;
         if (redo) {
           lt = l2 + xl2[(half ^ 1) * kQ + m];
@@ -707,34 +703,25 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       return true;
     };
 
-    // Output of step s: this warp takes rows lane 16*half .. 16*half+15 of
-    // its quadrant, all D columns: O / l and lse.  When every query of the
-    // step exists and there is room, the rows are staged in this warp's own
-    // 16-row region (128B-swizzled, like the operand tiles) and lane 0
-    // writes them with TMA scatter4; otherwise each lane stores its row.
-    const bool mine = (lane >> 4) == half;
-    uint8_t* my_ost = ost_s + (size_t)sw * (16 * D * 2);
-    bool st_pending = false;  // lane 0: a scatter from my_ost may still be reading it
+    // Output of step s: the two warps of a quadrant split the D columns; each
+    // writes its half of O / l for all 32 rows straight to the rows' original
+    // positions (the two halves of a row's line meet in L2), and half 0 the
+    // lse.
     auto o_pass = [&](const Unit& U, int ts, int s, const RowState& st) -> bool {
       const int buf = (int)(ts % K::kNbuf);
       const uint32_t o_tmem = tmem_base + lane_off + buf * K::kBufCols + K::kNk;
-      const bool stage = kStageO && (s + 1) * kQ <= p.L;  // every query of the step exists
-      if (!mbar_wait(&o_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
+      if (!mbar_wait_spin(&o_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
       tc_fence_after_sync();
-      if (stage && lane == 0 && st_pending) bulk_wait_read_all();
-      __syncwarp();
       const bool q_valid = st.qpos != INT_MAX;
       const size_t seg_row = ((size_t)U.bh * p.n_h + U.r) * p.L;
       const float inv_l = st.any ? 1.f / st.lt : 0.f;
       __nv_bfloat16* orow = p.o_rounds + (seg_row + (q_valid ? st.qpos : 0)) * D;
       const __nv_bfloat16* vrow = p.v + ((size_t)U.bh * p.L + (q_valid ? st.qpos : 0)) * D;
-      const int r16 = lane & 15;
-      const bool put = mine && q_valid;
-      // rows with nothing but themselves to attend to (rare) output v_i
-      const bool self_only = put && !st.any;
+      const bool self_only = q_valid && !st.any;
       const bool any_self_only = __any_sync(0xffffffffu, self_only);
+      __syncwarp();
 #pragma unroll
-      for (int d0 = 0; d0 < D; d0 += 32) {
+      for (int d0 = half * (D / 2); d0 < (half + 1) * (D / 2); d0 += 32) {
         uint32_t ov[32];
         tmem_ld_32x32b_x32(o_tmem + d0, ov);
         tmem_ld_wait(ov);
@@ -758,39 +745,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
             w[q] = vq;
           }
         }
-        if (stage) {
-          const uint32_t atom = smem_u32(my_ost + (d0 / 64) * (16 * 128));
+        if (q_valid) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) st_shared_if(put, atom + sw128_offset(r16, (d0 % 64) + 8 * q), w[q]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < 4; ++q)
-            if (put) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
+          for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
         }
       }
-      if (mine && q_valid)
+      if (half == 0 && q_valid)
         p.lse_rounds[seg_row + st.qpos] = st.any ? st.ref * kLn2 + logf(st.lt) : kSelfScore;
       tc_fence_before_sync();
-      if (stage) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[buf]);
-      if (stage) {
-        // destination rows of my 16 rows, gathered to lane 0
-        const int dst = (int)(seg_row + st.qpos);
-        int y[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) y[k] = __shfl_sync(0xffffffffu, dst, 16 * half + k);
-        if (lane == 0) {
-#pragma unroll
-          for (int g = 0; g < 4; ++g)
-#pragma unroll
-            for (int h = 0; h < D / 64; ++h)
-              tma_scatter4(&omap, my_ost + h * (16 * 128) + g * 512, h * 64, y[4 * g],
-                           y[4 * g + 1], y[4 * g + 2], y[4 * g + 3]);
-          bulk_commit_group();
-          st_pending = true;
-        }
-      }
       return true;
     };
 
@@ -811,7 +775,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       if (lane == 0) atomicOr(p.err, kErrWaitEpilogue);
       *abort_flag = 1;
     }
-    if (lane == 0 && st_pending) bulk_wait_all();  // staged stores done before the CTA exits
   }
 
   tc_fence_before_sync();
@@ -850,13 +813,12 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   p.ksc = kLog2e / sqrtf((float)pr.d);
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
-  // [B*H*L, d] views of qk and v and the [B*H*n_h*L, d] view of o_rounds:
-  // boxes of one row of 64 elements (128 B), 128B swizzle; gathered rows
-  // outside the tensor read as zeros (stores are only issued for real rows).
-  CUtensorMap maps[3];
-  const void* bases[3] = {qk, v, o_rounds};
-  for (int k = 0; k < 3; ++k) {
-    const cuuint64_t rows = (cuuint64_t)pr.BH() * pr.L * (k == 2 ? pr.n_h : 1);
+  // [B*H*L, d] views of qk and v: boxes of one row of 64 elements (128 B),
+  // 128B swizzle; gathered rows outside the tensor read as zeros.
+  CUtensorMap maps[2];
+  const void* bases[2] = {qk, v};
+  for (int k = 0; k < 2; ++k) {
+    const cuuint64_t rows = (cuuint64_t)pr.BH() * pr.L;
     const cuuint64_t dims[2] = {(cuuint64_t)D, rows};
     const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
     const cuuint32_t box[2] = {64, 1};
@@ -872,7 +834,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], maps[2], p);
+  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], p);
   return cudaGetLastError();
 }
 
