@@ -160,9 +160,15 @@ LSH_ATTN_API lsh_status lsh_attn_forward(const lsh_shape* shape, const void* qk,
 
 /* ---------------------------------------------------------------------- *
  * The forward pass from HOST buffers: copies qk, v and rotations to the
- * device, runs lsh_attn_forward, and copies out and lse back, all enqueued on
- * `stream`.  The caller synchronises `stream` before reading out_host /
- * lse_host.  Host buffers should be page-locked for the copies to overlap.
+ * device, runs the forward pass, and copies out and lse back.  The (batch,
+ * head) pairs are independent, so they go in up to 8 groups through three
+ * library-owned streams (copy in, compute, copy out): a group's inputs cross
+ * PCIe while the previous group computes and the one before it copies back.
+ * The work starts after what is already queued on `stream`, and `stream`
+ * waits for all of it, so the caller synchronises `stream` before reading
+ * out_host / lse_host.  Calls on one device enqueue one at a time (a mutex
+ * guards the shared streams).  Host buffers should be page-locked for the
+ * copies to overlap.
  *   device_buffer: caller-owned device memory of at least
  *   lsh_attn_forward_host_device_bytes() bytes, 256-byte aligned; it holds the
  *   device copies of the inputs and outputs plus the workspace.

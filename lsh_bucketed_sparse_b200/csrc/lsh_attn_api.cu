@@ -182,6 +182,35 @@ HostStaging host_layout(const Problem& p) {
   return h;
 }
 
+// The host-buffer pass is split into groups of (batch, head) pairs that flow
+// through three streams: copies in, compute, copies out.  Group g's inputs
+// cross PCIe while group g-1 is computed and group g-2's outputs come back;
+// the compute stream runs the groups in order, so one workspace serves all.
+constexpr int kMaxGroups = 8;
+struct HostPipe {
+  cudaStream_t in, comp, out;
+  cudaEvent_t start, in_done[kMaxGroups], comp_done[kMaxGroups], out_done;
+  bool ok;
+};
+HostPipe g_pipe[kMaxDevices];
+std::once_flag g_pipe_once[kMaxDevices];
+std::mutex g_pipe_mutex[kMaxDevices];
+
+HostPipe* host_pipe(int dev) {
+  std::call_once(g_pipe_once[dev], [dev] {
+    HostPipe& h = g_pipe[dev];
+    h.ok = cudaStreamCreateWithFlags(&h.in, cudaStreamNonBlocking) == cudaSuccess &&
+           cudaStreamCreateWithFlags(&h.comp, cudaStreamNonBlocking) == cudaSuccess &&
+           cudaStreamCreateWithFlags(&h.out, cudaStreamNonBlocking) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h.start, cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&h.out_done, cudaEventDisableTiming) == cudaSuccess;
+    for (int g = 0; h.ok && g < kMaxGroups; ++g)
+      h.ok = cudaEventCreateWithFlags(&h.in_done[g], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h.comp_done[g], cudaEventDisableTiming) == cudaSuccess;
+  });
+  return g_pipe[dev].ok ? &g_pipe[dev] : nullptr;
+}
+
 }  // namespace
 
 unsigned int* device_error_word() {
@@ -304,21 +333,59 @@ lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void* qk_host,
     return fail(LSH_ERR_WORKSPACE, "device_buffer of %zu bytes, need %zu", device_bytes, h.total);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char* base = static_cast<char*>(device_buffer);
-  cudaError_t e;
-  // One cudaMemcpyAsync per tensor.
-  if ((e = cudaMemcpyAsync(base + h.qk, qk_host, h.in_bytes, cudaMemcpyHostToDevice, st)))
-    return cuda_fail(e, "copy qk to device");
-  if ((e = cudaMemcpyAsync(base + h.v, v_host, h.in_bytes, cudaMemcpyHostToDevice, st)))
-    return cuda_fail(e, "copy v to device");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LSH_ERR_UNSUPPORTED, "device %d", dev);
+  HostPipe* hp = host_pipe(dev);
+  if (!hp) return fail(LSH_ERR_CUDA, "could not create the copy/compute streams");
+  // Calls on one device enqueue one at a time (the streams and events are shared).
+  std::lock_guard<std::mutex> lock(g_pipe_mutex[dev]);
+  const int BH = p.BH();
+  const int G = BH < kMaxGroups ? BH : kMaxGroups;
+  const size_t row_in = (size_t)p.L * p.d * p.elem();  // bytes of one (b, h) pair
+  const size_t row_lse = (size_t)p.L * sizeof(float);
+  // Everything starts after the work already on the caller's stream.
+  if ((e = cudaEventRecord(hp->start, st))) return cuda_fail(e, "record start");
+  if ((e = cudaStreamWaitEvent(hp->in, hp->start, 0))) return cuda_fail(e, "wait start");
+  if ((e = cudaStreamWaitEvent(hp->comp, hp->start, 0))) return cuda_fail(e, "wait start");
+  if ((e = cudaStreamWaitEvent(hp->out, hp->start, 0))) return cuda_fail(e, "wait start");
   if (h.rot_bytes &&
-      (e = cudaMemcpyAsync(base + h.rot, rotations_host, h.rot_bytes, cudaMemcpyHostToDevice, st)))
+      (e = cudaMemcpyAsync(base + h.rot, rotations_host, h.rot_bytes, cudaMemcpyHostToDevice,
+                           hp->in)))
     return cuda_fail(e, "copy rotations to device");
-  CHECK(forward_body(p, base + h.qk, base + h.v, h.rot_bytes ? base + h.rot : nullptr,
-                     base + h.out, reinterpret_cast<float*>(base + h.lse), base + h.ws, st));
-  if ((e = cudaMemcpyAsync(out_host, base + h.out, h.out_bytes, cudaMemcpyDeviceToHost, st)))
-    return cuda_fail(e, "copy out to host");
-  if ((e = cudaMemcpyAsync(lse_host, base + h.lse, h.lse_bytes, cudaMemcpyDeviceToHost, st)))
-    return cuda_fail(e, "copy lse to host");
+  for (int g = 0; g < G; ++g) {
+    const int b0 = (int)((long long)BH * g / G), b1 = (int)((long long)BH * (g + 1) / G);
+    const size_t in_off = (size_t)b0 * row_in, in_len = (size_t)(b1 - b0) * row_in;
+    const size_t l_off = (size_t)b0 * row_lse, l_len = (size_t)(b1 - b0) * row_lse;
+    // one cudaMemcpyAsync per tensor slice
+    if ((e = cudaMemcpyAsync(base + h.qk + in_off, static_cast<const char*>(qk_host) + in_off,
+                             in_len, cudaMemcpyHostToDevice, hp->in)))
+      return cuda_fail(e, "copy qk to device");
+    if ((e = cudaMemcpyAsync(base + h.v + in_off, static_cast<const char*>(v_host) + in_off,
+                             in_len, cudaMemcpyHostToDevice, hp->in)))
+      return cuda_fail(e, "copy v to device");
+    if ((e = cudaEventRecord(hp->in_done[g], hp->in))) return cuda_fail(e, "record copy-in");
+    if ((e = cudaStreamWaitEvent(hp->comp, hp->in_done[g], 0))) return cuda_fail(e, "wait copy-in");
+    Problem pg = p;
+    pg.B = 1;
+    pg.H = b1 - b0;
+    CHECK(forward_body(pg, base + h.qk + in_off, base + h.v + in_off,
+                       h.rot_bytes ? base + h.rot : nullptr, base + h.out + in_off,
+                       reinterpret_cast<float*>(base + h.lse + l_off), base + h.ws, hp->comp));
+    if ((e = cudaEventRecord(hp->comp_done[g], hp->comp))) return cuda_fail(e, "record compute");
+    if ((e = cudaStreamWaitEvent(hp->out, hp->comp_done[g], 0))) return cuda_fail(e, "wait compute");
+    if ((e = cudaMemcpyAsync(static_cast<char*>(out_host) + in_off, base + h.out + in_off, in_len,
+                             cudaMemcpyDeviceToHost, hp->out)))
+      return cuda_fail(e, "copy out to host");
+    if ((e = cudaMemcpyAsync(reinterpret_cast<char*>(lse_host) + l_off, base + h.lse + l_off,
+                             l_len, cudaMemcpyDeviceToHost, hp->out)))
+      return cuda_fail(e, "copy lse to host");
+  }
+  // The caller's stream continues once the last copy-out is done (which
+  // follows every compute and copy-in through the events above).
+  if ((e = cudaEventRecord(hp->out_done, hp->out))) return cuda_fail(e, "record done");
+  if ((e = cudaStreamWaitEvent(st, hp->out_done, 0))) return cuda_fail(e, "join stream");
   return LSH_OK;
 }
 
