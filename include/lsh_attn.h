@@ -113,7 +113,11 @@ LSH_ATTN_API lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, co
  *   undo    [B, H, n_h, L]  int32 out, may be NULL: undo[.., perm[.., s]] = s.
  *   counts  [B, H, n_h, n_b] int32 out, may be NULL: tokens per bucket.
  * Bucket ids outside [0, n_b) are undefined behaviour (stage 1 never makes
- * them); the kernel does not read or write out of bounds for them.
+ * them); the kernels do not read or write out of bounds for them.
+ * The call takes n_h * B * H * ceil(L / 2048) * n_b * 4 bytes of temporary
+ * device memory from the device's stream-ordered pool (cudaMallocAsync on
+ * `stream`, freed on `stream` after use); a failed allocation returns
+ * LSH_ERR_CUDA.  The fused calls take it from their workspace instead.
  * ---------------------------------------------------------------------- */
 LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
                          int32_t* undo, int32_t* counts, void* stream);

@@ -34,7 +34,7 @@ lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null = false
 lsh_status check_rotations(const Problem& p, const void* rot);
 // Byte offsets of the fused pass's intermediates inside its workspace.
 struct Workspace {
-  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, total;
+  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, sort_scratch, total;
 };
 Workspace workspace_layout(const Problem& p);
 // Stages 1-4 into a checked workspace of workspace_layout(p).total bytes.
@@ -53,8 +53,10 @@ cudaError_t launch_hash_tc(const Problem& p, const void* qk, const void* rot, in
                            float* inv_norm, cudaStream_t st);
 
 // ---- stage 2: sort -------------------------------------------------------
+// Device scratch the sort needs (per-tile bucket counts), in bytes.
+size_t sort_scratch_bytes(const Problem& p);
 cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int32_t* undo,
-                        int32_t* counts, cudaStream_t st);
+                        int32_t* counts, void* scratch, cudaStream_t st);
 
 // ---- stage 3: chunked attention --------------------------------------------
 cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,

@@ -106,8 +106,8 @@ lsh_status run_hash(const Problem& p, const void* qk, const void* rot, int16_t* 
 }
 
 lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int32_t* undo,
-                    int32_t* counts, cudaStream_t st) {
-  cudaError_t e = launch_sort(p, buckets, perm, undo, counts, st);
+                    int32_t* counts, void* scratch, cudaStream_t st) {
+  cudaError_t e = launch_sort(p, buckets, perm, undo, counts, scratch, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
 }
 
@@ -138,6 +138,7 @@ Workspace workspace_layout(const Problem& p) {
   w.perm = off;       off += align256(slots * sizeof(int32_t));
   w.o_rounds = off;   off += align256(slots * p.d * p.elem());
   w.lse_rounds = off; off += align256(slots * sizeof(float));
+  w.sort_scratch = off; off += align256(sort_scratch_bytes(p));
   w.total = off;
   return w;
 }
@@ -152,7 +153,7 @@ lsh_status forward_body(const Problem& p, const void* qk, const void* v, const v
   void* o_r = base + w.o_rounds;
   float* lse_r = reinterpret_cast<float*>(base + w.lse_rounds);
   CHECK(run_hash(p, qk, rot, buckets, inv_norm, st));
-  CHECK(run_sort(p, buckets, perm, nullptr, nullptr, st));
+  CHECK(run_sort(p, buckets, perm, nullptr, nullptr, base + w.sort_scratch, st));
   CHECK(run_attn(p, qk, v, inv_norm, perm, o_r, lse_r, st));
   CHECK(run_combine(p, o_r, lse_r, out, lse, st));
   return LSH_OK;
@@ -249,7 +250,16 @@ lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t
   CHECK(check_ptr(perm, "perm"));
   CHECK(check_ptr(undo, "undo", true));
   CHECK(check_ptr(counts, "counts", true));
-  return run_sort(p, buckets, perm, undo, counts, static_cast<cudaStream_t>(stream));
+  // The per-tile counts live in stream-ordered scratch from the device's
+  // memory pool, released on the same stream once the sort has used them.
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  void* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(&scratch, sort_scratch_bytes(p), st);
+  if (e != cudaSuccess) return cuda_fail(e, "sort scratch");
+  const lsh_status r = run_sort(p, buckets, perm, undo, counts, scratch, st);
+  e = cudaFreeAsync(scratch, st);
+  if (r != LSH_OK) return r;
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort scratch release");
 }
 
 lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,

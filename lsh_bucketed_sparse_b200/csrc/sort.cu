@@ -5,14 +5,16 @@
 // A "Implementation").
 //
 // Positions already increase in input order, so one stable counting pass on
-// the bucket id gives the full key order (a single radix digit).  One CTA
-// sorts one segment of L keys:
-//   1. the segment is split into W contiguous owner ranges (one per warp);
-//      a shared-memory histogram counts each owner's keys per bucket;
-//   2. per bucket, an exclusive scan over owners, then an exclusive scan of
-//      the bucket totals, gives every (owner, bucket) its first output slot;
-//   3. each owner warp walks its range in order, 32 keys at a time; equal
-//      keys inside the warp are ranked with __match_any_sync, so equal
+// the bucket id gives the full key order (a single radix digit).  Each
+// segment of L keys is cut into tiles of kTileKeys keys, so the work spreads
+// over every SM:
+//   1. count: one CTA per tile counts its keys per bucket (shared-memory
+//      histogram) into cnt[segment][tile][bucket];
+//   2. scan: one CTA per segment turns the counts into each (tile, bucket)'s
+//      first output slot: an exclusive scan over tiles per bucket plus the
+//      bucket's start (exclusive scan of the bucket totals);
+//   3. scatter: one warp per tile walks its keys in order, 32 at a time;
+//      equal keys inside the warp are ranked with __match_any_sync, so equal
 //      buckets keep position order (stability) without global atomics.
 #include "common.cuh"
 #include "internal.h"
@@ -20,13 +22,37 @@
 namespace lsh {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kBatch = 16;  // keys per thread loaded ahead
-constexpr int kMaxSmem = 227 * 1024 - 1024;  // leave room for static shared memory
+constexpr int kTileKeys = 2048;
+constexpr int kCountThreads = 256;
+constexpr int kScanThreads = 1024;
+constexpr int kBatch = 16;  // rows of 32 keys loaded ahead in the scatter
 
-// Exclusive scan of a[0..n) in place by the whole block; returns nothing.
+__global__ void __launch_bounds__(kCountThreads)
+sort_count_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ cnt, int L,
+                  int n_b, int T) {
+  extern __shared__ int32_t hist[];  // [n_b]
+  const int seg = blockIdx.x, tile = blockIdx.y;
+  for (int b = threadIdx.x; b < n_b; b += blockDim.x) hist[b] = 0;
+  __syncthreads();
+  const int16_t* keys = buckets + (size_t)seg * L;
+  const int beg = tile * kTileKeys, end = min(L, beg + kTileKeys);
+  int kb[kTileKeys / kCountThreads];
+#pragma unroll
+  for (int i = 0; i < kTileKeys / kCountThreads; ++i) {
+    const int e = beg + i * kCountThreads + threadIdx.x;
+    kb[i] = e < end ? (int)keys[e] : -1;
+  }
+#pragma unroll
+  for (int i = 0; i < kTileKeys / kCountThreads; ++i)
+    if ((unsigned)kb[i] < (unsigned)n_b) atomicAdd(&hist[kb[i]], 1);
+  __syncthreads();
+  int32_t* out = cnt + ((size_t)seg * T + tile) * n_b;
+  for (int b = threadIdx.x; b < n_b; b += blockDim.x) out[b] = hist[b];
+}
+
+// Exclusive scan of a[0..n) in place by the whole block.
 __device__ void block_exclusive_scan(int32_t* a, int n) {
-  __shared__ int32_t warp_tot[kThreads / 32];
+  __shared__ int32_t warp_tot[kScanThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int per = (n + blockDim.x - 1) / blockDim.x;
   const int lo = min(n, tid * per), hi = min(n, lo + per);
@@ -61,107 +87,102 @@ __device__ void block_exclusive_scan(int32_t* a, int n) {
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kThreads)
-sort_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ perm,
-            int32_t* __restrict__ undo, int32_t* __restrict__ counts, int L, int n_b, int W) {
-  extern __shared__ int32_t sh[];  // [W][n_b] owner offsets, then [n_b] totals if W > 1
-  const size_t seg = blockIdx.x;
-  const int16_t* keys = buckets + seg * L;
-  int32_t* P = perm + seg * L;
-  int32_t* U = undo ? undo + seg * L : nullptr;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  int32_t* tot = (W > 1) ? sh + (size_t)W * n_b : sh;
-  const int len = (((L + W - 1) / W) + 31) & ~31;  // owner range, a multiple of 32
-
-  for (int t = tid; t < W * n_b; t += blockDim.x) sh[t] = 0;
+// cnt[seg][t][b] -> first output slot of tile t's keys of bucket b.
+__global__ void __launch_bounds__(kScanThreads)
+sort_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ counts, int n_b, int T) {
+  extern __shared__ int32_t base[];  // [n_b]
+  const int seg = blockIdx.x;
+  int32_t* c = cnt + (size_t)seg * T * n_b;
+  for (int b = threadIdx.x; b < n_b; b += blockDim.x) {
+    int32_t run = 0;
+    for (int t = 0; t < T; ++t) {
+      const int32_t x = c[(size_t)t * n_b + b];
+      c[(size_t)t * n_b + b] = run;
+      run += x;
+    }
+    base[b] = run;
+    if (counts) counts[(size_t)seg * n_b + b] = run;
+  }
   __syncthreads();
-  // kBatch loads in flight per thread before their counts, so the loop pays
-  // the memory latency once per batch rather than once per key
-  for (int e0 = tid; e0 < L; e0 += kBatch * blockDim.x) {
+  block_exclusive_scan(base, n_b);  // base[b] = first slot of bucket b
+  for (int b = threadIdx.x; b < n_b; b += blockDim.x) {
+    const int32_t x = base[b];
+    for (int t = 0; t < T; ++t) c[(size_t)t * n_b + b] += x;
+  }
+}
+
+__global__ void __launch_bounds__(32)
+sort_scatter_kernel(const int16_t* __restrict__ buckets, const int32_t* __restrict__ cnt,
+                    int32_t* __restrict__ perm, int32_t* __restrict__ undo, int L, int n_b,
+                    int T) {
+  extern __shared__ int32_t off[];  // [n_b]
+  const int seg = blockIdx.x, tile = blockIdx.y, lane = threadIdx.x;
+  const int32_t* c = cnt + ((size_t)seg * T + tile) * n_b;
+  for (int b = lane; b < n_b; b += 32) off[b] = c[b];
+  __syncwarp();
+  const int16_t* keys = buckets + (size_t)seg * L;
+  int32_t* P = perm + (size_t)seg * L;
+  int32_t* U = undo ? undo + (size_t)seg * L : nullptr;
+  const int beg = tile * kTileKeys, end = min(L, beg + kTileKeys);
+  for (int base0 = beg; base0 < end; base0 += 32 * kBatch) {
     int kb[kBatch];
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int e = e0 + i * blockDim.x;
-      kb[i] = e < L ? (int)keys[e] : -1;
+      const int e = base0 + 32 * i + lane;
+      kb[i] = (e < end) ? (int)keys[e] : -1 - lane;
     }
 #pragma unroll
     for (int i = 0; i < kBatch; ++i) {
-      const int e = e0 + i * blockDim.x;
-      if ((unsigned)kb[i] < (unsigned)n_b) atomicAdd(&sh[(e / len) * n_b + kb[i]], 1);
-    }
-  }
-  __syncthreads();
-  if (W > 1) {
-    for (int b = tid; b < n_b; b += blockDim.x) {
-      int32_t run = 0;
-      for (int o = 0; o < W; ++o) {
-        const int32_t t = sh[o * n_b + b];
-        sh[o * n_b + b] = run;
-        run += t;
+      const int e = base0 + 32 * i + lane;
+      const int b = kb[i];
+      const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
+      const unsigned peers = __match_any_sync(0xffffffffu, b);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      int slot = 0;
+      if (valid) slot = off[b] + rank;
+      __syncwarp();
+      if (valid) {
+        P[slot] = e;
+        if (U) U[e] = slot;
+        if (lane == 31 - __clz(peers)) off[b] += __popc(peers);
       }
-      tot[b] = run;
-    }
-    __syncthreads();
-  }
-  if (counts)
-    for (int b = tid; b < n_b; b += blockDim.x) counts[seg * n_b + b] = tot[b];
-  __syncthreads();
-  block_exclusive_scan(tot, n_b);  // tot[b] = first slot of bucket b
-  if (W > 1) {
-    for (int t = tid; t < W * n_b; t += blockDim.x) sh[t] += tot[t % n_b];
-    __syncthreads();
-  }
-
-  if (warp < W) {
-    int32_t* off = sh + (size_t)warp * n_b;
-    const int beg = warp * len, end = min(L, beg + len);
-    for (int base0 = beg; base0 < end; base0 += 32 * kBatch) {
-      // the next kBatch rows of 32 keys, loaded ahead of their ranking
-      int kb[kBatch];
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int e = base0 + 32 * i + lane;
-        kb[i] = (e < end) ? (int)keys[e] : -1 - lane;
-      }
-#pragma unroll
-      for (int i = 0; i < kBatch; ++i) {
-        const int e = base0 + 32 * i + lane;
-        const int b = kb[i];
-        const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
-        const unsigned peers = __match_any_sync(0xffffffffu, b);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        int slot = 0;
-        if (valid) slot = off[b] + rank;
-        __syncwarp();
-        if (valid) {
-          P[slot] = e;
-          if (U) U[e] = slot;
-          if (lane == 31 - __clz(peers)) off[b] += __popc(peers);
-        }
-        __syncwarp();
-      }
+      __syncwarp();
     }
   }
 }
 
 }  // namespace
 
+size_t sort_scratch_bytes(const Problem& p) {
+  const size_t T = (size_t)(p.L + kTileKeys - 1) / kTileKeys;
+  return (size_t)p.BH() * p.n_h * T * p.n_b * sizeof(int32_t);
+}
+
 cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int32_t* undo,
-                        int32_t* counts, cudaStream_t st) {
+                        int32_t* counts, void* scratch, cudaStream_t st) {
   const int n_b = p.n_b;
-  const long long per = (long long)n_b * 4;
-  int W = (int)((kMaxSmem - per) / per);
-  if (W > kThreads / 32) W = kThreads / 32;
-  const int max_owners = (p.L + 31) / 32;
-  if (W > max_owners) W = max_owners;
-  if (W < 2) W = 1;
-  const size_t smem = (size_t)(W > 1 ? W + 1 : 1) * per;
-  if (smem > (size_t)kMaxSmem) return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
-  if (e != cudaSuccess) return e;
+  const size_t hist_bytes = (size_t)n_b * sizeof(int32_t);
+  if (hist_bytes > 200 * 1024) return cudaErrorInvalidValue;
+  const int T = (p.L + kTileKeys - 1) / kTileKeys;
   const unsigned segs = (unsigned)((long long)p.BH() * p.n_h);
-  sort_kernel<<<segs, kThreads, smem, st>>>(buckets, perm, undo, counts, p.L, n_b, W);
+  if (T > 65535) return cudaErrorInvalidValue;
+  int32_t* cnt = static_cast<int32_t*>(scratch);
+  cudaError_t e;
+  if (hist_bytes > 48 * 1024) {
+    if ((e = cudaFuncSetAttribute(sort_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)hist_bytes)))
+      return e;
+    if ((e = cudaFuncSetAttribute(sort_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)hist_bytes)))
+      return e;
+    if ((e = cudaFuncSetAttribute(sort_scatter_kernel,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes)))
+      return e;
+  }
+  sort_count_kernel<<<dim3(segs, T), kCountThreads, hist_bytes, st>>>(buckets, cnt, p.L, n_b, T);
+  sort_scan_kernel<<<segs, kScanThreads, hist_bytes, st>>>(cnt, counts, n_b, T);
+  sort_scatter_kernel<<<dim3(segs, T), 32, hist_bytes, st>>>(buckets, cnt, perm, undo, p.L, n_b,
+                                                              T);
   return cudaGetLastError();
 }
 
