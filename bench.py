@@ -106,55 +106,80 @@ def traffic_for(stage, workload):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks and throttle reasons, sampled every 50 ms from before
+    the timed region to its end; summary() keeps the samples whose own
+    timestamps fall inside the region marked with start() / stop()."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
         self.proc = None
+        self.lines = []
+        self.t0 = self.t1 = None
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            if ln.strip():
+                self.lines.append(ln.strip())
 
     def __enter__(self):
+        import threading
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True, bufsize=1)
         except OSError:
             self.proc = None
+            return self
+        self.reader = threading.Thread(target=self._read, daemon=True)
+        self.reader.start()
+        t_end = time.time() + 3.0  # until nvidia-smi is producing samples
+        while not self.lines and time.time() < t_end:
+            time.sleep(0.01)
         return self
 
+    def start(self):
+        self.t0 = datetime.datetime.now()
+
+    def stop(self):
+        self.t1 = datetime.datetime.now()
+
     def __exit__(self, *a):
-        self.lines = []
         if self.proc is not None:
-            time.sleep(0.25)
+            time.sleep(0.1)  # the sample that covers the end of the region
             self.proc.terminate()
             try:
-                out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+                self.proc.wait()
+            self.reader.join(timeout=5)
 
     def summary(self):
         rows = []
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
                 continue
             try:
-                rows.append((float(f[1]), float(f[2]), f))
+                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f")
+                rows.append((ts, float(f[2]), float(f[3]), f[1:]))
             except ValueError:
                 continue
         if not rows:
             return None
-        max_mhz = max(r[1] for r in rows)
-        loaded = [r for r in rows if r[0] >= 0.5 * max_mhz] or rows
+        if self.t0 is not None and self.t1 is not None:
+            pad = datetime.timedelta(milliseconds=60)
+            inside = [r for r in rows if self.t0 <= r[0] <= self.t1 + pad]
+            rows = inside or rows
+        max_mhz = max(r[2] for r in rows)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[k] for r in rows for k in range(4)
-                          if r[2][5 + k].lower().startswith("active")})
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max_mhz,
+                          if r[3][5 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[1] for r in rows), "sm_max_mhz": max_mhz,
                 "reasons": reasons, "samples": len(rows)}
 
 
@@ -308,13 +333,16 @@ def run_one_stage(args, wl):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=list(W.BY_NAME))
     ap.add_argument("--cpu-rounds", type=int, default=2,
                     help="hashing rounds of one head the CPU baseline times")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--dedup", action="store_true",
+                    help="the pass with the duplicate-count correction (CUDA-core attention); "
+                         "a separate measurement, not the headline")
     ap.add_argument("--only-stage", choices=["hash", "sort", "chunked_attention", "combine"],
                     help="time one stage call alone (for profiling); prints its own JSON line")
     args = ap.parse_args(argv)
@@ -335,7 +363,7 @@ def main(argv=None):
     qk, v = qk_h.to(dev), v_h.to(dev)
     rot = rot_h.to(dev) if rot_h is not None else None
     shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
-                         wl.chunk_len, wl.causal, wl.dtype)
+                         wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup)
     ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
     out = torch.empty_like(qk)
     lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
@@ -343,7 +371,7 @@ def main(argv=None):
 
     def step():
         lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
-                             workspace=ws, out=out, lse=lse)
+                             workspace=ws, out=out, lse=lse, dedup=args.dedup)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -355,12 +383,14 @@ def main(argv=None):
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local) as clocks:
+        clocks.start()
         for k in range(args.steps):
             flush.fill_(float(k))
             starts[k].record(stream)
             step()
             ends[k].record(stream)
         torch.cuda.synchronize()
+        clocks.stop()
     barrier(world)
     lsh.lsh_attn_device_check()
     ms_local = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
@@ -377,10 +407,14 @@ def main(argv=None):
         ev[0].record(stream)
         b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
         ev[1].record(stream)
-        perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+        perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=args.dedup)
         ev[2].record(stream)
-        o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
-                                            n_buckets=wl.n_buckets)
+        if args.dedup:
+            o_r, l_r = lsh.lsh_attn_chunked_fwd_dedup(qk, v, inv, perm, undo, wl.chunk_len,
+                                                      wl.causal, n_buckets=wl.n_buckets)
+        else:
+            o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                                n_buckets=wl.n_buckets)
         ev[3].record(stream)
         lsh.lsh_attn_combine(o_r, l_r)
         ev[4].record(stream)
@@ -388,7 +422,7 @@ def main(argv=None):
         if it >= 2:
             for j, k in enumerate(stage_ms):
                 stage_ms[k] += ev[j].elapsed_time(ev[j + 1]) / n_stage
-        del b, inv, perm, o_r, l_r
+        del b, inv, perm, undo, o_r, l_r
 
     # End to end through the host-buffer entry point: copies in and out timed.
     pin = [t.pin_memory() if t is not None else None for t in (qk_h, v_h, rot_h)]
@@ -433,7 +467,7 @@ def main(argv=None):
     roofline["pass_frac"] = t_roof * 1e3 / ms_per_step
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.dedup:
         cpu = cpu_baseline(wl, args.cpu_rounds)
 
     if rank == 0:
@@ -443,12 +477,15 @@ def main(argv=None):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
             "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
-                           parallelism=f"independent (batch, head) problems, 1 per GPU x{world}"),
+                           parallelism=f"independent (batch, head) problems, 1 per GPU x{world}",
+                           **({"variant": "duplicate-count correction (LSH_FLAG_DEDUP), "
+                                          "CUDA-core attention"} if args.dedup else {})),
             "clocks": clocks.summary(),
             "e2e": {"value": world * wl.tokens / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            "gpu_launches": 4 * args.steps,
+            # per forward: hash 1, sort 3 (count, scan, scatter), attention 1, combine 1
+            "gpu_launches": 6 * args.steps,
             "roofline": roofline,
             "cpu_baseline": cpu,
         }

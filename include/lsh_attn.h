@@ -70,6 +70,17 @@ typedef enum lsh_dtype {
 #define LSH_FLAG_PORTABLE 1u   /* use the CUDA-core kernels even where the
                                   tensor-core (tcgen05) kernels apply; for
                                   cross-checking the two kernel families   */
+#define LSH_FLAG_DEDUP 2u      /* duplicate-count correction ("Reformer: The
+                                  Efficient Transformer", Appendix A "Multi-
+                                  round LSH attention"): a key that falls in
+                                  a query's window in N rounds has log N
+                                  subtracted from its score in each of them,
+                                  so the combined output weighs every
+                                  distinct key once.  N counts the rounds r
+                                  with chunk(undo_r[i]) - chunk(undo_r[j]) in
+                                  {0, 1}.  Runs on the CUDA-core attention
+                                  kernel; the stage call is
+                                  lsh_attn_chunked_fwd_dedup.              */
 
 typedef struct lsh_shape {
   int32_t batch;       /* B >= 1                                             */
@@ -139,6 +150,18 @@ LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buc
 LSH_ATTN_API lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,
                                 const float* inv_norm, const int32_t* perm, void* o_rounds,
                                 float* lse_rounds, void* stream);
+
+/* ---------------------------------------------------------------------- *
+ * Stage 3 with the duplicate-count correction (LSH_FLAG_DEDUP; the flag is
+ * implied here): as lsh_attn_chunked_fwd, plus
+ *   undo [B, H, n_h, L] int32 in: every round's inverse permutation (the
+ *        undo output of lsh_attn_sort), from which the kernel counts, for
+ *        each (query, key) pair, the rounds whose window holds the pair.
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_chunked_fwd_dedup(const lsh_shape* shape, const void* qk,
+                                      const void* v, const float* inv_norm,
+                                      const int32_t* perm, const int32_t* undo,
+                                      void* o_rounds, float* lse_rounds, void* stream);
 
 /* ---------------------------------------------------------------------- *
  * Stage 4: combine.  Appendix A "Multi-round attention": each round's output

@@ -9,6 +9,12 @@
 // time, one key per lane for the score, with an online softmax; the value
 // accumulation gives each lane the output dimensions lane, lane + 32, ...
 // The result is stored at the query's original position.
+//
+// With `undo` (the duplicate-count correction of Appendix A "Multi-round LSH
+// attention"), the score of key j for query i loses log N_ij, N_ij = the
+// number of rounds r' in which j sits in i's window, i.e. in which
+// chunk(undo_r'[i]) - chunk(undo_r'[j]) is 0 or 1; the self pair keeps its
+// replacement score.
 #include "common.cuh"
 #include "internal.h"
 
@@ -22,8 +28,9 @@ template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                      const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
-                     T* __restrict__ o_rounds, float* __restrict__ lse_rounds, int L, int d,
-                     int n_h, int c, int causal, float scale) {
+                     const int32_t* __restrict__ undo, T* __restrict__ o_rounds,
+                     float* __restrict__ lse_rounds, int L, int d, int n_h, int c, int causal,
+                     float scale) {
   extern __shared__ float q_all[];  // [kWarps][d]
   const int n_c = L / c;
   const int k = (int)(blockIdx.x % n_c);
@@ -34,6 +41,7 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   const T* X = qk + bh * (size_t)L * d;
   const T* V = v + bh * (size_t)L * d;
   const float* IN = inv_norm + bh * (size_t)L;
+  const int32_t* UD = undo ? undo + bh * (size_t)n_h * L : nullptr;  // [n_h][L]
   float* qs = q_all + warp * d;
   const int k0 = k > 0 ? (k - 1) * c : 0, k1 = (k + 1) * c;
   constexpr int kPer = kMaxD / 32;
@@ -60,6 +68,14 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
           const T* xj = X + (size_t)j * d;
           for (int e = 0; e < d; ++e) dot = fmaf(qs[e], to_f32(xj[e]), dot);
           s = dot * IN[j] * scale;
+          if (UD) {
+            int n = 0;
+            for (int rr = 0; rr < n_h; ++rr) {
+              const int dc = UD[(size_t)rr * L + i] / c - UD[(size_t)rr * L + j] / c;
+              n += (dc == 0 || dc == 1) ? 1 : 0;
+            }
+            s -= logf((float)n);
+          }
         }
       }
       const float mnew = fmaxf(m, warp_max(s));
@@ -97,19 +113,21 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
 }  // namespace
 
 cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,
-                                 const float* inv_norm, const int32_t* perm, void* o_rounds,
-                                 float* lse_rounds, cudaStream_t st) {
+                                 const float* inv_norm, const int32_t* perm,
+                                 const int32_t* undo, void* o_rounds, float* lse_rounds,
+                                 cudaStream_t st) {
+  if (!p.dedup) undo = nullptr;
   if (p.d > kMaxD) return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
   const size_t smem = (size_t)kWarps * p.d * sizeof(float);
   const float scale = 1.0f / sqrtf((float)p.d);
   if (p.bf16)
     attn_portable_kernel<__nv_bfloat16><<<grid, kWarps * 32, smem, st>>>(
-        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm,
+        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm, undo,
         (__nv_bfloat16*)o_rounds, lse_rounds, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
   else
     attn_portable_kernel<float><<<grid, kWarps * 32, smem, st>>>(
-        (const float*)qk, (const float*)v, inv_norm, perm, (float*)o_rounds, lse_rounds, p.L,
+        (const float*)qk, (const float*)v, inv_norm, perm, undo, (float*)o_rounds, lse_rounds, p.L,
         p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
   return cudaGetLastError();
 }

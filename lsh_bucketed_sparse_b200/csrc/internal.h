@@ -16,6 +16,7 @@ struct Problem {
   bool causal;
   bool bf16;         // element type of qk, v, rotations, out, o_rounds
   bool portable;     // LSH_FLAG_PORTABLE: CUDA-core kernels only
+  bool dedup;        // LSH_FLAG_DEDUP: duplicate-count correction
   int BH() const { return B * H; }
   int half() const { return n_b / 2; }  // projections per round, 0 when n_b == 1
   int n_chunks() const { return L / c; }
@@ -34,7 +35,7 @@ lsh_status check_ptr(const void* ptr, const char* name, bool may_be_null = false
 lsh_status check_rotations(const Problem& p, const void* rot);
 // Byte offsets of the fused pass's intermediates inside its workspace.
 struct Workspace {
-  size_t buckets, inv_norm, perm, o_rounds, lse_rounds, sort_scratch, total;
+  size_t buckets, inv_norm, perm, undo, o_rounds, lse_rounds, sort_scratch, total;
 };
 Workspace workspace_layout(const Problem& p);
 // Stages 1-4 into a checked workspace of workspace_layout(p).total bytes.
@@ -59,9 +60,11 @@ cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm,
                         int32_t* counts, void* scratch, cudaStream_t st);
 
 // ---- stage 3: chunked attention --------------------------------------------
+// undo: every round's inverse permutation when p.dedup, else ignored.
 cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,
-                                 const float* inv_norm, const int32_t* perm, void* o_rounds,
-                                 float* lse_rounds, cudaStream_t st);
+                                 const float* inv_norm, const int32_t* perm,
+                                 const int32_t* undo, void* o_rounds, float* lse_rounds,
+                                 cudaStream_t st);
 bool attn_tc_supported(const Problem& p);
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                            const int32_t* perm, void* o_rounds, float* lse_rounds,

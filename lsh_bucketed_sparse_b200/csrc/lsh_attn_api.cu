@@ -56,7 +56,8 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   if (s->causal != 0 && s->causal != 1) return fail(LSH_ERR_INVALID_ARG, "causal must be 0 or 1");
   if (s->dtype != LSH_F32 && s->dtype != LSH_BF16)
     return fail(LSH_ERR_INVALID_ARG, "dtype=%d: must be LSH_F32 or LSH_BF16", s->dtype);
-  if (s->flags & ~LSH_FLAG_PORTABLE) return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
+  if (s->flags & ~(LSH_FLAG_PORTABLE | LSH_FLAG_DEDUP))
+    return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
   const long long bh = (long long)s->batch * s->heads;
   if (bh > (1LL << 30)) return fail(LSH_ERR_INVALID_ARG, "batch*heads too large");
   const long long chunks = bh * s->n_hashes * (s->seq_len / s->chunk_len);
@@ -66,6 +67,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   p->n_h = s->n_hashes; p->n_b = s->n_buckets; p->c = s->chunk_len;
   p->causal = s->causal != 0; p->bf16 = s->dtype == LSH_BF16;
   p->portable = (s->flags & LSH_FLAG_PORTABLE) != 0;
+  p->dedup = (s->flags & LSH_FLAG_DEDUP) != 0;
   return LSH_OK;
 }
 
@@ -111,11 +113,13 @@ lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
 }
 
+// The duplicate-count correction runs on the CUDA-core kernel only.
 lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
-                    const int32_t* perm, void* o_r, float* lse_r, cudaStream_t st) {
-  cudaError_t e = (!p.portable && attn_tc_supported(p))
+                    const int32_t* perm, const int32_t* undo, void* o_r, float* lse_r,
+                    cudaStream_t st) {
+  cudaError_t e = (!p.portable && !p.dedup && attn_tc_supported(p))
                       ? launch_attn_tc(p, qk, v, inv_norm, perm, o_r, lse_r, st)
-                      : launch_attn_portable(p, qk, v, inv_norm, perm, o_r, lse_r, st);
+                      : launch_attn_portable(p, qk, v, inv_norm, perm, undo, o_r, lse_r, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
 }
 
@@ -136,6 +140,7 @@ Workspace workspace_layout(const Problem& p) {
   w.buckets = off;    off += align256(slots * sizeof(int16_t));
   w.inv_norm = off;   off += align256((size_t)p.BH() * p.L * sizeof(float));
   w.perm = off;       off += align256(slots * sizeof(int32_t));
+  w.undo = off;       off += p.dedup ? align256(slots * sizeof(int32_t)) : 0;
   w.o_rounds = off;   off += align256(slots * p.d * p.elem());
   w.lse_rounds = off; off += align256(slots * sizeof(float));
   w.sort_scratch = off; off += align256(sort_scratch_bytes(p));
@@ -153,8 +158,9 @@ lsh_status forward_body(const Problem& p, const void* qk, const void* v, const v
   void* o_r = base + w.o_rounds;
   float* lse_r = reinterpret_cast<float*>(base + w.lse_rounds);
   CHECK(run_hash(p, qk, rot, buckets, inv_norm, st));
-  CHECK(run_sort(p, buckets, perm, nullptr, nullptr, base + w.sort_scratch, st));
-  CHECK(run_attn(p, qk, v, inv_norm, perm, o_r, lse_r, st));
+  int32_t* undo = p.dedup ? reinterpret_cast<int32_t*>(base + w.undo) : nullptr;
+  CHECK(run_sort(p, buckets, perm, undo, nullptr, base + w.sort_scratch, st));
+  CHECK(run_attn(p, qk, v, inv_norm, perm, undo, o_r, lse_r, st));
   CHECK(run_combine(p, o_r, lse_r, out, lse, st));
   return LSH_OK;
 }
@@ -273,7 +279,28 @@ lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const vo
   CHECK(check_ptr(perm, "perm"));
   CHECK(check_ptr(o_rounds, "o_rounds"));
   CHECK(check_ptr(lse_rounds, "lse_rounds"));
-  return run_attn(p, qk, v, inv_norm, perm, o_rounds, lse_rounds,
+  if (p.dedup)
+    return fail(LSH_ERR_INVALID_ARG,
+                "LSH_FLAG_DEDUP needs every round's undo: call lsh_attn_chunked_fwd_dedup");
+  return run_attn(p, qk, v, inv_norm, perm, nullptr, o_rounds, lse_rounds,
+                  static_cast<cudaStream_t>(stream));
+}
+
+lsh_status lsh_attn_chunked_fwd_dedup(const lsh_shape* shape, const void* qk, const void* v,
+                                      const float* inv_norm, const int32_t* perm,
+                                      const int32_t* undo, void* o_rounds, float* lse_rounds,
+                                      void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  CHECK(check_ptr(qk, "qk"));
+  CHECK(check_ptr(v, "v"));
+  CHECK(check_ptr(inv_norm, "inv_norm"));
+  CHECK(check_ptr(perm, "perm"));
+  CHECK(check_ptr(undo, "undo"));
+  CHECK(check_ptr(o_rounds, "o_rounds"));
+  CHECK(check_ptr(lse_rounds, "lse_rounds"));
+  p.dedup = true;
+  return run_attn(p, qk, v, inv_norm, perm, undo, o_rounds, lse_rounds,
                   static_cast<cudaStream_t>(stream));
 }
 

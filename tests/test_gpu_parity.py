@@ -6,6 +6,7 @@ floating-point outputs within the tolerances in ``parity.py``.  The fused
 ``lsh_attn_forward`` must equal the four stage calls bit for bit.
 """
 
+import ctypes
 import math
 
 import numpy as np
@@ -317,3 +318,76 @@ def test_sharded_ranks_concatenate_to_the_full_pass():
         lses.append(l[0])
     assert torch.equal(torch.cat(outs), full_out.reshape(6, *full_out.shape[2:]))
     assert torch.equal(torch.cat(lses), full_lse.reshape(6, -1))
+
+
+# ---------------------------------------------------------------------------
+# Duplicate-count correction (LSH_FLAG_DEDUP): few buckets, so pairs share a
+# window in several rounds and N_ij > 1 is common.
+DEDUP = [
+    W.small("dedup-bf16-causal", heads=2, seq_len=512, n_hashes=4, n_buckets=8),
+    W.small("dedup-bf16-noncausal-d128", heads=2, seq_len=256, d_k=128, n_hashes=3,
+            n_buckets=4, chunk_len=32, causal=False),
+    W.small("dedup-f32-causal", heads=1, seq_len=256, n_hashes=3, n_buckets=8,
+            dtype=torch.float32),
+]
+
+
+@pytest.mark.parametrize("wl", DEDUP, ids=[w.name for w in DEDUP])
+def test_dedup_matches_oracle(wl):
+    qk, v, rot = W.make_inputs(wl)
+    qk_d, v_d = qk.to(DEV), v.to(DEV)
+    rot_d = rot.to(DEV)
+    b, inv = lsh.lsh_attn_hash(qk_d, rot_d, wl.n_buckets, wl.n_hashes)
+    perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets)
+    o_r, lse_r = lsh.lsh_attn_chunked_fwd_dedup(qk_d, v_d, inv, perm, undo, wl.chunk_len,
+                                               wl.causal, n_buckets=wl.n_buckets)
+    out, lse = lsh.lsh_attn_combine(o_r, lse_r)
+    f_out, f_lse = lsh.lsh_attn_forward(qk_d, v_d, rot_d, wl.n_hashes, wl.n_buckets,
+                                        wl.chunk_len, wl.causal, dedup=True)
+    lsh.lsh_attn_device_check()
+    # the fused pass runs the same kernels in the same order
+    assert torch.equal(f_out, out) and torch.equal(f_lse, lse)
+    # the correction is on: some pair shares a window in more than one round
+    res0 = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal,
+                     buckets=b.cpu().numpy().astype(np.int64))
+    res = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal,
+                    buckets=b.cpu().numpy().astype(np.int64), dedup=True)
+    assert np.abs(res["lse"] - res0["lse"]).max() > 1e-3
+    bf16 = wl.dtype == torch.bfloat16
+    P.check_float(o_r, res["o_rounds"], bf16, "o_rounds", 3)
+    P.check_lse(lse_r, res["lse_rounds"], bf16, "lse_rounds")
+    P.check_float(out, res["out"], bf16, "out")
+    P.check_lse(lse, res["lse"], bf16, "lse")
+
+
+def test_dedup_stage_call_needs_undo():
+    wl = DEDUP[0]
+    qk, v, rot = [t.to(DEV) for t in W.make_inputs(wl)]
+    b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+    perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype, dedup=True)
+    o_r = torch.empty(1, wl.heads, wl.n_hashes, wl.seq_len, wl.d_k, dtype=qk.dtype, device=DEV)
+    l_r = torch.empty(1, wl.heads, wl.n_hashes, wl.seq_len, dtype=torch.float32, device=DEV)
+    st = lsh.lib().lsh_attn_chunked_fwd(ctypes.byref(shp), lsh._ptr(qk), lsh._ptr(v),
+                                        lsh._ptr(inv), lsh._ptr(perm), lsh._ptr(o_r),
+                                        lsh._ptr(l_r), None)
+    assert st == 1  # LSH_ERR_INVALID_ARG: the flag needs every round's undo
+
+
+def test_host_pipeline_uneven_groups():
+    # 10 (batch, head) pairs go through 8 groups of one or two pairs each
+    wl = W.small("host-groups", batch=2, heads=5, seq_len=256, n_hashes=2, n_buckets=16)
+    qk, v, rot = W.make_inputs(wl)
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype)
+    dev = torch.empty(lsh.lsh_attn_forward_host_device_bytes(shp), dtype=torch.uint8,
+                      device=DEV)
+    out_h = torch.empty_like(qk).pin_memory()
+    lse_h = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32).pin_memory()
+    lsh.lsh_attn_forward_host(shp, qk.pin_memory(), v.pin_memory(), rot.pin_memory(), out_h,
+                              lse_h, dev)
+    torch.cuda.current_stream().synchronize()
+    ref_out, ref_lse = lsh.lsh_attn_forward(qk.to(DEV), v.to(DEV), rot.to(DEV), wl.n_hashes,
+                                            wl.n_buckets, wl.chunk_len, wl.causal)
+    assert torch.equal(out_h, ref_out.cpu()) and torch.equal(lse_h, ref_lse.cpu())
