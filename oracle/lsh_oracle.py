@@ -32,7 +32,10 @@ Readings where the pages are silent (each is also listed in the design notes):
   * n_buckets == 1 puts every token in bucket 0 and needs no rotations;
   * the first chunk of a round has no look-back (no wrap to the last chunk,
     no crossing into another round);
-  * no bucket-equality mask inside a window: the window is the attended set;
+  * no bucket-equality mask inside a window: the window is the attended set
+    (``bucket_mask=True`` is the variant that also drops the window's keys
+    whose bucket in that round differs from the query's, section 2 "LSH
+    attention": a query attends only to targets in its own hash bucket);
   * scores are (q . k_hat) / sqrt(d_k);
   * the self-mask REPLACES the score of j == i by SELF_SCORE = -1e5, a finite
     penalty, so a token that sees only itself in every round outputs v_i;
@@ -115,13 +118,16 @@ def window_slots(k: int, chunk_len: int):
     return lo, (k + 1) * chunk_len
 
 
-def attend_round(x, v, perm_r, chunk_len: int, causal: bool, dedup_undo=None):
+def attend_round(x, v, perm_r, chunk_len: int, causal: bool, dedup_undo=None,
+                 bucket_r=None):
     """One hashing round: chunked attention in sorted order, results unsorted.
 
     x, v: [L, d] float64; perm_r: [L] sorted order of this round.
     Returns (o [L, d], lse [L]) indexed by ORIGINAL position.
     ``dedup_undo`` ([n_h, L] undo of every round) turns on the duplicate-count
-    correction of Appendix A.
+    correction of Appendix A.  ``bucket_r`` ([L] bucket of every position in
+    this round) turns on the bucket-equality mask: a key whose bucket differs
+    from the query's is not attended.
     """
     L, d = x.shape
     c = chunk_len
@@ -139,6 +145,8 @@ def attend_round(x, v, perm_r, chunk_len: int, causal: bool, dedup_undo=None):
         kp = pos[k0:k1][None, :]
         if dedup_undo is not None:
             s = s - np.log(duplicate_counts(dedup_undo, pos[q0:q1], pos[k0:k1], c))
+        if bucket_r is not None:
+            s = np.where(bucket_r[kp] != bucket_r[qp], -np.inf, s)
         s = np.where(kp == qp, SELF_SCORE, s)
         if causal:
             s = np.where(kp > qp, -np.inf, s)
@@ -216,8 +224,9 @@ def sort_all(buckets):
     return perm, undo
 
 
-def attend_all(qk, v, perm, chunk_len, causal, dedup=False):
-    """Per-round outputs at original positions: o [B,H,n_h,L,d], lse [B,H,n_h,L]."""
+def attend_all(qk, v, perm, chunk_len, causal, dedup=False, buckets=None):
+    """Per-round outputs at original positions: o [B,H,n_h,L,d], lse [B,H,n_h,L].
+    ``buckets`` ([B,H,n_h,L]) turns on the bucket-equality mask."""
     qk, v = as_f64(qk), as_f64(v)
     perm = np.asarray(perm)
     B, H, n_h, L = perm.shape
@@ -232,8 +241,9 @@ def attend_all(qk, v, perm, chunk_len, causal, dedup=False):
                 for r in range(n_h):
                     undo[r, perm[b, h, r]] = np.arange(L)
             for r in range(n_h):
+                bk = None if buckets is None else np.asarray(buckets)[b, h, r]
                 o[b, h, r], lse[b, h, r] = attend_round(qk[b, h], v[b, h], perm[b, h, r],
-                                                        chunk_len, causal, undo)
+                                                        chunk_len, causal, undo, bk)
     return o, lse
 
 
@@ -248,7 +258,8 @@ def combine_all(o_rounds, lse_rounds):
     return out, lse
 
 
-def forward(qk, v, rotations, n_buckets, chunk_len, causal, buckets=None, dedup=False):
+def forward(qk, v, rotations, n_buckets, chunk_len, causal, buckets=None, dedup=False,
+            bucket_mask=False):
     """The whole pass.  If ``buckets`` is given, hashing is skipped and those
     ids are used (this is how GPU bucket ids are fed back so that the later
     stages can be compared exactly).  Returns a dict of every intermediate."""
@@ -258,7 +269,8 @@ def forward(qk, v, rotations, n_buckets, chunk_len, causal, buckets=None, dedup=
         res["margins"] = margins
     buckets = np.asarray(buckets, np.int64)
     perm, undo = sort_all(buckets)
-    o_r, lse_r = attend_all(qk, v, perm, chunk_len, causal, dedup=dedup)
+    o_r, lse_r = attend_all(qk, v, perm, chunk_len, causal, dedup=dedup,
+                            buckets=buckets if bucket_mask else None)
     out, lse = combine_all(o_r, lse_r)
     res.update(buckets=buckets, perm=perm, undo=undo, o_rounds=o_r, lse_rounds=lse_r,
                out=out, lse=lse)

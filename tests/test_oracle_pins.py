@@ -362,3 +362,52 @@ def test_zero_norm_key_reads_as_zero_vector():
     v = np.arange(8.0).reshape(1, 1, 4, 2)
     res = O.forward(x, v, None, 1, 4, False, buckets=np.zeros((1, 1, 1, 4), np.int64))
     assert np.isfinite(res["out"]).all() and np.isfinite(res["lse"]).all()
+
+
+# ------------------------------------------------- bucket-equality mask --
+def test_bucket_mask_brute_force():
+    # The variant of section 2 "LSH attention" (a query attends only to keys
+    # in its own bucket), written from the set definition: for each query,
+    # loop over all positions and keep those in its window (same or previous
+    # chunk of the sorted order), in its bucket, not in its future; the self
+    # pair scores -1e5.
+    rng = np.random.default_rng(21)
+    L, d, c, n_h, n_b = 48, 8, 8, 2, 6
+    x = rng.standard_normal((1, 1, L, d))
+    v = rng.standard_normal((1, 1, L, d))
+    R = rng.standard_normal((n_h, d, n_b // 2))
+    for causal in (False, True):
+        res = O.forward(x, v, R, n_b, c, causal, bucket_mask=True)
+        xx, vv = x[0, 0], v[0, 0]
+        for r in range(n_h):
+            bk = res["buckets"][0, 0, r]
+            slot = res["undo"][0, 0, r]
+            for i in range(L):
+                keys, scores = [], []
+                for j in range(L):
+                    ci, cj = slot[i] // c, slot[j] // c
+                    if ci - cj not in (0, 1) or bk[j] != bk[i] or (causal and j > i):
+                        continue
+                    s = O.SELF_SCORE if j == i else \
+                        xx[i] @ (xx[j] / np.linalg.norm(xx[j])) / math.sqrt(d)
+                    keys.append(j)
+                    scores.append(s)
+                scores = np.array(scores)
+                m = scores.max()
+                w = np.exp(scores - m)
+                o = (w[:, None] * vv[keys]).sum(0) / w.sum()
+                np.testing.assert_allclose(res["o_rounds"][0, 0, r, i], o, rtol=1e-10, atol=1e-12)
+                np.testing.assert_allclose(res["lse_rounds"][0, 0, r, i], m + np.log(w.sum()),
+                                           rtol=1e-12, atol=1e-10)
+
+
+def test_bucket_mask_is_a_no_op_within_one_bucket():
+    rng = np.random.default_rng(22)
+    L, d, c, n_h = 64, 8, 16, 2
+    x = rng.standard_normal((1, 2, L, d))
+    v = rng.standard_normal((1, 2, L, d))
+    zero = np.zeros((1, 2, n_h, L), np.int64)
+    a = O.forward(x, v, None, 1, c, True, buckets=zero)
+    b = O.forward(x, v, None, 1, c, True, buckets=zero, bucket_mask=True)
+    np.testing.assert_array_equal(a["out"], b["out"])
+    np.testing.assert_array_equal(a["lse"], b["lse"])
