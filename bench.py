@@ -343,6 +343,9 @@ def main(argv=None):
     ap.add_argument("--dedup", action="store_true",
                     help="the pass with the duplicate-count correction (CUDA-core attention); "
                          "a separate measurement, not the headline")
+    ap.add_argument("--bucket-mask", action="store_true",
+                    help="the pass with the bucket-equality mask (CUDA-core attention); a "
+                         "separate measurement, not the headline")
     ap.add_argument("--only-stage", choices=["hash", "sort", "chunked_attention", "combine"],
                     help="time one stage call alone (for profiling); prints its own JSON line")
     args = ap.parse_args(argv)
@@ -363,7 +366,8 @@ def main(argv=None):
     qk, v = qk_h.to(dev), v_h.to(dev)
     rot = rot_h.to(dev) if rot_h is not None else None
     shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
-                         wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup)
+                         wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup,
+                         bucket_mask=args.bucket_mask)
     ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
     out = torch.empty_like(qk)
     lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
@@ -371,7 +375,8 @@ def main(argv=None):
 
     def step():
         lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
-                             workspace=ws, out=out, lse=lse, dedup=args.dedup)
+                             workspace=ws, out=out, lse=lse, dedup=args.dedup,
+                             bucket_mask=args.bucket_mask)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -409,9 +414,10 @@ def main(argv=None):
         ev[1].record(stream)
         perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=args.dedup)
         ev[2].record(stream)
-        if args.dedup:
-            o_r, l_r = lsh.lsh_attn_chunked_fwd_dedup(qk, v, inv, perm, undo, wl.chunk_len,
-                                                      wl.causal, n_buckets=wl.n_buckets)
+        if args.dedup or args.bucket_mask:
+            o_r, l_r = lsh.lsh_attn_chunked_fwd_ex(
+                qk, v, inv, perm, wl.chunk_len, wl.causal, undo=undo if args.dedup else None,
+                buckets=b if args.bucket_mask else None, n_buckets=wl.n_buckets)
         else:
             o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
                                                 n_buckets=wl.n_buckets)
@@ -467,7 +473,8 @@ def main(argv=None):
     roofline["pass_frac"] = t_roof * 1e3 / ms_per_step
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.dedup:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not (args.dedup or
+                                                                      args.bucket_mask):
         cpu = cpu_baseline(wl, args.cpu_rounds)
 
     if rank == 0:
@@ -478,8 +485,12 @@ def main(argv=None):
             "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
             "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
                            parallelism=f"independent (batch, head) problems, 1 per GPU x{world}",
-                           **({"variant": "duplicate-count correction (LSH_FLAG_DEDUP), "
-                                          "CUDA-core attention"} if args.dedup else {})),
+                           **({"variant": " + ".join(
+                               (["duplicate-count correction (LSH_FLAG_DEDUP)"] if args.dedup
+                                else []) +
+                               (["bucket-equality mask (LSH_FLAG_BUCKET_MASK)"]
+                                if args.bucket_mask else [])) + ", CUDA-core attention"}
+                              if (args.dedup or args.bucket_mask) else {})),
             "clocks": clocks.summary(),
             "e2e": {"value": world * wl.tokens / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

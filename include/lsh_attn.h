@@ -80,7 +80,14 @@ typedef enum lsh_dtype {
                                   with chunk(undo_r[i]) - chunk(undo_r[j]) in
                                   {0, 1}.  Runs on the CUDA-core attention
                                   kernel; the stage call is
-                                  lsh_attn_chunked_fwd_dedup.              */
+                                  lsh_attn_chunked_fwd_ex.                 */
+#define LSH_FLAG_BUCKET_MASK 4u /* bucket-equality mask (section 2 "LSH
+                                  attention": a query attends only to
+                                  targets in its own hash bucket): inside a
+                                  window, keys whose bucket in that round
+                                  differs from the query's are not attended.
+                                  Runs on the CUDA-core attention kernel;
+                                  the stage call is lsh_attn_chunked_fwd_ex. */
 
 typedef struct lsh_shape {
   int32_t batch;       /* B >= 1                                             */
@@ -152,16 +159,20 @@ LSH_ATTN_API lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void*
                                 float* lse_rounds, void* stream);
 
 /* ---------------------------------------------------------------------- *
- * Stage 3 with the duplicate-count correction (LSH_FLAG_DEDUP; the flag is
- * implied here): as lsh_attn_chunked_fwd, plus
- *   undo [B, H, n_h, L] int32 in: every round's inverse permutation (the
- *        undo output of lsh_attn_sort), from which the kernel counts, for
- *        each (query, key) pair, the rounds whose window holds the pair.
+ * Stage 3 for the variants (LSH_FLAG_DEDUP, LSH_FLAG_BUCKET_MASK, set in
+ * shape->flags): as lsh_attn_chunked_fwd, plus
+ *   undo    [B, H, n_h, L] int32 in, required with LSH_FLAG_DEDUP: every
+ *           round's inverse permutation (the undo output of lsh_attn_sort),
+ *           from which the kernel counts, for each (query, key) pair, the
+ *           rounds whose window holds the pair; else may be NULL.
+ *   buckets [B, H, n_h, L] int16 in, required with LSH_FLAG_BUCKET_MASK:
+ *           the bucket ids of stage 1; else may be NULL.
  * ---------------------------------------------------------------------- */
-LSH_ATTN_API lsh_status lsh_attn_chunked_fwd_dedup(const lsh_shape* shape, const void* qk,
-                                      const void* v, const float* inv_norm,
-                                      const int32_t* perm, const int32_t* undo,
-                                      void* o_rounds, float* lse_rounds, void* stream);
+LSH_ATTN_API lsh_status lsh_attn_chunked_fwd_ex(const lsh_shape* shape, const void* qk,
+                                   const void* v, const float* inv_norm,
+                                   const int32_t* perm, const int32_t* undo,
+                                   const int16_t* buckets, void* o_rounds,
+                                   float* lse_rounds, void* stream);
 
 /* ---------------------------------------------------------------------- *
  * Stage 4: combine.  Appendix A "Multi-round attention": each round's output

@@ -21,11 +21,11 @@ import torch
 
 __all__ = [
     "LshError", "Shape", "lib", "make_shape", "lsh_attn_hash", "lsh_attn_sort",
-    "lsh_attn_chunked_fwd", "lsh_attn_chunked_fwd_dedup", "lsh_attn_combine", "lsh_attn_forward",
+    "lsh_attn_chunked_fwd", "lsh_attn_chunked_fwd_ex", "lsh_attn_combine", "lsh_attn_forward",
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
     "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
     "LIB_PATH", "HEADER_PATH", "NOALLOC_SCRATCH_BYTES",
-    "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP",
+    "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP", "FLAG_BUCKET_MASK",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +35,7 @@ HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "lsh_attn.h")
 F32, BF16 = 0, 1
 FLAG_PORTABLE = 1
 FLAG_DEDUP = 2
+FLAG_BUCKET_MASK = 4
 NOALLOC_SCRATCH_BYTES = 64 << 20  # LSH_ATTN_NOALLOC_SCRATCH_BYTES
 STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED",
           3: "LSH_ERR_WORKSPACE", 4: "LSH_ERR_CUDA", 5: "LSH_ERR_DEVICE_TIMEOUT"}
@@ -62,7 +63,7 @@ _SIGS = {
     "lsh_attn_hash": [_SHP, _P, _P, _P, _P, _P],
     "lsh_attn_sort": [_SHP, _P, _P, _P, _P, _P],
     "lsh_attn_chunked_fwd": [_SHP, _P, _P, _P, _P, _P, _P, _P],
-    "lsh_attn_chunked_fwd_dedup": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P],
+    "lsh_attn_chunked_fwd_ex": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lsh_attn_combine": [_SHP, _P, _P, _P, _P, _P],
     "lsh_attn_forward_workspace_size": [_SHP, ctypes.POINTER(_SZ)],
     "lsh_attn_forward": [_SHP, _P, _P, _P, _P, _P, _P, _SZ, _P],
@@ -115,10 +116,11 @@ def _dtype_code(t: torch.dtype) -> int:
 
 
 def make_shape(batch, heads, seq_len, d_k, n_hashes, n_buckets, chunk_len, causal,
-               dtype=torch.bfloat16, portable=False, dedup=False) -> Shape:
+               dtype=torch.bfloat16, portable=False, dedup=False, bucket_mask=False) -> Shape:
     return Shape(batch, heads, seq_len, d_k, n_hashes, n_buckets, chunk_len, int(bool(causal)),
                  dtype if isinstance(dtype, int) else _dtype_code(dtype),
-                 (FLAG_PORTABLE if portable else 0) | (FLAG_DEDUP if dedup else 0))
+                 (FLAG_PORTABLE if portable else 0) | (FLAG_DEDUP if dedup else 0)
+                 | (FLAG_BUCKET_MASK if bucket_mask else 0))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -140,10 +142,11 @@ def _stream(stream):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup=False):
+def _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup=False,
+              bucket_mask=False):
     B, H, L, d = qk.shape
     return make_shape(B, H, L, d, n_hashes, n_buckets, chunk_len, causal, qk.dtype, portable,
-                      dedup)
+                      dedup, bucket_mask)
 
 
 # --------------------------------------------------------------------------
@@ -196,22 +199,28 @@ def lsh_attn_chunked_fwd(qk, v, inv_norm, perm, chunk_len, causal, *, n_buckets=
     return o_r, lse_r
 
 
-def lsh_attn_chunked_fwd_dedup(qk, v, inv_norm, perm, undo, chunk_len, causal, *,
-                               n_buckets=2, stream=None):
-    """Stage 3 with the duplicate-count correction (every round's ``undo``
-    [B,H,n_h,L] int32 from lsh_attn_sort).  Returns (o_rounds, lse_rounds)."""
+def lsh_attn_chunked_fwd_ex(qk, v, inv_norm, perm, chunk_len, causal, *, undo=None,
+                            buckets=None, n_buckets=2, stream=None):
+    """Stage 3 for the variants: the duplicate-count correction when ``undo``
+    (every round's [B,H,n_h,L] int32, from lsh_attn_sort) is given, the
+    bucket-equality mask when ``buckets`` ([B,H,n_h,L] int16) is given.
+    Returns (o_rounds, lse_rounds)."""
     _cuda(qk, "qk")
     _cuda(v, "v", qk.dtype)
     _cuda(inv_norm, "inv_norm", torch.float32)
     _cuda(perm, "perm", torch.int32)
-    _cuda(undo, "undo", torch.int32)
+    if undo is not None:
+        _cuda(undo, "undo", torch.int32)
+    if buckets is not None:
+        _cuda(buckets, "buckets", torch.int16)
     B, H, n_h, L = perm.shape
-    shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, False, True)
+    shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, False, undo is not None,
+                    buckets is not None)
     o_r = torch.empty(B, H, n_h, L, qk.shape[-1], dtype=qk.dtype, device=qk.device)
     lse_r = torch.empty(B, H, n_h, L, dtype=torch.float32, device=qk.device)
-    _check(lib().lsh_attn_chunked_fwd_dedup(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(inv_norm),
-                                            _ptr(perm), _ptr(undo), _ptr(o_r), _ptr(lse_r),
-                                            _stream(stream)))
+    _check(lib().lsh_attn_chunked_fwd_ex(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(inv_norm),
+                                         _ptr(perm), _ptr(undo), _ptr(buckets), _ptr(o_r),
+                                         _ptr(lse_r), _stream(stream)))
     return o_r, lse_r
 
 
@@ -236,7 +245,7 @@ def lsh_attn_forward_workspace_size(shape: Shape) -> int:
 
 def lsh_attn_forward(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *,
                      workspace=None, out=None, lse=None, portable=False, dedup=False,
-                     stream=None):
+                     bucket_mask=False, stream=None):
     """The fused pass.  Returns (out [B,H,L,d], lse f32 [B,H,L]).  ``workspace`` (a
     uint8 CUDA tensor) can be passed in to avoid an allocation per call."""
     _cuda(qk, "qk")
@@ -244,7 +253,7 @@ def lsh_attn_forward(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *
     if rotations is not None:
         _cuda(rotations, "rotations", qk.dtype)
     B, H, L, d = qk.shape
-    shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup)
+    shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup, bucket_mask)
     need = lsh_attn_forward_workspace_size(shp)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=qk.device)

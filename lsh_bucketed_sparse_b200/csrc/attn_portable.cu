@@ -14,7 +14,9 @@
 // attention"), the score of key j for query i loses log N_ij, N_ij = the
 // number of rounds r' in which j sits in i's window, i.e. in which
 // chunk(undo_r'[i]) - chunk(undo_r'[j]) is 0 or 1; the self pair keeps its
-// replacement score.
+// replacement score.  With `buckets` (the bucket-equality mask, section 2
+// "LSH attention": a query attends only to targets in its own bucket), keys
+// whose bucket in this round differs from the query's are left out.
 #include "common.cuh"
 #include "internal.h"
 
@@ -28,7 +30,8 @@ template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                      const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
-                     const int32_t* __restrict__ undo, T* __restrict__ o_rounds,
+                     const int32_t* __restrict__ undo, const int16_t* __restrict__ bkt,
+                     T* __restrict__ o_rounds,
                      float* __restrict__ lse_rounds, int L, int d, int n_h, int c, int causal,
                      float scale) {
   extern __shared__ float q_all[];  // [kWarps][d]
@@ -42,6 +45,7 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   const T* V = v + bh * (size_t)L * d;
   const float* IN = inv_norm + bh * (size_t)L;
   const int32_t* UD = undo ? undo + bh * (size_t)n_h * L : nullptr;  // [n_h][L]
+  const int16_t* BK = bkt ? bkt + (bh * n_h + r) * (size_t)L : nullptr;  // this round
   float* qs = q_all + warp * d;
   const int k0 = k > 0 ? (k - 1) * c : 0, k1 = (k + 1) * c;
   constexpr int kPer = kMaxD / 32;
@@ -60,7 +64,8 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
       const bool in_window = js < k1;
       const int j = in_window ? P[js] : 0;
       float s = -INFINITY;
-      if (in_window && !(causal && j > i)) {
+      const bool other_bucket = BK && in_window && BK[j] != BK[i];
+      if (in_window && !(causal && j > i) && !other_bucket) {
         if (j == i) {
           s = kSelfScore;
         } else {
@@ -114,20 +119,21 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
 
 cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,
                                  const float* inv_norm, const int32_t* perm,
-                                 const int32_t* undo, void* o_rounds, float* lse_rounds,
-                                 cudaStream_t st) {
+                                 const int32_t* undo, const int16_t* buckets, void* o_rounds,
+                                 float* lse_rounds, cudaStream_t st) {
   if (!p.dedup) undo = nullptr;
+  if (!p.bucket_mask) buckets = nullptr;
   if (p.d > kMaxD) return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
   const size_t smem = (size_t)kWarps * p.d * sizeof(float);
   const float scale = 1.0f / sqrtf((float)p.d);
   if (p.bf16)
     attn_portable_kernel<__nv_bfloat16><<<grid, kWarps * 32, smem, st>>>(
-        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm, undo,
+        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm, undo, buckets,
         (__nv_bfloat16*)o_rounds, lse_rounds, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
   else
     attn_portable_kernel<float><<<grid, kWarps * 32, smem, st>>>(
-        (const float*)qk, (const float*)v, inv_norm, perm, undo, (float*)o_rounds, lse_rounds, p.L,
+        (const float*)qk, (const float*)v, inv_norm, perm, undo, buckets, (float*)o_rounds, lse_rounds, p.L,
         p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
   return cudaGetLastError();
 }

@@ -17,6 +17,7 @@ struct Problem {
   bool bf16;         // element type of qk, v, rotations, out, o_rounds
   bool portable;     // LSH_FLAG_PORTABLE: CUDA-core kernels only
   bool dedup;        // LSH_FLAG_DEDUP: duplicate-count correction
+  bool bucket_mask;  // LSH_FLAG_BUCKET_MASK: bucket-equality mask
   int BH() const { return B * H; }
   int half() const { return n_b / 2; }  // projections per round, 0 when n_b == 1
   int n_chunks() const { return L / c; }
@@ -60,11 +61,12 @@ cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm,
                         int32_t* counts, void* scratch, cudaStream_t st);
 
 // ---- stage 3: chunked attention --------------------------------------------
-// undo: every round's inverse permutation when p.dedup, else ignored.
+// undo: every round's inverse permutation when p.dedup, else ignored;
+// buckets: the bucket ids when p.bucket_mask, else ignored.
 cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v,
                                  const float* inv_norm, const int32_t* perm,
-                                 const int32_t* undo, void* o_rounds, float* lse_rounds,
-                                 cudaStream_t st);
+                                 const int32_t* undo, const int16_t* buckets, void* o_rounds,
+                                 float* lse_rounds, cudaStream_t st);
 bool attn_tc_supported(const Problem& p);
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                            const int32_t* perm, void* o_rounds, float* lse_rounds,

@@ -56,7 +56,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   if (s->causal != 0 && s->causal != 1) return fail(LSH_ERR_INVALID_ARG, "causal must be 0 or 1");
   if (s->dtype != LSH_F32 && s->dtype != LSH_BF16)
     return fail(LSH_ERR_INVALID_ARG, "dtype=%d: must be LSH_F32 or LSH_BF16", s->dtype);
-  if (s->flags & ~(LSH_FLAG_PORTABLE | LSH_FLAG_DEDUP))
+  if (s->flags & ~(LSH_FLAG_PORTABLE | LSH_FLAG_DEDUP | LSH_FLAG_BUCKET_MASK))
     return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
   const long long bh = (long long)s->batch * s->heads;
   if (bh > (1LL << 30)) return fail(LSH_ERR_INVALID_ARG, "batch*heads too large");
@@ -68,6 +68,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   p->causal = s->causal != 0; p->bf16 = s->dtype == LSH_BF16;
   p->portable = (s->flags & LSH_FLAG_PORTABLE) != 0;
   p->dedup = (s->flags & LSH_FLAG_DEDUP) != 0;
+  p->bucket_mask = (s->flags & LSH_FLAG_BUCKET_MASK) != 0;
   return LSH_OK;
 }
 
@@ -113,13 +114,16 @@ lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
 }
 
-// The duplicate-count correction runs on the CUDA-core kernel only.
+// The variants (duplicate-count correction, bucket-equality mask) run on the
+// CUDA-core kernel only.
 lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
-                    const int32_t* perm, const int32_t* undo, void* o_r, float* lse_r,
-                    cudaStream_t st) {
-  cudaError_t e = (!p.portable && !p.dedup && attn_tc_supported(p))
-                      ? launch_attn_tc(p, qk, v, inv_norm, perm, o_r, lse_r, st)
-                      : launch_attn_portable(p, qk, v, inv_norm, perm, undo, o_r, lse_r, st);
+                    const int32_t* perm, const int32_t* undo, const int16_t* buckets,
+                    void* o_r, float* lse_r, cudaStream_t st) {
+  const bool variant = p.dedup || p.bucket_mask;
+  cudaError_t e =
+      (!p.portable && !variant && attn_tc_supported(p))
+          ? launch_attn_tc(p, qk, v, inv_norm, perm, o_r, lse_r, st)
+          : launch_attn_portable(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
 }
 
@@ -160,7 +164,7 @@ lsh_status forward_body(const Problem& p, const void* qk, const void* v, const v
   CHECK(run_hash(p, qk, rot, buckets, inv_norm, st));
   int32_t* undo = p.dedup ? reinterpret_cast<int32_t*>(base + w.undo) : nullptr;
   CHECK(run_sort(p, buckets, perm, undo, nullptr, base + w.sort_scratch, st));
-  CHECK(run_attn(p, qk, v, inv_norm, perm, undo, o_r, lse_r, st));
+  CHECK(run_attn(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st));
   CHECK(run_combine(p, o_r, lse_r, out, lse, st));
   return LSH_OK;
 }
@@ -279,28 +283,29 @@ lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const vo
   CHECK(check_ptr(perm, "perm"));
   CHECK(check_ptr(o_rounds, "o_rounds"));
   CHECK(check_ptr(lse_rounds, "lse_rounds"));
-  if (p.dedup)
+  if (p.dedup || p.bucket_mask)
     return fail(LSH_ERR_INVALID_ARG,
-                "LSH_FLAG_DEDUP needs every round's undo: call lsh_attn_chunked_fwd_dedup");
-  return run_attn(p, qk, v, inv_norm, perm, nullptr, o_rounds, lse_rounds,
+                "LSH_FLAG_DEDUP / LSH_FLAG_BUCKET_MASK need undo / buckets: "
+                "call lsh_attn_chunked_fwd_ex");
+  return run_attn(p, qk, v, inv_norm, perm, nullptr, nullptr, o_rounds, lse_rounds,
                   static_cast<cudaStream_t>(stream));
 }
 
-lsh_status lsh_attn_chunked_fwd_dedup(const lsh_shape* shape, const void* qk, const void* v,
-                                      const float* inv_norm, const int32_t* perm,
-                                      const int32_t* undo, void* o_rounds, float* lse_rounds,
-                                      void* stream) {
+lsh_status lsh_attn_chunked_fwd_ex(const lsh_shape* shape, const void* qk, const void* v,
+                                   const float* inv_norm, const int32_t* perm,
+                                   const int32_t* undo, const int16_t* buckets, void* o_rounds,
+                                   float* lse_rounds, void* stream) {
   Problem p;
   CHECK(to_problem(shape, &p));
   CHECK(check_ptr(qk, "qk"));
   CHECK(check_ptr(v, "v"));
   CHECK(check_ptr(inv_norm, "inv_norm"));
   CHECK(check_ptr(perm, "perm"));
-  CHECK(check_ptr(undo, "undo"));
+  CHECK(check_ptr(undo, "undo", !p.dedup));
+  CHECK(check_ptr(buckets, "buckets", !p.bucket_mask));
   CHECK(check_ptr(o_rounds, "o_rounds"));
   CHECK(check_ptr(lse_rounds, "lse_rounds"));
-  p.dedup = true;
-  return run_attn(p, qk, v, inv_norm, perm, undo, o_rounds, lse_rounds,
+  return run_attn(p, qk, v, inv_norm, perm, undo, buckets, o_rounds, lse_rounds,
                   static_cast<cudaStream_t>(stream));
 }
 

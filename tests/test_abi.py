@@ -87,7 +87,7 @@ def test_workspace_size_and_too_small(L):
 
 def test_unknown_flag_rejected(L):
     shp = shape()
-    shp.flags = 4
+    shp.flags = 8  # bits 0-2 are LSH_FLAG_PORTABLE, _DEDUP, _BUCKET_MASK
     assert fwd(L, shp) == 1
 
 

@@ -339,8 +339,8 @@ def test_dedup_matches_oracle(wl):
     rot_d = rot.to(DEV)
     b, inv = lsh.lsh_attn_hash(qk_d, rot_d, wl.n_buckets, wl.n_hashes)
     perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets)
-    o_r, lse_r = lsh.lsh_attn_chunked_fwd_dedup(qk_d, v_d, inv, perm, undo, wl.chunk_len,
-                                               wl.causal, n_buckets=wl.n_buckets)
+    o_r, lse_r = lsh.lsh_attn_chunked_fwd_ex(qk_d, v_d, inv, perm, wl.chunk_len, wl.causal,
+                                            undo=undo, n_buckets=wl.n_buckets)
     out, lse = lsh.lsh_attn_combine(o_r, lse_r)
     f_out, f_lse = lsh.lsh_attn_forward(qk_d, v_d, rot_d, wl.n_hashes, wl.n_buckets,
                                         wl.chunk_len, wl.causal, dedup=True)
@@ -373,6 +373,11 @@ def test_dedup_stage_call_needs_undo():
                                         lsh._ptr(inv), lsh._ptr(perm), lsh._ptr(o_r),
                                         lsh._ptr(l_r), None)
     assert st == 1  # LSH_ERR_INVALID_ARG: the flag needs every round's undo
+    shp.flags = lsh.FLAG_BUCKET_MASK
+    st = lsh.lib().lsh_attn_chunked_fwd(ctypes.byref(shp), lsh._ptr(qk), lsh._ptr(v),
+                                        lsh._ptr(inv), lsh._ptr(perm), lsh._ptr(o_r),
+                                        lsh._ptr(l_r), None)
+    assert st == 1  # and the bucket mask the bucket ids
 
 
 def test_host_pipeline_uneven_groups():
@@ -391,3 +396,40 @@ def test_host_pipeline_uneven_groups():
     ref_out, ref_lse = lsh.lsh_attn_forward(qk.to(DEV), v.to(DEV), rot.to(DEV), wl.n_hashes,
                                             wl.n_buckets, wl.chunk_len, wl.causal)
     assert torch.equal(out_h, ref_out.cpu()) and torch.equal(lse_h, ref_lse.cpu())
+
+
+# ---------------------------------------------------------------------------
+# Bucket-equality mask (LSH_FLAG_BUCKET_MASK), alone and with the correction.
+MASKED = [
+    (W.small("bmask-bf16-causal", heads=2, seq_len=512, n_hashes=3, n_buckets=16), False),
+    (W.small("bmask-f32-noncausal", heads=1, seq_len=256, n_hashes=2, n_buckets=8,
+             causal=False, dtype=torch.float32), False),
+    (W.small("bmask-dedup-bf16-d128", heads=2, seq_len=256, d_k=128, n_hashes=3, n_buckets=4,
+             chunk_len=32, causal=True), True),
+]
+
+
+@pytest.mark.parametrize("wl,dedup", MASKED, ids=[w.name for w, _ in MASKED])
+def test_bucket_mask_matches_oracle(wl, dedup):
+    qk, v, rot = W.make_inputs(wl)
+    qk_d, v_d, rot_d = qk.to(DEV), v.to(DEV), rot.to(DEV)
+    b, inv = lsh.lsh_attn_hash(qk_d, rot_d, wl.n_buckets, wl.n_hashes)
+    perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets)
+    o_r, lse_r = lsh.lsh_attn_chunked_fwd_ex(qk_d, v_d, inv, perm, wl.chunk_len, wl.causal,
+                                            undo=undo if dedup else None, buckets=b,
+                                            n_buckets=wl.n_buckets)
+    out, lse = lsh.lsh_attn_combine(o_r, lse_r)
+    f_out, f_lse = lsh.lsh_attn_forward(qk_d, v_d, rot_d, wl.n_hashes, wl.n_buckets,
+                                        wl.chunk_len, wl.causal, dedup=dedup, bucket_mask=True)
+    lsh.lsh_attn_device_check()
+    assert torch.equal(f_out, out) and torch.equal(f_lse, lse)
+    gb = b.cpu().numpy().astype(np.int64)
+    res0 = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal, buckets=gb, dedup=dedup)
+    res = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal, buckets=gb, dedup=dedup,
+                    bucket_mask=True)
+    assert np.abs(res["lse"] - res0["lse"]).max() > 1e-3  # the mask drops some keys
+    bf16 = wl.dtype == torch.bfloat16
+    P.check_float(o_r, res["o_rounds"], bf16, "o_rounds", 3)
+    P.check_lse(lse_r, res["lse_rounds"], bf16, "lse_rounds")
+    P.check_float(out, res["out"], bf16, "out")
+    P.check_lse(lse, res["lse"], bf16, "lse")

@@ -73,8 +73,9 @@ def test_pin_catches_mutation(monkeypatch, name, mutant, pin):
 def test_pin_catches_missing_scale(monkeypatch):
     real = O.attend_round
 
-    def no_scale(x, v, perm_r, chunk_len, causal, dedup_undo=None):
-        return real(x * math.sqrt(x.shape[1]), v, perm_r, chunk_len, causal, dedup_undo)
+    def no_scale(x, v, perm_r, chunk_len, causal, dedup_undo=None, bucket_r=None):
+        return real(x * math.sqrt(x.shape[1]), v, perm_r, chunk_len, causal, dedup_undo,
+                    bucket_r)
 
     monkeypatch.setattr(O, "attend_round", no_scale)
     with pytest.raises(AssertionError):
