@@ -40,6 +40,11 @@ Readings where the pages are silent (each is also listed in the design notes):
   * the self-mask REPLACES the score of j == i by SELF_SCORE = -1e5, a finite
     penalty, so a token that sees only itself in every round outputs v_i;
   * a key of zero norm normalises to the zero vector;
+  * the routing-style assignment (``kmeans=True``; the pages name online
+    k-means for the Routing Transformer and give no more) puts token x in
+    the bucket of the centroid with the largest dot product, argmax_j x . mu_j
+    (lowest index on ties), with the centroids given ([n_h, d, n_b], one set
+    per round) and not updated;
   * the duplicate-count correction of Appendix A is off unless asked for
     (``dedup=True`` subtracts log N_ij, N_ij = number of rounds whose window
     of query i contains key j).
@@ -199,8 +204,29 @@ def as_f64(t) -> np.ndarray:
     return np.asarray(t, dtype=np.float64)
 
 
-def hash_all(qk, rotations, n_buckets):
-    """[B, H, L, d] -> buckets, margins [B, H, n_h, L]."""
+def kmeans_head(x: np.ndarray, centroids, n_buckets: int):
+    """Routing-style assignment: bucket = argmax_j x . mu_j over the round's
+    n_b centroids (first maximal index).  x: [L, d]; centroids: [n_h, d, n_b].
+    Returns (buckets [n_h, L], margins [n_h, L]) like hash_head."""
+    n_h, d, nb = centroids.shape
+    assert nb == n_buckets and d == x.shape[1]
+    L = x.shape[0]
+    buckets = np.empty((n_h, L), np.int64)
+    margins = np.empty((n_h, L), np.float64)
+    for r in range(n_h):
+        p = x @ centroids[r]                       # [L, n_b]
+        buckets[r] = np.argmax(p, axis=1)
+        if nb >= 2:
+            top2 = np.partition(p, nb - 2, axis=1)[:, nb - 2:]
+            margins[r] = top2[:, 1] - top2[:, 0]
+        else:
+            margins[r] = np.inf
+    return buckets, margins
+
+
+def hash_all(qk, rotations, n_buckets, kmeans=False):
+    """[B, H, L, d] -> buckets, margins [B, H, n_h, L].  With ``kmeans`` the
+    rotations are centroids [n_h, d, n_b] and kmeans_head assigns."""
     qk = as_f64(qk)
     rot = None if rotations is None else as_f64(rotations)
     B, H, L, _ = qk.shape
@@ -209,7 +235,10 @@ def hash_all(qk, rotations, n_buckets):
     margins = np.empty((B, H, n_h, L))
     for b in range(B):
         for h in range(H):
-            buckets[b, h], margins[b, h] = hash_head(qk[b, h], rot, n_buckets)
+            if kmeans:
+                buckets[b, h], margins[b, h] = kmeans_head(qk[b, h], rot, n_buckets)
+            else:
+                buckets[b, h], margins[b, h] = hash_head(qk[b, h], rot, n_buckets)
     return buckets, margins
 
 
@@ -259,13 +288,13 @@ def combine_all(o_rounds, lse_rounds):
 
 
 def forward(qk, v, rotations, n_buckets, chunk_len, causal, buckets=None, dedup=False,
-            bucket_mask=False):
+            bucket_mask=False, kmeans=False):
     """The whole pass.  If ``buckets`` is given, hashing is skipped and those
     ids are used (this is how GPU bucket ids are fed back so that the later
     stages can be compared exactly).  Returns a dict of every intermediate."""
     res = {}
     if buckets is None:
-        buckets, margins = hash_all(qk, rotations, n_buckets)
+        buckets, margins = hash_all(qk, rotations, n_buckets, kmeans=kmeans)
         res["margins"] = margins
     buckets = np.asarray(buckets, np.int64)
     perm, undo = sort_all(buckets)

@@ -411,3 +411,26 @@ def test_bucket_mask_is_a_no_op_within_one_bucket():
     b = O.forward(x, v, None, 1, c, True, buckets=zero, bucket_mask=True)
     np.testing.assert_array_equal(a["out"], b["out"])
     np.testing.assert_array_equal(a["lse"], b["lse"])
+
+
+# ------------------------------------------------ routing-style assignment --
+def test_kmeans_with_plus_minus_rotation_is_the_lsh_hash():
+    # Centroids [R, -R] give dot products [xR; -xR]: the assignment must equal
+    # the random-rotation hash, bucket for bucket and margin for margin.
+    rng = np.random.default_rng(31)
+    x = rng.standard_normal((2, 3, 40, 8))
+    R = rng.standard_normal((3, 8, 5))
+    lb, lm = O.hash_all(x, R, 10)
+    kb, km = O.hash_all(x, np.concatenate([R, -R], axis=2), 10, kmeans=True)
+    np.testing.assert_array_equal(kb, lb)
+    np.testing.assert_array_equal(km, lm)
+
+
+def test_kmeans_picks_the_largest_coordinate_with_basis_centroids():
+    # Centroids e_0..e_{d-1}: x . e_j = x_j, so the bucket is the index of the
+    # largest coordinate (the first one on ties).
+    x = np.array([[0.5, 2.0, -3.0, 2.0], [-1.0, -2.0, -0.5, -4.0], [1.0, 1.0, 1.0, 1.0]])
+    C = np.eye(4)[None]                            # [1, d, n_b = d]
+    b, m = O.kmeans_head(x, C, 4)
+    np.testing.assert_array_equal(b[0], [1, 2, 0])
+    np.testing.assert_allclose(m[0], [0.0, 0.5, 0.0])
