@@ -346,6 +346,9 @@ def main(argv=None):
     ap.add_argument("--bucket-mask", action="store_true",
                     help="the pass with the bucket-equality mask (CUDA-core attention); a "
                          "separate measurement, not the headline")
+    ap.add_argument("--kmeans", action="store_true",
+                    help="routing-style assignment to n_buckets centroids (CUDA-core hash) "
+                         "instead of the random-rotation hash; a separate measurement")
     ap.add_argument("--only-stage", choices=["hash", "sort", "chunked_attention", "combine"],
                     help="time one stage call alone (for profiling); prints its own JSON line")
     args = ap.parse_args(argv)
@@ -363,11 +366,13 @@ def main(argv=None):
     stream = torch.cuda.current_stream(dev)
 
     qk_h, v_h, rot_h = W.make_inputs(wl)
+    if args.kmeans:
+        rot_h = W.make_centroids(wl)
     qk, v = qk_h.to(dev), v_h.to(dev)
     rot = rot_h.to(dev) if rot_h is not None else None
     shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
                          wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup,
-                         bucket_mask=args.bucket_mask)
+                         bucket_mask=args.bucket_mask, kmeans=args.kmeans)
     ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
     out = torch.empty_like(qk)
     lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
@@ -376,7 +381,7 @@ def main(argv=None):
     def step():
         lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
                              workspace=ws, out=out, lse=lse, dedup=args.dedup,
-                             bucket_mask=args.bucket_mask)
+                             bucket_mask=args.bucket_mask, kmeans=args.kmeans)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -410,7 +415,7 @@ def main(argv=None):
         flush.fill_(2.0)
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         ev[0].record(stream)
-        b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+        b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes, kmeans=args.kmeans)
         ev[1].record(stream)
         perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=args.dedup)
         ev[2].record(stream)
@@ -473,8 +478,8 @@ def main(argv=None):
     roofline["pass_frac"] = t_roof * 1e3 / ms_per_step
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not (args.dedup or
-                                                                      args.bucket_mask):
+    variant = args.dedup or args.bucket_mask or args.kmeans
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         cpu = cpu_baseline(wl, args.cpu_rounds)
 
     if rank == 0:
@@ -489,8 +494,10 @@ def main(argv=None):
                                (["duplicate-count correction (LSH_FLAG_DEDUP)"] if args.dedup
                                 else []) +
                                (["bucket-equality mask (LSH_FLAG_BUCKET_MASK)"]
-                                if args.bucket_mask else [])) + ", CUDA-core attention"}
-                              if (args.dedup or args.bucket_mask) else {})),
+                                if args.bucket_mask else []) +
+                               (["routing-style assignment to n_buckets centroids "
+                                 "(LSH_FLAG_KMEANS)"] if args.kmeans else []))}
+                              if variant else {})),
             "clocks": clocks.summary(),
             "e2e": {"value": world * wl.tokens / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

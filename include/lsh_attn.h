@@ -88,6 +88,17 @@ typedef enum lsh_dtype {
                                   differs from the query's are not attended.
                                   Runs on the CUDA-core attention kernel;
                                   the stage call is lsh_attn_chunked_fwd_ex. */
+#define LSH_FLAG_KMEANS 8u     /* routing-style bucket assignment (the pages
+                                  name online k-means for the Routing
+                                  Transformer): `rotations` holds centroids
+                                  [n_h, d, n_b], one set per round, and a
+                                  token goes to the bucket of the centroid
+                                  with the largest dot product (lowest index
+                                  on ties); n_b may then be any value in
+                                  [2, 32768].  bf16 with d in {64, 128} and
+                                  n_b a multiple of 32 runs on the tensor-
+                                  core hash kernel, other shapes on the
+                                  CUDA-core one.                            */
 
 typedef struct lsh_shape {
   int32_t batch;       /* B >= 1                                             */
@@ -133,9 +144,11 @@ LSH_ATTN_API lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, co
  * Bucket ids outside [0, n_b) are undefined behaviour (stage 1 never makes
  * them); the kernels do not read or write out of bounds for them.
  * The call takes n_h * B * H * ceil(L / 2048) * n_b * 4 bytes of temporary
- * device memory from the device's stream-ordered pool (cudaMallocAsync on
- * `stream`, freed on `stream` after use); a failed allocation returns
- * LSH_ERR_CUDA.  The fused calls take it from their workspace instead.
+ * device memory, stream-ordered on `stream` from a memory pool the library
+ * creates on first use on each device and keeps (cudaMallocFromPoolAsync /
+ * cudaFreeAsync; the pool's blocks stay with it for reuse until the process
+ * exits); a failed allocation returns LSH_ERR_CUDA.  The fused calls take it
+ * from their workspace instead.
  * ---------------------------------------------------------------------- */
 LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
                          int32_t* undo, int32_t* counts, void* stream);

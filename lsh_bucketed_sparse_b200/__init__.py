@@ -25,7 +25,7 @@ __all__ = [
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
     "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
     "LIB_PATH", "HEADER_PATH", "NOALLOC_SCRATCH_BYTES",
-    "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP", "FLAG_BUCKET_MASK",
+    "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP", "FLAG_BUCKET_MASK", "FLAG_KMEANS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -36,6 +36,7 @@ F32, BF16 = 0, 1
 FLAG_PORTABLE = 1
 FLAG_DEDUP = 2
 FLAG_BUCKET_MASK = 4
+FLAG_KMEANS = 8
 NOALLOC_SCRATCH_BYTES = 64 << 20  # LSH_ATTN_NOALLOC_SCRATCH_BYTES
 STATUS = {0: "LSH_OK", 1: "LSH_ERR_INVALID_ARG", 2: "LSH_ERR_UNSUPPORTED",
           3: "LSH_ERR_WORKSPACE", 4: "LSH_ERR_CUDA", 5: "LSH_ERR_DEVICE_TIMEOUT"}
@@ -116,11 +117,12 @@ def _dtype_code(t: torch.dtype) -> int:
 
 
 def make_shape(batch, heads, seq_len, d_k, n_hashes, n_buckets, chunk_len, causal,
-               dtype=torch.bfloat16, portable=False, dedup=False, bucket_mask=False) -> Shape:
+               dtype=torch.bfloat16, portable=False, dedup=False, bucket_mask=False,
+               kmeans=False) -> Shape:
     return Shape(batch, heads, seq_len, d_k, n_hashes, n_buckets, chunk_len, int(bool(causal)),
                  dtype if isinstance(dtype, int) else _dtype_code(dtype),
                  (FLAG_PORTABLE if portable else 0) | (FLAG_DEDUP if dedup else 0)
-                 | (FLAG_BUCKET_MASK if bucket_mask else 0))
+                 | (FLAG_BUCKET_MASK if bucket_mask else 0) | (FLAG_KMEANS if kmeans else 0))
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -143,14 +145,15 @@ def _stream(stream):
 
 
 def _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup=False,
-              bucket_mask=False):
+              bucket_mask=False, kmeans=False):
     B, H, L, d = qk.shape
     return make_shape(B, H, L, d, n_hashes, n_buckets, chunk_len, causal, qk.dtype, portable,
-                      dedup, bucket_mask)
+                      dedup, bucket_mask, kmeans)
 
 
 # --------------------------------------------------------------------------
-def lsh_attn_hash(qk, rotations, n_buckets, n_hashes=None, *, portable=False, stream=None):
+def lsh_attn_hash(qk, rotations, n_buckets, n_hashes=None, *, portable=False, kmeans=False,
+                  stream=None):
     """Stage 1.  qk [B,H,L,d]; rotations [n_h,d,n_b/2] (None when n_b == 1).
     Returns (buckets int16 [B,H,n_h,L], inv_norm float32 [B,H,L])."""
     _cuda(qk, "qk")
@@ -160,7 +163,7 @@ def lsh_attn_hash(qk, rotations, n_buckets, n_hashes=None, *, portable=False, st
     if n_hashes is None:
         n_hashes = 1
     B, H, L, d = qk.shape
-    shp = _shape_of(qk, n_hashes, n_buckets, 1, False, portable)
+    shp = _shape_of(qk, n_hashes, n_buckets, 1, False, portable, kmeans=kmeans)
     buckets = torch.empty(B, H, n_hashes, L, dtype=torch.int16, device=qk.device)
     inv_norm = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
     _check(lib().lsh_attn_hash(ctypes.byref(shp), _ptr(qk), _ptr(rotations), _ptr(buckets),
@@ -245,7 +248,7 @@ def lsh_attn_forward_workspace_size(shape: Shape) -> int:
 
 def lsh_attn_forward(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *,
                      workspace=None, out=None, lse=None, portable=False, dedup=False,
-                     bucket_mask=False, stream=None):
+                     bucket_mask=False, kmeans=False, stream=None):
     """The fused pass.  Returns (out [B,H,L,d], lse f32 [B,H,L]).  ``workspace`` (a
     uint8 CUDA tensor) can be passed in to avoid an allocation per call."""
     _cuda(qk, "qk")
@@ -253,7 +256,8 @@ def lsh_attn_forward(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *
     if rotations is not None:
         _cuda(rotations, "rotations", qk.dtype)
     B, H, L, d = qk.shape
-    shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup, bucket_mask)
+    shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup, bucket_mask,
+                    kmeans)
     need = lsh_attn_forward_workspace_size(shp)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=qk.device)

@@ -8,6 +8,10 @@
 // row is staged in shared memory, each lane owns projection columns
 // j = lane, lane + 32, ..., accumulates x . R[:, j] in float32 in order
 // k = 0..d-1, tracks its best (|p|, z-index) and the warp reduces them.
+//
+// With `kmeans` (routing-style assignment) the n_b columns of the round's
+// matrix are centroids and the bucket is argmax_j x . mu_j (lowest j on
+// ties): the same loop over signed values instead of |p|.
 #include "common.cuh"
 #include "internal.h"
 
@@ -20,7 +24,7 @@ template <typename T>
 __global__ void __launch_bounds__(kWarps * 32)
 hash_portable_kernel(const T* __restrict__ qk, const T* __restrict__ rot,
                      int16_t* __restrict__ buckets, float* __restrict__ inv_norm, int BH, int L,
-                     int d, int n_h, int half) {
+                     int d, int n_h, int half, int n_cent) {
   extern __shared__ float xs_all[];  // [kWarps][d]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* xs = xs_all + warp * d;
@@ -41,7 +45,21 @@ hash_portable_kernel(const T* __restrict__ qk, const T* __restrict__ rot,
     for (int r = 0; r < n_h; ++r) {
       float best_a = -1.f;
       int best_z = 0x7fffffff;
-      if (half > 0) {
+      if (n_cent > 0) {
+        best_a = -INFINITY;
+        const T* C = rot + (size_t)r * d * n_cent;
+        for (int j = lane; j < n_cent; j += 32) {
+          float p = 0.f;
+          for (int k = 0; k < d; ++k) p = fmaf(xs[k], to_f32(C[(size_t)k * n_cent + j]), p);
+          if (z_better(p, j, best_a, best_z)) { best_a = p; best_z = j; }
+        }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) {
+          const float oa = __shfl_xor_sync(0xffffffffu, best_a, o);
+          const int oz = __shfl_xor_sync(0xffffffffu, best_z, o);
+          if (z_better(oa, oz, best_a, best_z)) { best_a = oa; best_z = oz; }
+        }
+      } else if (half > 0) {
         const T* R = rot + (size_t)r * d * half;
         for (int j = lane; j < half; j += 32) {
           float p = 0.f;
@@ -76,11 +94,11 @@ cudaError_t launch_hash_portable(const Problem& p, const void* qk, const void* r
   if (p.bf16)
     hash_portable_kernel<__nv_bfloat16><<<(unsigned)blocks, kWarps * 32, smem, st>>>(
         (const __nv_bfloat16*)qk, (const __nv_bfloat16*)rot, buckets, inv_norm, p.BH(), p.L,
-        p.d, p.n_h, p.half());
+        p.d, p.n_h, p.kmeans ? 0 : p.half(), p.kmeans ? p.n_b : 0);
   else
     hash_portable_kernel<float><<<(unsigned)blocks, kWarps * 32, smem, st>>>(
         (const float*)qk, (const float*)rot, buckets, inv_norm, p.BH(), p.L, p.d, p.n_h,
-        p.half());
+        p.kmeans ? 0 : p.half(), p.kmeans ? p.n_b : 0);
   return cudaGetLastError();
 }
 

@@ -101,11 +101,26 @@ __device__ __forceinline__ float chunk_max_abs(const uint32_t* u) {
   return fmaxf(max3f(w0, w1, w2), w3);
 }
 
+// Largest signed p of a 32-column chunk (the routing-style assignment).
+__device__ __forceinline__ float chunk_max_signed(const uint32_t* u) {
+  float v[11];
+#pragma unroll
+  for (int t = 0; t < 10; ++t)
+    v[t] = max3f(__uint_as_float(u[3 * t]), __uint_as_float(u[3 * t + 1]),
+                 __uint_as_float(u[3 * t + 2]));
+  v[10] = fmaxf(__uint_as_float(u[30]), __uint_as_float(u[31]));
+  const float w0 = max3f(v[0], v[1], v[2]), w1 = max3f(v[3], v[4], v[5]);
+  const float w2 = max3f(v[6], v[7], v[8]), w3 = fmaxf(v[9], v[10]);
+  return fmaxf(max3f(w0, w1, w2), w3);
+}
+
+// KM: the routing-style assignment (argmax over the n_b columns of given
+// centroids, lowest column on ties) instead of argmax([xR; -xR]).
 // NP > 0: every piece is NP pairs of 32-column chunks and a round is a whole
 // number of pairs (P % 64 == 0), so each epilogue warp takes one chunk of
 // every pair at fixed positions and loads the next chunk while it reduces the
 // current one.  NP == 0: any P that is a multiple of 32.
-template <int NP>
+template <int NP, bool KM>
 __global__ void __launch_bounds__(kThreads, 1)
 hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
   extern __shared__ uint8_t smem_raw[];
@@ -291,15 +306,19 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     };
     int it = 0, gp = 0, ex = 0;
     bool ok = true;
-    float best_a = -1.f;
+    // no candidate yet: below every |p| (hash) or every p (assignment)
+    constexpr float kNone = KM ? -INFINITY : -1.f;
+    float best_a = kNone;
     int best_j0 = 0;
 
     // One 32-column chunk starting at round column j0: keep it when it holds
-    // a larger |p| than every earlier chunk of the round.
+    // a larger |p| (hash) or p (assignment) than every earlier chunk of the
+    // round; on equal values the earlier chunk stays, except for the hash's
+    // positive-entry rule below.
     auto take_chunk = [&](const uint32_t* u, int j0) {
-      const float cm = chunk_max_abs(u);
+      const float cm = KM ? chunk_max_signed(u) : chunk_max_abs(u);
       bool take = cm > best_a;
-      if (__any_sync(0xffffffffu, cm == best_a)) {
+      if (!KM && __any_sync(0xffffffffu, cm == best_a)) {
         // Equal largest |p| in an earlier chunk (rare): a positive entry
         // wins over negative ones, and the earlier chunk wins otherwise.
         float sv[kChunk];
@@ -322,18 +341,18 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     auto round_end = [&](int bh, int t0, int rr, bool row_valid) -> bool {
       int z = INT_MAX;
       const float a = best_a;
-      if (best_a >= 0.f) {
+      if (best_a > kNone) {
         float sv[kChunk];
         load_saved(sv);
         int tp = -1, tn = 0;
 #pragma unroll
         for (int t = kChunk - 1; t >= 0; --t) {
           if (sv[t] == best_a) tp = t;
-          if (sv[t] == -best_a) tn = t;
+          if (!KM && sv[t] == -best_a) tn = t;
         }
         z = tp >= 0 ? best_j0 + tp : p.P + best_j0 + tn;
       }
-      best_a = -1.f;
+      best_a = kNone;
       const int xb = ex & 1;
       const uint32_t par = (ex >> 1) & 1;
       ++ex;
@@ -456,9 +475,13 @@ struct Plan {
   size_t smem;
 };
 
+// Projection columns per round: n_b / 2 for the hash, n_b centroids for the
+// routing-style assignment.
+int round_cols(const Problem& pr) { return pr.kmeans ? pr.n_b : pr.half(); }
+
 bool make_plan(const Problem& pr, Plan* out) {
   const long long n_tiles = (long long)pr.BH() * ((pr.L + kRows - 1) / kRows);
-  const int P = pr.half();
+  const int P = round_cols(pr);
   if (P <= 0 || P % kChunk) return false;
   const int d = pr.d;
   // The largest group of rounds (a divisor of n_h) whose rotations, at least
@@ -527,7 +550,7 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   p.buckets = buckets;
   p.inv_norm = inv_norm;
   p.err = err;
-  p.BH = pr.BH(); p.L = pr.L; p.d = pr.d; p.n_h = pr.n_h; p.P = pr.half();
+  p.BH = pr.BH(); p.L = pr.L; p.d = pr.d; p.n_h = pr.n_h; p.P = round_cols(pr);
   p.gr = plan.gr;
   p.G = plan.G;
   p.tiles_per_head = (pr.L + kRows - 1) / kRows;
@@ -537,12 +560,22 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   p.n_pieces = plan.n_pieces;
   p.stages = plan.stages;
   void (*kernel)(const CUtensorMap, const Params);
-  switch (plan.np) {
-    case 1: kernel = hash_tc_kernel<1>; break;
-    case 2: kernel = hash_tc_kernel<2>; break;
-    case 3: kernel = hash_tc_kernel<3>; break;
-    case 4: kernel = hash_tc_kernel<4>; break;
-    default: kernel = hash_tc_kernel<0>; break;
+  if (pr.kmeans) {
+    switch (plan.np) {
+      case 1: kernel = hash_tc_kernel<1, true>; break;
+      case 2: kernel = hash_tc_kernel<2, true>; break;
+      case 3: kernel = hash_tc_kernel<3, true>; break;
+      case 4: kernel = hash_tc_kernel<4, true>; break;
+      default: kernel = hash_tc_kernel<0, true>; break;
+    }
+  } else {
+    switch (plan.np) {
+      case 1: kernel = hash_tc_kernel<1, false>; break;
+      case 2: kernel = hash_tc_kernel<2, false>; break;
+      case 3: kernel = hash_tc_kernel<3, false>; break;
+      case 4: kernel = hash_tc_kernel<4, false>; break;
+      default: kernel = hash_tc_kernel<0, false>; break;
+    }
   }
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);

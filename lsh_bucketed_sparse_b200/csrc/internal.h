@@ -18,6 +18,7 @@ struct Problem {
   bool portable;     // LSH_FLAG_PORTABLE: CUDA-core kernels only
   bool dedup;        // LSH_FLAG_DEDUP: duplicate-count correction
   bool bucket_mask;  // LSH_FLAG_BUCKET_MASK: bucket-equality mask
+  bool kmeans;       // LSH_FLAG_KMEANS: argmax over n_b given centroids
   int BH() const { return B * H; }
   int half() const { return n_b / 2; }  // projections per round, 0 when n_b == 1
   int n_chunks() const { return L / c; }

@@ -47,7 +47,12 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   if (s->d_k < 8 || s->d_k > 256 || s->d_k % 8)
     return fail(LSH_ERR_INVALID_ARG, "d_k=%d: must be a multiple of 8 in [8, 256]", s->d_k);
   if (s->n_hashes < 1) return fail(LSH_ERR_INVALID_ARG, "n_hashes must be >= 1");
-  if (!(s->n_buckets == 1 || (s->n_buckets >= 2 && s->n_buckets <= 32768 && s->n_buckets % 2 == 0)))
+  const bool kmeans = (s->flags & LSH_FLAG_KMEANS) != 0;
+  if (kmeans && !(s->n_buckets >= 2 && s->n_buckets <= 32768))
+    return fail(LSH_ERR_INVALID_ARG, "n_buckets=%d: must be in [2, 32768] with LSH_FLAG_KMEANS",
+                s->n_buckets);
+  if (!kmeans &&
+      !(s->n_buckets == 1 || (s->n_buckets >= 2 && s->n_buckets <= 32768 && s->n_buckets % 2 == 0)))
     return fail(LSH_ERR_INVALID_ARG, "n_buckets=%d: must be 1 or even in [2, 32768]",
                 s->n_buckets);
   if (s->chunk_len < 1 || s->seq_len % s->chunk_len)
@@ -56,7 +61,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   if (s->causal != 0 && s->causal != 1) return fail(LSH_ERR_INVALID_ARG, "causal must be 0 or 1");
   if (s->dtype != LSH_F32 && s->dtype != LSH_BF16)
     return fail(LSH_ERR_INVALID_ARG, "dtype=%d: must be LSH_F32 or LSH_BF16", s->dtype);
-  if (s->flags & ~(LSH_FLAG_PORTABLE | LSH_FLAG_DEDUP | LSH_FLAG_BUCKET_MASK))
+  if (s->flags & ~(LSH_FLAG_PORTABLE | LSH_FLAG_DEDUP | LSH_FLAG_BUCKET_MASK | LSH_FLAG_KMEANS))
     return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
   const long long bh = (long long)s->batch * s->heads;
   if (bh > (1LL << 30)) return fail(LSH_ERR_INVALID_ARG, "batch*heads too large");
@@ -69,6 +74,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
   p->portable = (s->flags & LSH_FLAG_PORTABLE) != 0;
   p->dedup = (s->flags & LSH_FLAG_DEDUP) != 0;
   p->bucket_mask = (s->flags & LSH_FLAG_BUCKET_MASK) != 0;
+  p->kmeans = kmeans;
   return LSH_OK;
 }
 
@@ -179,7 +185,7 @@ struct HostStaging {
 HostStaging host_layout(const Problem& p) {
   HostStaging h;
   h.in_bytes = (size_t)p.BH() * p.L * p.d * p.elem();
-  h.rot_bytes = p.n_b > 1 ? (size_t)p.n_h * p.d * p.half() * p.elem() : 0;
+  h.rot_bytes = p.n_b > 1 ? (size_t)p.n_h * p.d * (p.kmeans ? p.n_b : p.half()) * p.elem() : 0;
   h.out_bytes = h.in_bytes;
   h.lse_bytes = (size_t)p.BH() * p.L * sizeof(float);
   size_t off = 0;
@@ -222,6 +228,29 @@ HostPipe* host_pipe(int dev) {
   return g_pipe[dev].ok ? &g_pipe[dev] : nullptr;
 }
 
+// A memory pool per device for the stage calls' temporary scratch; its
+// release threshold is unlimited, so freed blocks stay with the pool.
+cudaMemPool_t g_pool[kMaxDevices];
+std::once_flag g_pool_once[kMaxDevices];
+
+cudaMemPool_t scratch_pool(int dev) {
+  std::call_once(g_pool_once[dev], [dev] {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t pool = nullptr;
+    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return;
+    uint64_t keep = ~0ull;
+    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
+      cudaMemPoolDestroy(pool);
+      return;
+    }
+    g_pool[dev] = pool;
+  });
+  return g_pool[dev];
+}
+
 }  // namespace
 
 unsigned int* device_error_word() {
@@ -260,11 +289,19 @@ lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t
   CHECK(check_ptr(perm, "perm"));
   CHECK(check_ptr(undo, "undo", true));
   CHECK(check_ptr(counts, "counts", true));
-  // The per-tile counts live in stream-ordered scratch from the device's
-  // memory pool, released on the same stream once the sort has used them.
+  // The per-tile counts live in stream-ordered scratch from the library's
+  // own memory pool on this device (it keeps its memory, so after the first
+  // call the allocation is a reuse), released on the same stream once the
+  // sort has used them.
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(LSH_ERR_UNSUPPORTED, "device %d", dev);
+  cudaMemPool_t pool = scratch_pool(dev);
+  if (!pool) return fail(LSH_ERR_CUDA, "could not create the scratch memory pool");
   void* scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(&scratch, sort_scratch_bytes(p), st);
+  e = cudaMallocFromPoolAsync(&scratch, sort_scratch_bytes(p), pool, st);
   if (e != cudaSuccess) return cuda_fail(e, "sort scratch");
   const lsh_status r = run_sort(p, buckets, perm, undo, counts, scratch, st);
   e = cudaFreeAsync(scratch, st);

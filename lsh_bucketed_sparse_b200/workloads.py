@@ -137,6 +137,15 @@ def make_inputs(wl: Workload, seed: Optional[int] = None):
     return qk.to(wl.dtype).contiguous(), v.to(wl.dtype).contiguous(), rot
 
 
+def make_centroids(wl: Workload, seed: Optional[int] = None):
+    """Centroids [n_hashes, d_k, n_buckets] for the routing-style assignment:
+    float32 N(0, 1) from their own generator (seed + 10000, so qk, v and the
+    rotations of make_inputs are unchanged), cast to ``wl.dtype``."""
+    gen = torch.Generator().manual_seed((wl.seed if seed is None else seed) + 10000)
+    c = torch.randn(wl.n_hashes, wl.d_k, wl.n_buckets, generator=gen, dtype=torch.float32)
+    return c.to(wl.dtype).contiguous()
+
+
 def small(name="tiny", batch=1, heads=2, seq_len=256, d_k=64, n_hashes=2, n_buckets=16,
           chunk_len=64, causal=True, dtype=torch.bfloat16, seed=7, clustered=False,
           n_clusters=16) -> Workload:

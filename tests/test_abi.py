@@ -87,7 +87,7 @@ def test_workspace_size_and_too_small(L):
 
 def test_unknown_flag_rejected(L):
     shp = shape()
-    shp.flags = 8  # bits 0-2 are LSH_FLAG_PORTABLE, _DEDUP, _BUCKET_MASK
+    shp.flags = 16  # bits 0-3 are LSH_FLAG_PORTABLE, _DEDUP, _BUCKET_MASK, _KMEANS
     assert fwd(L, shp) == 1
 
 

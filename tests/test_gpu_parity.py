@@ -433,3 +433,67 @@ def test_bucket_mask_matches_oracle(wl, dedup):
     P.check_lse(lse_r, res["lse_rounds"], bf16, "lse_rounds")
     P.check_float(out, res["out"], bf16, "out")
     P.check_lse(lse, res["lse"], bf16, "lse")
+
+
+# ---------------------------------------------------------------------------
+# Routing-style assignment (LSH_FLAG_KMEANS): argmax over given centroids.
+KMEANS = [
+    W.small("kmeans-bf16-causal", heads=2, seq_len=512, n_hashes=3, n_buckets=24),
+    W.small("kmeans-f32-noncausal-odd", heads=1, seq_len=256, n_hashes=2, n_buckets=7,
+            causal=False, dtype=torch.float32, chunk_len=32),
+    W.small("kmeans-bf16-d128-wide", heads=2, seq_len=256, d_k=128, n_hashes=2, n_buckets=300),
+    # multiples of 32 centroids take the tensor-core hash: 64-column rounds and
+    # a ragged tile, 96-column rounds with d = 128, 512-column rounds
+    W.small("kmeans-tc-p64", heads=2, seq_len=1088, n_hashes=3, n_buckets=64),
+    W.small("kmeans-tc-p96-d128", heads=2, seq_len=512, d_k=128, n_hashes=2, n_buckets=96,
+            chunk_len=128, causal=False),
+    W.small("kmeans-tc-p512", heads=2, seq_len=640, n_hashes=2, n_buckets=512),
+]
+
+
+@pytest.mark.parametrize("wl", KMEANS, ids=[w.name for w in KMEANS])
+def test_kmeans_assignment_matches_oracle(wl):
+    qk, v, _ = W.make_inputs(wl)
+    cen = W.make_centroids(wl)
+    qk_d, v_d, cen_d = qk.to(DEV), v.to(DEV), cen.to(DEV)
+    b, inv = lsh.lsh_attn_hash(qk_d, cen_d, wl.n_buckets, wl.n_hashes, kmeans=True)
+    ob, margins = O.hash_all(qk, cen, wl.n_buckets, kmeans=True)
+    report = P.check_buckets(b, ob, margins)
+    assert len(np.unique(ob)) > 1
+    out, lse = lsh.lsh_attn_forward(qk_d, v_d, cen_d, wl.n_hashes, wl.n_buckets, wl.chunk_len,
+                                    wl.causal, kmeans=True)
+    lsh.lsh_attn_device_check()
+    res = O.forward(qk, v, cen, wl.n_buckets, wl.chunk_len, wl.causal,
+                    buckets=b.cpu().numpy().astype(np.int64))
+    bf16 = wl.dtype == torch.bfloat16
+    P.check_float(out, res["out"], bf16, "out")
+    P.check_lse(lse, res["lse"], bf16, "lse")
+    print(wl.name, report)
+
+
+@pytest.mark.parametrize("n_buckets", [64, 96, 512])
+def test_kmeans_breaks_exact_ties_by_lowest_index(n_buckets):
+    # centroid 3 (scaled by 4, so it usually wins) repeated at a later column
+    # of the same and of another 32-column chunk: the lowest column must win
+    wl = W.small(f"kmeans-ties-{n_buckets}", heads=2, seq_len=640, n_hashes=2,
+                 n_buckets=n_buckets)
+    qk, _, _ = W.make_inputs(wl)
+    cen = W.make_centroids(wl).clone()
+    cen[:, :, 3] *= 4
+    for j in (7, 35, min(70, n_buckets - 1)):
+        cen[:, :, j] = cen[:, :, 3]
+    b, _ = lsh.lsh_attn_hash(qk.to(DEV), cen.to(DEV), wl.n_buckets, wl.n_hashes, kmeans=True)
+    b = b.cpu().numpy().astype(np.int64)
+    x, C = P.np64(qk), P.np64(cen)
+    checked = 0
+    for h in range(wl.heads):
+        for r in range(wl.n_hashes):
+            pr = x[0, h] @ C[r]
+            top = pr.max(1, keepdims=True)
+            below = np.where(pr < top, pr, -np.inf).max(1)
+            clear = (top[:, 0] - below) >= 1e-5
+            want = np.argmax(pr, axis=1)
+            ok = b[0, h, r] == want
+            assert ok[clear].all(), np.nonzero(~ok & clear)[0][:10]
+            checked += int(clear.sum())
+    assert checked > 0.9 * wl.heads * wl.n_hashes * wl.seq_len
