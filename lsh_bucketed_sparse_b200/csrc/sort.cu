@@ -26,6 +26,7 @@ constexpr int kTileKeys = 2048;
 constexpr int kCountThreads = 256;
 constexpr int kScanThreads = 1024;
 constexpr int kBatch = 16;  // rows of 32 keys loaded ahead in the scatter
+constexpr int kScanBatch = 16;  // tiles loaded ahead in the scan
 
 __global__ void __launch_bounds__(kCountThreads)
 sort_count_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ cnt, int L,
@@ -93,12 +94,21 @@ sort_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ counts, int n_
   extern __shared__ int32_t base[];  // [n_b]
   const int seg = blockIdx.x;
   int32_t* c = cnt + (size_t)seg * T * n_b;
+  // Both passes walk the tiles kScanBatch at a time with all of a batch's
+  // loads issued before any is used, so a thread waits on memory once per
+  // batch rather than once per tile.
   for (int b = threadIdx.x; b < n_b; b += blockDim.x) {
     int32_t run = 0;
-    for (int t = 0; t < T; ++t) {
-      const int32_t x = c[(size_t)t * n_b + b];
-      c[(size_t)t * n_b + b] = run;
-      run += x;
+    for (int t0 = 0; t0 < T; t0 += kScanBatch) {
+      int32_t x[kScanBatch];
+#pragma unroll
+      for (int k = 0; k < kScanBatch; ++k)
+        x[k] = t0 + k < T ? c[(size_t)(t0 + k) * n_b + b] : 0;
+#pragma unroll
+      for (int k = 0; k < kScanBatch; ++k) {
+        if (t0 + k < T) c[(size_t)(t0 + k) * n_b + b] = run;
+        run += x[k];
+      }
     }
     base[b] = run;
     if (counts) counts[(size_t)seg * n_b + b] = run;
@@ -106,8 +116,16 @@ sort_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ counts, int n_
   __syncthreads();
   block_exclusive_scan(base, n_b);  // base[b] = first slot of bucket b
   for (int b = threadIdx.x; b < n_b; b += blockDim.x) {
-    const int32_t x = base[b];
-    for (int t = 0; t < T; ++t) c[(size_t)t * n_b + b] += x;
+    const int32_t add = base[b];
+    for (int t0 = 0; t0 < T; t0 += kScanBatch) {
+      int32_t x[kScanBatch];
+#pragma unroll
+      for (int k = 0; k < kScanBatch; ++k)
+        x[k] = t0 + k < T ? c[(size_t)(t0 + k) * n_b + b] : 0;
+#pragma unroll
+      for (int k = 0; k < kScanBatch; ++k)
+        if (t0 + k < T) c[(size_t)(t0 + k) * n_b + b] = x[k] + add;
+    }
   }
 }
 
