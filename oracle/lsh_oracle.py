@@ -32,6 +32,9 @@ Readings where the pages are silent (each is also listed in the design notes):
   * n_buckets == 1 puts every token in bucket 0 and needs no rotations;
   * the first chunk of a round has no look-back (no wrap to the last chunk,
     no crossing into another round);
+  * when chunk_len does not divide L the last chunk holds the remaining
+    L mod chunk_len slots (as if padded with slots that neither attend nor
+    are attended);
   * no bucket-equality mask inside a window: the window is the attended set
     (``bucket_mask=True`` is the variant that also drops the window's keys
     whose bucket in that round differs from the query's, section 2 "LSH
@@ -117,10 +120,11 @@ def normalised_keys(x: np.ndarray) -> np.ndarray:
     return np.where(n[:, None] > 0, x / safe[:, None], 0.0)
 
 
-def window_slots(k: int, chunk_len: int):
-    """Sorted slots a query in chunk k attends: chunk k-1 (if k > 0) and chunk k."""
+def window_slots(k: int, chunk_len: int, L: int):
+    """Sorted slots a query in chunk k attends: chunk k-1 (if k > 0) and chunk
+    k; the last chunk ends at L when chunk_len does not divide L."""
     lo = (k - 1) * chunk_len if k > 0 else 0
-    return lo, (k + 1) * chunk_len
+    return lo, min((k + 1) * chunk_len, L)
 
 
 def attend_round(x, v, perm_r, chunk_len: int, causal: bool, dedup_undo=None,
@@ -136,15 +140,14 @@ def attend_round(x, v, perm_r, chunk_len: int, causal: bool, dedup_undo=None,
     """
     L, d = x.shape
     c = chunk_len
-    assert L % c == 0
-    n_c = L // c
+    n_c = -(-L // c)  # the last chunk holds the L mod c remaining slots
     khat = normalised_keys(x)
     xs, ks, vs, pos = x[perm_r], khat[perm_r], v[perm_r], perm_r
     o = np.empty((L, d))
     lse = np.empty(L)
     for k in range(n_c):
-        q0, q1 = k * c, (k + 1) * c
-        k0, k1 = window_slots(k, c)
+        q0, q1 = k * c, min((k + 1) * c, L)
+        k0, k1 = window_slots(k, c, L)
         s = xs[q0:q1] @ ks[k0:k1].T / math.sqrt(d)
         qp = pos[q0:q1][:, None]
         kp = pos[k0:k1][None, :]
@@ -320,7 +323,7 @@ def token_rounds(x, v, perm, undo, chunk_len, causal, i):
     xi = x[i]
     for r in range(n_h):
         k = undo[r, i] // chunk_len
-        k0, k1 = window_slots(k, chunk_len)
+        k0, k1 = window_slots(k, chunk_len, x.shape[0])
         kp = perm[r, k0:k1]
         keys = normalised_keys(x[kp])
         s = keys @ xi / math.sqrt(d)

@@ -14,12 +14,13 @@ from oracle import lsh_oracle as O
 import test_oracle_pins as P
 
 
-def _no_lookback(k, chunk_len):
-    return k * chunk_len, (k + 1) * chunk_len
+def _no_lookback(k, chunk_len, L):
+    return k * chunk_len, min((k + 1) * chunk_len, L)
 
 
-def _wrap_lookback(k, chunk_len):
-    return (k - 1) * chunk_len if k > 0 else 0, (k + 1) * chunk_len + (chunk_len if k == 0 else 0)
+def _wrap_lookback(k, chunk_len, L):
+    return (k - 1) * chunk_len if k > 0 else 0, \
+        min((k + 1) * chunk_len + (chunk_len if k == 0 else 0), L)
 
 
 def _unnormalised_keys(x):

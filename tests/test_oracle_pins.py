@@ -237,7 +237,9 @@ def _brute_force(x, v, buckets, c, causal):
 
 @pytest.mark.parametrize("L,c,n_b,n_h,causal", [
     (16, 4, 4, 2, True), (24, 8, 6, 3, False), (64, 8, 8, 2, True), (32, 32, 4, 1, False),
-    (48, 8, 2, 4, True)])
+    (48, 8, 2, 4, True),
+    # chunk_len not dividing L: the last chunk is short
+    (20, 8, 4, 2, True), (30, 8, 6, 3, False), (50, 16, 8, 2, True), (7, 16, 4, 2, False)])
 def test_brute_force_small(L, c, n_b, n_h, causal):
     rng = np.random.default_rng(L * 7 + n_b)
     d = 6
