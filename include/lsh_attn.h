@@ -103,11 +103,12 @@ typedef enum lsh_dtype {
 typedef struct lsh_shape {
   int32_t batch;       /* B >= 1                                             */
   int32_t heads;       /* H >= 1                                             */
-  int32_t seq_len;     /* L >= 1, a multiple of chunk_len, < 2^31 / n_h      */
+  int32_t seq_len;     /* L >= 1, < 2^31 / n_h                                */
   int32_t d_k;         /* d: 8..256, a multiple of 8                         */
   int32_t n_hashes;    /* n_h >= 1 hashing rounds                            */
   int32_t n_buckets;   /* n_b: 1, or even with 2 <= n_b <= 32768             */
-  int32_t chunk_len;   /* c >= 1, divides L                                  */
+  int32_t chunk_len;   /* c >= 1; when c does not divide L the last chunk of
+                          the sorted order holds the L mod c remaining slots */
   int32_t causal;      /* 0 or 1                                             */
   int32_t dtype;       /* lsh_dtype of the floating-point tensors            */
   uint32_t flags;      /* LSH_FLAG_* bits, 0 by default                      */

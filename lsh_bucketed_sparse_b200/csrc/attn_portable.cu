@@ -35,7 +35,7 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                      float* __restrict__ lse_rounds, int L, int d, int n_h, int c, int causal,
                      float scale) {
   extern __shared__ float q_all[];  // [kWarps][d]
-  const int n_c = L / c;
+  const int n_c = (L + c - 1) / c;  // the last chunk may be short
   const int k = (int)(blockIdx.x % n_c);
   const int r = (int)((blockIdx.x / n_c) % n_h);
   const size_t bh = blockIdx.x / ((size_t)n_c * n_h);
@@ -47,10 +47,10 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   const int32_t* UD = undo ? undo + bh * (size_t)n_h * L : nullptr;  // [n_h][L]
   const int16_t* BK = bkt ? bkt + (bh * n_h + r) * (size_t)L : nullptr;  // this round
   float* qs = q_all + warp * d;
-  const int k0 = k > 0 ? (k - 1) * c : 0, k1 = (k + 1) * c;
+  const int k0 = k > 0 ? (k - 1) * c : 0, k1 = min((k + 1) * c, L);
   constexpr int kPer = kMaxD / 32;
 
-  for (int qslot = k * c + warp; qslot < (k + 1) * c; qslot += kWarps) {
+  for (int qslot = k * c + warp; qslot < k1; qslot += kWarps) {
     const int i = P[qslot];
     for (int e = lane; e < d; e += 32) qs[e] = to_f32(X[(size_t)i * d + e]);
     __syncwarp();

@@ -21,7 +21,7 @@ struct Problem {
   bool kmeans;       // LSH_FLAG_KMEANS: argmax over n_b given centroids
   int BH() const { return B * H; }
   int half() const { return n_b / 2; }  // projections per round, 0 when n_b == 1
-  int n_chunks() const { return L / c; }
+  int n_chunks() const { return (L + c - 1) / c; }  // the last one may be short
   size_t elem() const { return bf16 ? 2 : 4; }
 };
 

@@ -55,9 +55,7 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
       !(s->n_buckets == 1 || (s->n_buckets >= 2 && s->n_buckets <= 32768 && s->n_buckets % 2 == 0)))
     return fail(LSH_ERR_INVALID_ARG, "n_buckets=%d: must be 1 or even in [2, 32768]",
                 s->n_buckets);
-  if (s->chunk_len < 1 || s->seq_len % s->chunk_len)
-    return fail(LSH_ERR_INVALID_ARG, "chunk_len=%d must be >= 1 and divide seq_len=%d",
-                s->chunk_len, s->seq_len);
+  if (s->chunk_len < 1) return fail(LSH_ERR_INVALID_ARG, "chunk_len=%d must be >= 1", s->chunk_len);
   if (s->causal != 0 && s->causal != 1) return fail(LSH_ERR_INVALID_ARG, "causal must be 0 or 1");
   if (s->dtype != LSH_F32 && s->dtype != LSH_BF16)
     return fail(LSH_ERR_INVALID_ARG, "dtype=%d: must be LSH_F32 or LSH_BF16", s->dtype);
@@ -65,7 +63,8 @@ lsh_status to_problem(const lsh_shape* s, Problem* p) {
     return fail(LSH_ERR_INVALID_ARG, "unknown flag bits");
   const long long bh = (long long)s->batch * s->heads;
   if (bh > (1LL << 30)) return fail(LSH_ERR_INVALID_ARG, "batch*heads too large");
-  const long long chunks = bh * s->n_hashes * (s->seq_len / s->chunk_len);
+  const long long chunks =
+      bh * s->n_hashes * ((s->seq_len + s->chunk_len - 1) / s->chunk_len);
   if (chunks >= (1LL << 31) || (long long)s->n_hashes * s->seq_len >= (1LL << 31))
     return fail(LSH_ERR_INVALID_ARG, "problem too large for 32-bit grid/slot indices");
   p->B = s->batch; p->H = s->heads; p->L = s->seq_len; p->d = s->d_k;

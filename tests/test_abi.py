@@ -50,7 +50,7 @@ def fwd(L, shp, ws_bytes=1 << 40, rot=FAKE, ws=FAKE, qk=FAKE):
 
 
 @pytest.mark.parametrize("kw", [
-    dict(seq_len=250),            # chunk_len does not divide seq_len
+    dict(seq_len=0), dict(chunk_len=-1),
     dict(d_k=60), dict(d_k=264), dict(d_k=0),
     dict(n_buckets=7), dict(n_buckets=0), dict(n_buckets=65536),
     dict(n_hashes=0), dict(batch=0), dict(chunk_len=0),
@@ -59,6 +59,14 @@ def fwd(L, shp, ws_bytes=1 << 40, rot=FAKE, ws=FAKE, qk=FAKE):
 def test_bad_shape_is_rejected(L, kw):
     assert fwd(L, shape(**kw)) == 1
     assert L.lsh_attn_last_error()
+
+
+def test_chunk_len_need_not_divide_seq_len(L):
+    # the last chunk of the sorted order is short; the workspace covers it
+    shp = shape(seq_len=250)
+    n = ctypes.c_size_t()
+    assert L.lsh_attn_forward_workspace_size(ctypes.byref(shp), ctypes.byref(n)) == 0
+    assert n.value > 0
 
 
 def test_bad_causal_flag_is_rejected(L):

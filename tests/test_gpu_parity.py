@@ -104,6 +104,14 @@ SMALL = [
     # 384-column rounds that end inside a piece
     W.small("tc-hash-p256", heads=2, seq_len=1088, n_hashes=3, n_buckets=512),
     W.small("tc-hash-p384", heads=2, seq_len=1088, n_hashes=2, n_buckets=768),
+    # chunk_len not dividing L: the last chunk of the sorted order is short
+    W.small("ragged-chunk-c64-L1000", heads=2, seq_len=1000, n_hashes=2, n_buckets=32),
+    W.small("ragged-chunk-c128-d128-L1500", heads=1, seq_len=1500, d_k=128, n_hashes=2,
+            n_buckets=64, chunk_len=128, causal=False),
+    W.small("ragged-chunk-c64-tc-hash-L1100", heads=2, seq_len=1100, n_hashes=3,
+            n_buckets=128),
+    W.small("ragged-chunk-f32-c48-L500", heads=2, seq_len=500, n_hashes=2, n_buckets=16,
+            chunk_len=48, dtype=torch.float32),
     # the four tensor-core attention specialisations (chunk, d_k)
     W.small("tc-attn-c64-d128", heads=2, seq_len=1472, d_k=128, n_hashes=2, n_buckets=64),
     W.small("tc-attn-c128-d64-causal", heads=2, seq_len=1408, n_hashes=3, n_buckets=64,
