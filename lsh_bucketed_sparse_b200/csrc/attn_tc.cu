@@ -83,6 +83,7 @@ struct Params {
   const __nv_bfloat16* v;
   __nv_bfloat16* o_rounds;
   float* lse_rounds;
+  const int16_t* buckets;  // [BH, n_h, L] bucket ids for the bucket-equality mask, else null
   unsigned int* err;
   int L, n_h, causal;
   int steps;          // ceil(L / 128) per segment
@@ -93,7 +94,7 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, p, pos, ksc, qref, xch, bars, misc, total;
+  uint32_t qk, v, p, pos, ksc, qref, bkt, xch, bars, misc, total;
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
@@ -101,7 +102,7 @@ __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
   return 2 * nq + 2 * nv + 2 * kMetaSlots + 12 + 8 + 4 + 1;
 }
 
-template <int C, int D>
+template <int C, int D, bool BM = false>
 __host__ __device__ constexpr Layout layout(int nq, int nv, int np) {
   using K = Cfg<C, D>;
   Layout l{};
@@ -112,6 +113,7 @@ __host__ __device__ constexpr Layout layout(int nq, int nv, int np) {
   l.pos = off;  off += kMetaSlots * kQ * 4;
   l.ksc = off;  off += kMetaSlots * kQ * 4;
   l.qref = off; off += kMetaSlots * kQ * 4;
+  l.bkt = off;  off += BM ? kMetaSlots * kQ * 4 : 0;  // bucket ids (bucket-equality mask)
   l.xch = off;  off += (2 * 2 + 2 + 2) * kQ * 4;   // partial sums [2][2], maxima [2], redo sums [2]
   l.bars = off; off += n_barriers(nq, nv) * 8;
   l.misc = off; off += 16;
@@ -239,24 +241,27 @@ struct Plan {
   bool ok;
 };
 
-template <int C, int D>
+template <int C, int D, bool BM = false>
 __host__ __device__ constexpr Plan make_plan() {
   constexpr uint32_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
   for (int pb = 2; pb >= 1; --pb) {
-    const uint32_t fixed = layout<C, D>(0, 0, pb).total + n_barriers(6, 6) * 8;
+    const uint32_t fixed = layout<C, D, BM>(0, 0, pb).total + n_barriers(6, 6) * 8;
     if (fixed >= limit) continue;
     const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
     if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
     const int q = (tiles + 1) / 2 < 5 ? (tiles + 1) / 2 : 5;
     const int v = tiles - q < 5 ? tiles - q : 5;
-    uint32_t smem = layout<C, D>(q, v, pb).total + 1024;
+    uint32_t smem = layout<C, D, BM>(q, v, pb).total + 1024;
     if (smem < 116 * 1024) smem = 116 * 1024;
     return Plan{q, v, pb, smem, smem <= (uint32_t)kSmemLimit};
   }
   return Plan{0, 0, 0, 0, false};
 }
 
-template <int C, int D, bool CAUSAL>
+// BMASK: the bucket-equality mask variant (section 2 "LSH attention": a
+// query attends only to targets in its own hash bucket): a key whose bucket
+// in this round differs from the query's is not visible.
+template <int C, int D, bool CAUSAL, bool BMASK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
                const Params p) {
@@ -264,15 +269,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  constexpr Plan PL = make_plan<C, D>();
+  constexpr Plan PL = make_plan<C, D, BMASK>();
   constexpr int NQ = PL.nq, NV = PL.nv, NP = PL.np, NM = kMetaSlots;
-  constexpr Layout Ly = layout<C, D>(NQ, NV, NP);
+  constexpr Layout Ly = layout<C, D, BMASK>(NQ, NV, NP);
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
   uint8_t* p_s = smem + Ly.p;
   int* pos_s = reinterpret_cast<int*>(smem + Ly.pos);
   float* ksc_s = reinterpret_cast<float*>(smem + Ly.ksc);
   float* qref_s = reinterpret_cast<float*>(smem + Ly.qref);
+  int* bkt_s = reinterpret_cast<int*>(smem + Ly.bkt);
   float* xl = reinterpret_cast<float*>(smem + Ly.xch);  // [2 buf][2 half][kQ]
   float* xm = xl + 4 * kQ;                              // [2 half][kQ]
   float* xl2 = xm + 2 * kQ;                             // [2 half][kQ]
@@ -346,22 +352,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     cursor_next(c2, p, u_step);
     int pos0[4], pos1[4];
     float in0[4];
+    int bk0[4];
     cursor_positions(c0, p, lane, pos0);
     cursor_positions(c1, p, lane, pos1);
+    // bucket id of a row in its round (-1 for a missing row: matches nothing)
+    auto bucket_of = [&](const Cursor& c, int pos) -> int {
+      if (!BMASK || !c.valid || pos == INT_MAX) return -1;
+      return p.buckets[((size_t)c.U.bh * p.n_h + c.U.r) * p.L + pos];
+    };
 #pragma unroll
-    for (int k = 0; k < 4; ++k)
+    for (int k = 0; k < 4; ++k) {
       in0[k] = pos0[k] != INT_MAX ? p.inv_norm[(size_t)c0.U.bh * p.L + pos0[k]] : 0.f;
+      bk0[k] = bucket_of(c0, pos0[k]);
+    }
     int li = 0;
     bool ok = true;
     for (; ok && c0.valid; ++li) {
       // prefetch for the next two blocks
       int pos2[4];
       float in1[4];
+      int bk1[4];
       cursor_positions(c2, p, lane, pos2);
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < 4; ++k) {
         in1[k] = (c1.valid && pos1[k] != INT_MAX)
                      ? p.inv_norm[(size_t)c1.U.bh * p.L + pos1[k]] : 0.f;
+        bk1[k] = bucket_of(c1, pos1[k]);
+      }
       const int qs = (int)(li % NQ), ms = (int)(li % NM);
       if (!mbar_wait_spin(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
       if (!mbar_wait_spin(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
@@ -381,6 +398,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         pos_s[row] = pos0[k];
         ksc_s[row] = in0[k] * p.ksc;
         qref_s[row] = in0[k] > 0.f ? p.ksc / in0[k] : 0.f;
+        if (BMASK) bkt_s[row] = bk0[k];
       }
       mbar_arrive(&m_full[ms]);
 #pragma unroll
@@ -388,6 +406,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         pos0[k] = pos1[k];
         pos1[k] = pos2[k];
         in0[k] = in1[k];
+        bk0[k] = bk1[k];
       }
       c0 = c1;
       c1 = c2;
@@ -556,6 +575,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       tc_fence_after_sync();
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
+      const int qb = BMASK ? bkt_s[cs * kQ + m] : 0;
       const int qlim = p.causal ? qpos : INT_MAX - 1;
       const int lo = has_prev ? win_lo : max(win_lo, C);
       // metadata row of key column j0 (a multiple of 32, all in one block)
@@ -575,13 +595,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           // Causal: a key is visible iff its position is below the query's
           // (one comparison, which also leaves the query itself out), and
           // the row sees some key iff the chunk's smallest position does.
-          if (CAUSAL) any |= __reduce_min_sync(0xffffffffu, pos_s[kb + lane]) < qpos;
+          if (CAUSAL && !BMASK) any |= __reduce_min_sync(0xffffffffu, pos_s[kb + lane]) < qpos;
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
             const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
             const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
             const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
             const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+            int kba[4] = {0, 0, 0, 0};
+            if (BMASK) {
+              const int4 kbv = *reinterpret_cast<const int4*>(bkt_s + kb + e);
+              kba[0] = kbv.x; kba[1] = kbv.y; kba[2] = kbv.z; kba[3] = kbv.w;
+            }
             float pr[4];
 #pragma unroll
             for (int h = 0; h < 4; ++h) {
@@ -590,8 +615,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 valid = kpa[h] < qpos;
               } else {
                 valid = kpa[h] <= qlim && kpa[h] != qpos;
-                any |= valid;
               }
+              if (BMASK) valid = valid && kba[h] == qb;
+              if (!CAUSAL || BMASK) any |= valid;
               const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
               pr[h] = valid ? ex2(x) : 0.f;
               la[h] += pr[h];
@@ -637,7 +663,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           const int kb = kbase(j0);
           for (int e = 0; e < 32; ++e) {
             const int kp = pos_s[kb + e];
-            if (kp <= qlim && kp != qpos) mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
+            if (kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e] == qb))
+              mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
           }
         }
         xm[half * kQ + m] = mx;
@@ -663,7 +690,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
               float pr[2];
               for (int g = 0; g < 2; ++g) {
                 const int kp = pos_s[kb + e + h + g];
-                const bool valid = kp <= qlim && kp != qpos;
+                const bool valid =
+                    kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e + h + g] == qb);
                 pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ksc_s[kb + e + h + g],
                                          -gmax))
                               : 0.f;
@@ -785,11 +813,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
 template <int C, int D>
 cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const float* inv_norm,
-                      const int32_t* perm, void* o_rounds, float* lse_rounds, cudaStream_t st) {
-  constexpr Plan PL = make_plan<C, D>();
-  static_assert(PL.ok, "no shared-memory plan for this (chunk, d)");
+                      const int32_t* perm, const int16_t* buckets, void* o_rounds,
+                      float* lse_rounds, cudaStream_t st) {
+  constexpr Plan PL = make_plan<C, D, false>();
+  constexpr Plan PLM = make_plan<C, D, true>();
+  static_assert(PL.ok && PLM.ok, "no shared-memory plan for this (chunk, d)");
   Params p;
-  const size_t smem = PL.smem;
+  const size_t smem = buckets ? PLM.smem : PL.smem;
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;
   p.v = static_cast<const __nv_bfloat16*>(v);
@@ -797,6 +827,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   p.perm = perm;
   p.o_rounds = static_cast<__nv_bfloat16*>(o_rounds);
   p.lse_rounds = lse_rounds;
+  p.buckets = buckets;
   p.err = err;
   p.L = pr.L;
   p.n_h = pr.n_h;
@@ -829,7 +860,11 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  auto kernel = pr.causal ? attn_tc_kernel<C, D, true> : attn_tc_kernel<C, D, false>;
+  const bool bmask = buckets != nullptr;
+  auto kernel = pr.causal ? (bmask ? attn_tc_kernel<C, D, true, true>
+                                   : attn_tc_kernel<C, D, true, false>)
+                          : (bmask ? attn_tc_kernel<C, D, false, true>
+                                   : attn_tc_kernel<C, D, false, false>);
   cudaError_t e = cudaFuncSetAttribute(kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -847,16 +882,17 @@ bool attn_tc_supported(const Problem& p) {
 }
 
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
-                           const int32_t* perm, void* o_rounds, float* lse_rounds,
-                           cudaStream_t st) {
+                           const int32_t* perm, const int16_t* buckets, void* o_rounds,
+                           float* lse_rounds, cudaStream_t st) {
+  if (!p.bucket_mask) buckets = nullptr;
   if (p.c == 64 && p.d == 64)
-    return launch_cd<64, 64>(p, qk, v, inv_norm, perm, o_rounds, lse_rounds, st);
+    return launch_cd<64, 64>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
   if (p.c == 64 && p.d == 128)
-    return launch_cd<64, 128>(p, qk, v, inv_norm, perm, o_rounds, lse_rounds, st);
+    return launch_cd<64, 128>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
   if (p.c == 128 && p.d == 64)
-    return launch_cd<128, 64>(p, qk, v, inv_norm, perm, o_rounds, lse_rounds, st);
+    return launch_cd<128, 64>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
   if (p.c == 128 && p.d == 128)
-    return launch_cd<128, 128>(p, qk, v, inv_norm, perm, o_rounds, lse_rounds, st);
+    return launch_cd<128, 128>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
   return cudaErrorNotSupported;
 }
 

@@ -119,15 +119,14 @@ lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
 }
 
-// The variants (duplicate-count correction, bucket-equality mask) run on the
-// CUDA-core kernel only.
+// The duplicate-count correction runs on the CUDA-core kernel only; the
+// bucket-equality mask on both.
 lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                     const int32_t* perm, const int32_t* undo, const int16_t* buckets,
                     void* o_r, float* lse_r, cudaStream_t st) {
-  const bool variant = p.dedup || p.bucket_mask;
   cudaError_t e =
-      (!p.portable && !variant && attn_tc_supported(p))
-          ? launch_attn_tc(p, qk, v, inv_norm, perm, o_r, lse_r, st)
+      (!p.portable && !p.dedup && attn_tc_supported(p))
+          ? launch_attn_tc(p, qk, v, inv_norm, perm, buckets, o_r, lse_r, st)
           : launch_attn_portable(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
 }

@@ -414,6 +414,12 @@ MASKED = [
              causal=False, dtype=torch.float32), False),
     (W.small("bmask-dedup-bf16-d128", heads=2, seq_len=256, d_k=128, n_hashes=3, n_buckets=4,
              chunk_len=32, causal=True), True),
+    # tensor-core attention with the mask: (c, d) = (128, 64) causal, (64, 128)
+    # non-causal with a short last chunk
+    (W.small("bmask-tc-c128-d64", heads=2, seq_len=1408, n_hashes=2, n_buckets=32,
+             chunk_len=128), False),
+    (W.small("bmask-tc-c64-d128-noncausal", heads=2, seq_len=1000, d_k=128, n_hashes=2,
+             n_buckets=16, causal=False), False),
 ]
 
 
