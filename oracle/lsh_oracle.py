@@ -336,3 +336,67 @@ def token_rounds(x, v, perm, undo, chunk_len, causal, i):
         o[r] = (e / l) @ v[kp]
         lse[r] = m + np.log(l)
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# 6. Backward (the survey's "next" row f3; no gradient through hash or sort)
+# ---------------------------------------------------------------------------
+def backward_head(x, v, perm, chunk_len: int, causal: bool, dout):
+    """Gradients of out w.r.t. the shared qk and v of one (batch, head), with
+    the buckets and their sort held fixed (the hash is piecewise constant).
+
+    The forward is re-stated in float64 torch, step for step as attend_round
+    and combine_head do it (windows of chunks k-1 and k in sorted order,
+    normalised keys, 1/sqrt(d), self score -1e5 as a constant, causal mask,
+    per-round logsumexp, combine over rounds); autograd then gives
+    (d qk [L, d], d v [L, d]) for the upstream gradient dout [L, d].  The
+    tests pin it against central finite differences and the numpy forward.
+    """
+    import torch
+    X = torch.tensor(np.asarray(x, np.float64), requires_grad=True)
+    V = torch.tensor(np.asarray(v, np.float64), requires_grad=True)
+    n_h, L = np.asarray(perm).shape
+    d = X.shape[1]
+    c = chunk_len
+    norm = torch.sqrt((X * X).sum(1))
+    K = torch.where(norm[:, None] > 0, X / torch.where(norm > 0, norm, 1.0)[:, None],
+                    torch.zeros_like(X))
+    outs, lses = [], []
+    for r in range(n_h):
+        pr = torch.as_tensor(np.asarray(perm)[r], dtype=torch.long)
+        o_r = torch.zeros(L, d, dtype=torch.float64)
+        l_r = torch.zeros(L, dtype=torch.float64)
+        for k in range(-(-L // c)):
+            q0, q1 = k * c, min((k + 1) * c, L)
+            k0, k1 = (k - 1) * c if k > 0 else 0, min((k + 1) * c, L)
+            qi, kj = pr[q0:q1], pr[k0:k1]
+            s = X[qi] @ K[kj].T / math.sqrt(d)
+            same = qi[:, None] == kj[None, :]
+            s = torch.where(same, torch.full_like(s, SELF_SCORE), s)
+            if causal:
+                s = torch.where(kj[None, :] > qi[:, None], torch.full_like(s, -math.inf), s)
+            lse = torch.logsumexp(s, dim=1)
+            p = torch.exp(s - lse[:, None])
+            o_r = o_r.index_put((qi,), p @ V[kj])
+            l_r = l_r.index_put((qi,), lse)
+        outs.append(o_r)
+        lses.append(l_r)
+    O = torch.stack(outs)                       # [n_h, L, d]
+    Lr = torch.stack(lses)                      # [n_h, L]
+    w = torch.softmax(Lr, dim=0)                # exp(lse_r - LSE)
+    out = (w[:, :, None] * O).sum(0)
+    out.backward(torch.as_tensor(np.asarray(dout, np.float64)))
+    return X.grad.numpy(), V.grad.numpy()
+
+
+def backward_all(qk, v, perm, chunk_len, causal, dout):
+    """[B, H, L, d] gradients of out for fixed perm [B, H, n_h, L]."""
+    qk, v, dout = as_f64(qk), as_f64(v), as_f64(dout)
+    perm = np.asarray(perm)
+    dq = np.empty_like(qk)
+    dv = np.empty_like(v)
+    for b in range(qk.shape[0]):
+        for h in range(qk.shape[1]):
+            dq[b, h], dv[b, h] = backward_head(qk[b, h], v[b, h], perm[b, h], chunk_len, causal,
+                                               dout[b, h])
+    return dq, dv

@@ -436,3 +436,57 @@ def test_kmeans_picks_the_largest_coordinate_with_basis_centroids():
     b, m = O.kmeans_head(x, C, 4)
     np.testing.assert_array_equal(b[0], [1, 2, 0])
     np.testing.assert_allclose(m[0], [0.0, 0.5, 0.0])
+
+
+# ------------------------------------------------------------- backward --
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_finite_differences(causal):
+    # d out . g w.r.t. qk and v by central differences, the buckets and their
+    # sort held fixed (the hash does not move for steps this small)
+    rng = np.random.default_rng(41)
+    L, d, c, n_h, n_b = 20, 4, 4, 2, 4
+    x = rng.standard_normal((1, 1, L, d))
+    v = rng.standard_normal((1, 1, L, d))
+    R = rng.standard_normal((n_h, d, n_b // 2))
+    g = rng.standard_normal((L, d))
+    res = O.forward(x, v, R, n_b, c, causal)
+    perm = res["perm"][0, 0]
+    buckets = res["buckets"]
+    dq, dv = O.backward_head(x[0, 0], v[0, 0], perm, c, causal, g)
+    h = 1e-6
+
+    def f(xx, vv):
+        r = O.forward(xx, vv, R, n_b, c, causal, buckets=buckets)
+        return float((r["out"][0, 0] * g).sum())
+
+    for (i, t) in [(0, 0), (3, 1), (7, 2), (12, 3), (19, 0)]:
+        xp, xm = x.copy(), x.copy()
+        xp[0, 0, i, t] += h
+        xm[0, 0, i, t] -= h
+        np.testing.assert_allclose(dq[i, t], (f(xp, v) - f(xm, v)) / (2 * h), rtol=1e-5,
+                                   atol=1e-7)
+        vp, vm = v.copy(), v.copy()
+        vp[0, 0, i, t] += h
+        vm[0, 0, i, t] -= h
+        np.testing.assert_allclose(dv[i, t], (f(x, vp) - f(x, vm)) / (2 * h), rtol=1e-5,
+                                   atol=1e-7)
+
+
+def test_backward_of_v_is_the_attention_transpose():
+    # out is linear in v: d v_j = sum_i A_ij g_i with A the combined attention
+    # weights, which the multiset form gives from the membership counts
+    rng = np.random.default_rng(42)
+    L, d, c, n_h, n_b = 32, 4, 8, 3, 4
+    x = rng.standard_normal((1, 1, L, d))
+    v = rng.standard_normal((1, 1, L, d))
+    R = rng.standard_normal((n_h, d, n_b // 2))
+    g = rng.standard_normal((L, d))
+    res = O.forward(x, v, R, n_b, c, True)
+    _, dv = O.backward_head(x[0, 0], v[0, 0], res["perm"][0, 0], c, True, g)
+    # A_ij from the same forward with v = e_j (linearity in v)
+    A = np.empty((L, L))
+    for j in range(L):
+        e = np.zeros((1, 1, L, 1))
+        e[0, 0, j, 0] = 1.0
+        A[:, j] = O.forward(x, e, R, n_b, c, True, buckets=res["buckets"])["out"][0, 0, :, 0]
+    np.testing.assert_allclose(dv, A.T @ g, rtol=1e-10, atol=1e-12)
