@@ -211,6 +211,30 @@ LSH_ATTN_API lsh_status lsh_attn_forward(const lsh_shape* shape, const void* qk,
                             size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- *
+ * Backward of the forward pass with the buckets and their sort held fixed
+ * (the hash is piecewise constant: no gradient flows through bucket ids).
+ * Gradients of `out` w.r.t. the shared qk and v for an upstream gradient
+ * dout, from the multiset form of the combined output (section 2 "LSH
+ * attention", Appendix A): with LSE the forward's lse output,
+ *   dv_j  += exp(s_ij - LSE_i) dout_i                 over every window pair,
+ *   ds_ij  = exp(s_ij - LSE_i) (dout_i . v_j - dout_i . out_i),
+ * into the query and the normalised key (the self pair's -1e5 is a constant).
+ *   qk, v, out, dout [B, H, L, d] dtype in; inv_norm [B, H, L] float32 and
+ *   perm [B, H, n_h, L] int32 from stages 1-2; lse [B, H, L] float32 from
+ *   the combine; dqk, dv [B, H, L, d] float32 out.
+ *   workspace: at least lsh_attn_backward_workspace_size() bytes, 256-byte
+ *   aligned.  CUDA cores with float32 atomics (the summation order, and so
+ *   the last bits, can differ between runs).  The variant flags are not
+ *   supported here (LSH_ERR_UNSUPPORTED).
+ * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_backward_workspace_size(const lsh_shape* shape, size_t* bytes);
+
+LSH_ATTN_API lsh_status lsh_attn_backward(const lsh_shape* shape, const void* qk, const void* v,
+                             const float* inv_norm, const int32_t* perm, const void* out,
+                             const float* lse, const void* dout, float* dqk, float* dv,
+                             void* workspace, size_t workspace_bytes, void* stream);
+
+/* ---------------------------------------------------------------------- *
  * The forward pass from HOST buffers: copies qk, v and rotations to the
  * device, runs the forward pass, and copies out and lse back.  The (batch,
  * head) pairs are independent, so they go in up to 8 groups through three

@@ -24,6 +24,7 @@ __all__ = [
     "lsh_attn_chunked_fwd", "lsh_attn_chunked_fwd_ex", "lsh_attn_combine", "lsh_attn_forward",
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
     "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
+    "lsh_attn_backward", "lsh_attn_backward_workspace_size",
     "LIB_PATH", "HEADER_PATH", "NOALLOC_SCRATCH_BYTES",
     "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP", "FLAG_BUCKET_MASK", "FLAG_KMEANS",
 ]
@@ -71,6 +72,8 @@ _SIGS = {
     "lsh_attn_forward_host_device_bytes": [_SHP, ctypes.POINTER(_SZ)],
     "lsh_attn_forward_host": [_SHP, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "lsh_attn_forward_noalloc": [_SHP, _P, _P, _P, _P, _P, _P],
+    "lsh_attn_backward_workspace_size": [_SHP, ctypes.POINTER(_SZ)],
+    "lsh_attn_backward": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
     "lsh_attn_status_string": [ctypes.c_int],
     "lsh_attn_last_error": [],
     "lsh_attn_device_check": [_P],
@@ -320,3 +323,35 @@ def lsh_attn_forward_noalloc(qk, v, rotations, n_hashes, n_buckets, chunk_len, c
 def lsh_attn_device_check(stream=None):
     """Synchronise the stream and raise if a kernel's bounded wait ran out."""
     _check(lib().lsh_attn_device_check(_stream(stream)))
+
+
+def lsh_attn_backward_workspace_size(shape: Shape) -> int:
+    n = _SZ()
+    _check(lib().lsh_attn_backward_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
+
+
+def lsh_attn_backward(qk, v, inv_norm, perm, out, lse, dout, chunk_len, causal, *,
+                      n_buckets=2, workspace=None, stream=None):
+    """Gradients of out w.r.t. qk and v with the buckets and sort held fixed.
+    perm [B,H,n_h,L] and inv_norm from stages 1-2, out and lse from the
+    forward.  Returns (dqk, dv), float32 [B,H,L,d]."""
+    _cuda(qk, "qk")
+    _cuda(v, "v", qk.dtype)
+    _cuda(inv_norm, "inv_norm", torch.float32)
+    _cuda(perm, "perm", torch.int32)
+    _cuda(out, "out", qk.dtype)
+    _cuda(lse, "lse", torch.float32)
+    _cuda(dout, "dout", qk.dtype)
+    B, H, n_h, L = perm.shape
+    shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, False)
+    need = lsh_attn_backward_workspace_size(shp)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=qk.device)
+    dqk = torch.empty(qk.shape, dtype=torch.float32, device=qk.device)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=qk.device)
+    _check(lib().lsh_attn_backward(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(inv_norm),
+                                   _ptr(perm), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dqk),
+                                   _ptr(dv), _ptr(workspace), _SZ(workspace.numel()),
+                                   _stream(stream)))
+    return dqk, dv

@@ -1,0 +1,199 @@
+// Backward of the forward pass with the hash and the sort held fixed (the
+// hash is piecewise constant, so no gradient flows through bucket ids; the
+// survey's "next" row f3).  "Reformer: The Efficient Transformer", section 2
+// "LSH attention" and Appendix A define the forward; its gradient follows
+// from the multiset form of the combined output,
+//   out_i = sum_r sum_{j in W_r(i)} exp(s_ij - LSE_i) v_j,
+// where W_r(i) is i's window in round r and LSE_i the combined log-sum-exp:
+//   dv_j     += exp(s_ij - LSE_i) dout_i                       (every pair)
+//   ds_ij     = exp(s_ij - LSE_i) (dout_i . v_j - dout_i . out_i)
+//   dq_i     += ds_ij k_hat_j / sqrt(d),  dk_hat_j += ds_ij q_i / sqrt(d)
+//                                          (pairs j != i, not masked)
+//   dqk_i     = dq_i + (dk_hat_i - k_hat_i (k_hat_i . dk_hat_i)) / ||qk_i||.
+// The self pair's score is the constant -1e5 (no gradient to qk), and a key
+// of zero norm has k_hat = 0 and passes no gradient through the key.
+//
+// CUDA cores, float32: one CTA per (b*h, round, chunk), one warp per query
+// (the forward's CUDA-core layout); dv, dq and dk_hat are accumulated with
+// float32 atomics, so the summation order (and the last bits) can change
+// from run to run.
+#include "common.cuh"
+#include "internal.h"
+
+namespace lsh {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kMaxD = 256;
+constexpr int kThreads = 256;
+
+// delta_i = dout_i . out_i; zero the accumulators.
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout, float* __restrict__ delta,
+                float* __restrict__ dqk, float* __restrict__ dv, float* __restrict__ dkh,
+                long long rows, int d) {
+  const int lane = threadIdx.x & 31;
+  const long long row = ((long long)blockIdx.x * kThreads + threadIdx.x) / 32;
+  if (row >= rows) return;
+  float acc = 0.f;
+  for (int e = lane; e < d; e += 32) {
+    const size_t k = (size_t)row * d + e;
+    acc = fmaf(to_f32(dout[k]), to_f32(out[k]), acc);
+    dqk[k] = 0.f;
+    dv[k] = 0.f;
+    dkh[k] = 0.f;
+  }
+  acc = warp_sum(acc);
+  if (lane == 0) delta[row] = acc;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
+                 const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
+                 const float* __restrict__ lse, const T* __restrict__ dout,
+                 const float* __restrict__ delta, float* __restrict__ dq, float* __restrict__ dv,
+                 float* __restrict__ dkh, int L, int d, int n_h, int c, int causal, float scale) {
+  extern __shared__ float sh[];  // [kWarps][2][d]: the query row and its dout
+  const int n_c = (L + c - 1) / c;
+  const int k = (int)(blockIdx.x % n_c);
+  const int r = (int)((blockIdx.x / n_c) % n_h);
+  const size_t bh = blockIdx.x / ((size_t)n_c * n_h);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* P = perm + (bh * n_h + r) * (size_t)L;
+  const T* X = qk + bh * (size_t)L * d;
+  const T* V = v + bh * (size_t)L * d;
+  const T* G = dout + bh * (size_t)L * d;
+  const float* IN = inv_norm + bh * (size_t)L;
+  float* DQ = dq + bh * (size_t)L * d;
+  float* DV = dv + bh * (size_t)L * d;
+  float* DK = dkh + bh * (size_t)L * d;
+  float* qs = sh + warp * 2 * d;
+  float* gs = qs + d;
+  const int k0 = k > 0 ? (k - 1) * c : 0, k1 = min((k + 1) * c, L);
+  constexpr int kPer = kMaxD / 32;
+
+  for (int qslot = k * c + warp; qslot < k1; qslot += kWarps) {
+    const int i = P[qslot];
+    for (int e = lane; e < d; e += 32) {
+      qs[e] = to_f32(X[(size_t)i * d + e]);
+      gs[e] = to_f32(G[(size_t)i * d + e]);
+    }
+    __syncwarp();
+    const float LSE = lse[bh * (size_t)L + i];
+    const float dl = delta[bh * (size_t)L + i];
+    float acc[kPer];  // dq_i, dimensions lane, lane + 32, ...
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) acc[t] = 0.f;
+
+    for (int t0 = k0; t0 < k1; t0 += 32) {
+      const int js = t0 + lane;
+      const bool in_window = js < k1;
+      const int j = in_window ? P[js] : 0;
+      const bool visible = in_window && !(causal && j > i);
+      float e_ij = 0.f, ds = 0.f, inj = 0.f;
+      if (visible) {
+        const T* xj = X + (size_t)j * d;
+        const T* vj = V + (size_t)j * d;
+        float dot = 0.f, gv = 0.f;
+        for (int e = 0; e < d; ++e) {
+          dot = fmaf(qs[e], to_f32(xj[e]), dot);
+          gv = fmaf(gs[e], to_f32(vj[e]), gv);
+        }
+        inj = IN[j];
+        const float s = (j == i) ? kSelfScore : dot * inj * scale;
+        e_ij = expf(s - LSE);
+        if (j != i) ds = e_ij * (gv - dl);
+        // dv_j += e_ij dout_i;  dk_hat_j += ds q_i / sqrt(d)
+        for (int e = 0; e < d; ++e) {
+          atomicAdd(&DV[(size_t)j * d + e], e_ij * gs[e]);
+          if (ds != 0.f && inj != 0.f) atomicAdd(&DK[(size_t)j * d + e], ds * scale * qs[e]);
+        }
+      }
+      // dq_i += ds k_hat_j / sqrt(d): broadcast each lane's pair
+      for (int src = 0; src < 32; ++src) {
+        const float dss = __shfl_sync(0xffffffffu, ds * inj * scale, src);
+        const int jj = __shfl_sync(0xffffffffu, j, src);
+        if (dss == 0.f) continue;
+        const T* xj = X + (size_t)jj * d;
+#pragma unroll
+        for (int t = 0; t < kPer; ++t) {
+          const int e = lane + 32 * t;
+          if (e < d) acc[t] = fmaf(dss, to_f32(xj[e]), acc[t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = lane + 32 * t;
+      if (e < d) atomicAdd(&DQ[(size_t)i * d + e], acc[t]);
+    }
+    __syncwarp();
+  }
+}
+
+// dqk_i += (dk_hat_i - k_hat_i (k_hat_i . dk_hat_i)) / ||qk_i||
+template <typename T>
+__global__ void __launch_bounds__(kThreads)
+bwd_finish_kernel(const T* __restrict__ qk, const float* __restrict__ inv_norm,
+                  const float* __restrict__ dkh, float* __restrict__ dqk, long long rows, int d) {
+  const int lane = threadIdx.x & 31;
+  const long long row = ((long long)blockIdx.x * kThreads + threadIdx.x) / 32;
+  if (row >= rows) return;
+  const float in = inv_norm[row];
+  if (in == 0.f) return;  // zero key: k_hat is the constant 0
+  float kd = 0.f;
+  for (int e = lane; e < d; e += 32) {
+    const size_t k = (size_t)row * d + e;
+    kd = fmaf(to_f32(qk[k]) * in, dkh[k], kd);
+  }
+  kd = warp_sum(kd);
+  for (int e = lane; e < d; e += 32) {
+    const size_t k = (size_t)row * d + e;
+    dqk[k] += (dkh[k] - to_f32(qk[k]) * in * kd) * in;
+  }
+}
+
+template <typename T>
+cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const float* inv_norm,
+                     const int32_t* perm, const void* out, const float* lse, const void* dout,
+                     float* dqk, float* dv, float* delta, float* dkh, cudaStream_t st) {
+  const long long rows = (long long)p.BH() * p.L;
+  const unsigned row_blocks = (unsigned)((rows * 32 + kThreads - 1) / kThreads);
+  bwd_prep_kernel<T><<<row_blocks, kThreads, 0, st>>>(
+      static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d);
+  const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
+  const size_t smem = (size_t)kWarps * 2 * p.d * sizeof(float);
+  bwd_pairs_kernel<T><<<grid, kWarps * 32, smem, st>>>(
+      static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
+      static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0,
+      1.0f / sqrtf((float)p.d));
+  bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm, dkh,
+                                                        dqk, rows, p.d);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(const Problem& p) {
+  const size_t rows = (size_t)p.BH() * p.L;
+  return ((rows * sizeof(float) + 255) & ~(size_t)255) + rows * p.d * sizeof(float);
+}
+
+cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
+                            const float* inv_norm, const int32_t* perm, const void* out,
+                            const float* lse, const void* dout, float* dqk, float* dv,
+                            void* workspace, cudaStream_t st) {
+  if (p.d > kMaxD) return cudaErrorInvalidValue;
+  const size_t rows = (size_t)p.BH() * p.L;
+  float* delta = static_cast<float*>(workspace);
+  float* dkh = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                        ((rows * sizeof(float) + 255) & ~(size_t)255));
+  return p.bf16 ? launch_t<__nv_bfloat16>(p, qk, v, inv_norm, perm, out, lse, dout, dqk, dv,
+                                          delta, dkh, st)
+                : launch_t<float>(p, qk, v, inv_norm, perm, out, lse, dout, dqk, dv, delta, dkh,
+                                  st);
+}
+
+}  // namespace lsh

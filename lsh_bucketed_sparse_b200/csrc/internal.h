@@ -44,6 +44,13 @@ Workspace workspace_layout(const Problem& p);
 lsh_status forward_body(const Problem& p, const void* qk, const void* v, const void* rot,
                         void* out, float* lse, void* ws, cudaStream_t st);
 
+// ---- backward (hash and sort held fixed) ------------------------------------
+size_t backward_workspace_bytes(const Problem& p);
+cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
+                            const float* inv_norm, const int32_t* perm, const void* out,
+                            const float* lse, const void* dout, float* dqk, float* dv,
+                            void* workspace, cudaStream_t st);
+
 // Address of the device word that kernels set when a bounded wait runs out.
 // Resolved for the current device (cudaGetSymbolAddress); nullptr on error.
 unsigned int* device_error_word();

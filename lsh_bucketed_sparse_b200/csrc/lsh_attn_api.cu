@@ -466,6 +466,42 @@ lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void* qk_host,
   return LSH_OK;
 }
 
+lsh_status lsh_attn_backward_workspace_size(const lsh_shape* shape, size_t* bytes) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (!bytes) return fail(LSH_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = backward_workspace_bytes(p);
+  return LSH_OK;
+}
+
+lsh_status lsh_attn_backward(const lsh_shape* shape, const void* qk, const void* v,
+                             const float* inv_norm, const int32_t* perm, const void* out,
+                             const float* lse, const void* dout, float* dqk, float* dv,
+                             void* workspace, size_t workspace_bytes, void* stream) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (p.dedup || p.bucket_mask)
+    return fail(LSH_ERR_UNSUPPORTED, "the backward pass has no variant flags");
+  CHECK(check_ptr(qk, "qk"));
+  CHECK(check_ptr(v, "v"));
+  CHECK(check_ptr(inv_norm, "inv_norm"));
+  CHECK(check_ptr(perm, "perm"));
+  CHECK(check_ptr(out, "out"));
+  CHECK(check_ptr(lse, "lse"));
+  CHECK(check_ptr(dout, "dout"));
+  CHECK(check_ptr(dqk, "dqk"));
+  CHECK(check_ptr(dv, "dv"));
+  CHECK(check_ptr(workspace, "workspace"));
+  if (reinterpret_cast<uintptr_t>(workspace) % 256)
+    return fail(LSH_ERR_INVALID_ARG, "workspace is not 256-byte aligned");
+  const size_t need = backward_workspace_bytes(p);
+  if (workspace_bytes < need)
+    return fail(LSH_ERR_WORKSPACE, "workspace of %zu bytes, need %zu", workspace_bytes, need);
+  cudaError_t e = launch_backward(p, qk, v, inv_norm, perm, out, lse, dout, dqk, dv, workspace,
+                                  static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "backward launch");
+}
+
 const char* lsh_attn_status_string(lsh_status status) {
   switch (status) {
     case LSH_OK: return "ok";

@@ -146,6 +146,15 @@ def make_centroids(wl: Workload, seed: Optional[int] = None):
     return c.to(wl.dtype).contiguous()
 
 
+def make_upstream(wl: Workload, seed: Optional[int] = None):
+    """An upstream gradient dout [batch, heads, seq_len, d_k] for the backward
+    pass: float32 N(0, 1) from its own generator (seed + 20000), cast to
+    ``wl.dtype``."""
+    gen = torch.Generator().manual_seed((wl.seed if seed is None else seed) + 20000)
+    g = torch.randn(wl.batch, wl.heads, wl.seq_len, wl.d_k, generator=gen, dtype=torch.float32)
+    return g.to(wl.dtype).contiguous()
+
+
 def small(name="tiny", batch=1, heads=2, seq_len=256, d_k=64, n_hashes=2, n_buckets=16,
           chunk_len=64, causal=True, dtype=torch.bfloat16, seed=7, clustered=False,
           n_clusters=16) -> Workload:

@@ -511,3 +511,47 @@ def test_kmeans_breaks_exact_ties_by_lowest_index(n_buckets):
             assert ok[clear].all(), np.nonzero(~ok & clear)[0][:10]
             checked += int(clear.sum())
     assert checked > 0.9 * wl.heads * wl.n_hashes * wl.seq_len
+
+
+# ---------------------------------------------------------------------------
+# Backward with the hash and sort held fixed (the oracle differentiates its
+# float64 re-statement of the forward with autograd).
+BWD = [
+    W.small("bwd-f32-causal", heads=2, seq_len=256, n_hashes=2, n_buckets=8,
+            dtype=torch.float32),
+    W.small("bwd-bf16-noncausal-d128", heads=1, seq_len=256, d_k=128, n_hashes=3,
+            n_buckets=16, chunk_len=32, causal=False),
+    W.small("bwd-bf16-causal-short-chunk", heads=2, seq_len=300, n_hashes=2, n_buckets=16),
+]
+
+
+@pytest.mark.parametrize("wl", BWD, ids=[w.name for w in BWD])
+def test_backward_matches_oracle(wl):
+    qk, v, rot = W.make_inputs(wl)
+    g = W.make_upstream(wl)
+    qk_d, v_d, rot_d, g_d = qk.to(DEV), v.to(DEV), rot.to(DEV), g.to(DEV)
+    b, inv = lsh.lsh_attn_hash(qk_d, rot_d, wl.n_buckets, wl.n_hashes)
+    perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+    o_r, l_r = lsh.lsh_attn_chunked_fwd(qk_d, v_d, inv, perm, wl.chunk_len, wl.causal,
+                                        n_buckets=wl.n_buckets)
+    out, lse = lsh.lsh_attn_combine(o_r, l_r)
+    dqk, dv = lsh.lsh_attn_backward(qk_d, v_d, inv, perm, out, lse, g_d, wl.chunk_len,
+                                    wl.causal, n_buckets=wl.n_buckets)
+    lsh.lsh_attn_device_check()
+    odq, odv = O.backward_all(qk, v, perm.cpu().numpy(), wl.chunk_len, wl.causal, g)
+    # A row that saw only itself (lse near -1e5) weighs its own v with
+    # exp(-1e5 - LSE), and float32 holds LSE there only to |LSE| 2^-24 ~ 6e-3
+    # (the forward's lse carries the same rounding): those rows get 1e-2.
+    ref_lse = O.forward(qk, v, rot, wl.n_buckets, wl.chunk_len, wl.causal,
+                        buckets=b.cpu().numpy().astype(np.int64))["lse"]
+    tol = 2e-2 if wl.dtype == torch.bfloat16 else 1e-4
+    for name, gpu, ref in (("dqk", dqk, odq), ("dv", dv, odv)):
+        gg = gpu.cpu().numpy().astype(np.float64)
+        assert np.isfinite(gg).all(), name
+        for h in range(wl.heads):
+            scale = np.abs(ref[0, h]).max()
+            err = np.abs(gg[0, h] - ref[0, h]).max(axis=1) / scale
+            alone = ref_lse[0, h] < -1e4
+            assert err[~alone].max() <= tol, f"{name} head {h}: {err[~alone].max():.3e}"
+            if alone.any():
+                assert err[alone].max() <= max(tol, 1e-2), f"{name} head {h} (alone)"
