@@ -282,6 +282,58 @@ def run_reference(args, wl):
     return 0
 
 
+def run_backward(args, wl):
+    """Time lsh_attn_backward (gradients of out w.r.t. qk and v with the hash
+    and sort held fixed) on GPU 0; the forward stages run once beforehand."""
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream(dev)
+    qk_h, v_h, rot_h = W.make_inputs(wl)
+    qk, v = qk_h.to(dev), v_h.to(dev)
+    rot = rot_h.to(dev) if rot_h is not None else None
+    g = W.make_upstream(wl).to(dev)
+    b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+    perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+    o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                        n_buckets=wl.n_buckets)
+    out, lse = lsh.lsh_attn_combine(o_r, l_r)
+    del o_r, l_r
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype)
+    ws = torch.empty(lsh.lsh_attn_backward_workspace_size(shp), dtype=torch.uint8, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        return lsh.lsh_attn_backward(qk, v, inv, perm, out, lse, g, wl.chunk_len, wl.causal,
+                                     n_buckets=wl.n_buckets, workspace=ws)
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        step()
+    ms = 0.0
+    with ClockSampler(0) as clocks:
+        clocks.start()
+        for k in range(args.steps):
+            flush.fill_(float(k))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
+        clocks.stop()
+    lsh.lsh_attn_device_check()
+    ms_per_step = ms / args.steps
+    print(json.dumps({
+        "metric": METRIC, "value": wl.tokens / (ms_per_step / 1e3), "unit": UNIT, "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f32 (gradients)", "data": "synthetic",
+        "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
+                       variant="backward: d qk, d v of out with the hash and sort held fixed "
+                               "(CUDA cores, float32 atomics)"),
+        "clocks": clocks.summary(), "gpu_launches": 3 * args.steps}), flush=True)
+    return 0
+
+
 def run_one_stage(args, wl):
     """Time one stage of the pass by itself on GPU 0 (inputs prepared by the
     earlier stages outside the timed loop).  Used to profile a single kernel."""
@@ -349,6 +401,9 @@ def main(argv=None):
     ap.add_argument("--kmeans", action="store_true",
                     help="routing-style assignment to n_buckets centroids (CUDA-core hash) "
                          "instead of the random-rotation hash; a separate measurement")
+    ap.add_argument("--backward", action="store_true",
+                    help="time the backward pass (hash and sort fixed) on the workload; a "
+                         "separate measurement, not the headline")
     ap.add_argument("--only-stage", choices=["hash", "sort", "chunked_attention", "combine"],
                     help="time one stage call alone (for profiling); prints its own JSON line")
     args = ap.parse_args(argv)
@@ -357,6 +412,8 @@ def main(argv=None):
         return run_reference(args, wl)
     if args.only_stage:
         return run_one_stage(args, wl)
+    if args.backward:
+        return run_backward(args, wl)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 

@@ -16,7 +16,9 @@
 // CUDA cores, float32: one CTA per (b*h, round, chunk), one warp per query
 // (the forward's CUDA-core layout); dv, dq and dk_hat are accumulated with
 // float32 atomics, so the summation order (and the last bits) can change
-// from run to run.
+// from run to run.  When the window's dv and dk_hat rows fit in shared
+// memory (SACC), the CTA sums its queries' contributions there and adds each
+// window row to global memory once.
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,6 +28,7 @@ namespace {
 constexpr int kWarps = 8;
 constexpr int kMaxD = 256;
 constexpr int kThreads = 256;
+constexpr size_t kSaccLimit = 200 * 1024;  // shared memory for the window sums
 
 // delta_i = dout_i . out_i; zero the accumulators.
 template <typename T>
@@ -48,14 +51,16 @@ bwd_prep_kernel(const T* __restrict__ out, const T* __restrict__ dout, float* __
   if (lane == 0) delta[row] = acc;
 }
 
-template <typename T>
+template <typename T, bool SACC>
 __global__ void __launch_bounds__(kWarps * 32)
 bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                  const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
                  const float* __restrict__ lse, const T* __restrict__ dout,
                  const float* __restrict__ delta, float* __restrict__ dq, float* __restrict__ dv,
                  float* __restrict__ dkh, int L, int d, int n_h, int c, int causal, float scale) {
-  extern __shared__ float sh[];  // [kWarps][2][d]: the query row and its dout
+  // [kWarps][2][d]: the query row and its dout; with SACC then dv and dk_hat
+  // of the window's rows, [2c][d] each
+  extern __shared__ float sh[];
   const int n_c = (L + c - 1) / c;
   const int k = (int)(blockIdx.x % n_c);
   const int r = (int)((blockIdx.x / n_c) % n_h);
@@ -73,6 +78,15 @@ bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   float* gs = qs + d;
   const int k0 = k > 0 ? (k - 1) * c : 0, k1 = min((k + 1) * c, L);
   constexpr int kPer = kMaxD / 32;
+  float* dv_s = sh + kWarps * 2 * d;       // SACC only
+  float* dk_s = dv_s + (size_t)2 * c * d;
+  if (SACC) {
+    for (int t = threadIdx.x; t < (k1 - k0) * d; t += blockDim.x) {
+      dv_s[t] = 0.f;
+      dk_s[t] = 0.f;
+    }
+    __syncthreads();
+  }
 
   for (int qslot = k * c + warp; qslot < k1; qslot += kWarps) {
     const int i = P[qslot];
@@ -106,9 +120,11 @@ bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
         e_ij = expf(s - LSE);
         if (j != i) ds = e_ij * (gv - dl);
         // dv_j += e_ij dout_i;  dk_hat_j += ds q_i / sqrt(d)
+        float* dvj = SACC ? dv_s + (size_t)(js - k0) * d : DV + (size_t)j * d;
+        float* dkj = SACC ? dk_s + (size_t)(js - k0) * d : DK + (size_t)j * d;
         for (int e = 0; e < d; ++e) {
-          atomicAdd(&DV[(size_t)j * d + e], e_ij * gs[e]);
-          if (ds != 0.f && inj != 0.f) atomicAdd(&DK[(size_t)j * d + e], ds * scale * qs[e]);
+          atomicAdd(&dvj[e], e_ij * gs[e]);
+          if (ds != 0.f && inj != 0.f) atomicAdd(&dkj[e], ds * scale * qs[e]);
         }
       }
       // dq_i += ds k_hat_j / sqrt(d): broadcast each lane's pair
@@ -130,6 +146,14 @@ bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
       if (e < d) atomicAdd(&DQ[(size_t)i * d + e], acc[t]);
     }
     __syncwarp();
+  }
+  if (SACC) {
+    __syncthreads();
+    for (int t = threadIdx.x; t < (k1 - k0) * d; t += blockDim.x) {
+      const int j = P[k0 + t / d], e = t % d;
+      atomicAdd(&DV[(size_t)j * d + e], dv_s[t]);
+      if (dk_s[t] != 0.f) atomicAdd(&DK[(size_t)j * d + e], dk_s[t]);
+    }
   }
 }
 
@@ -164,8 +188,17 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
   bwd_prep_kernel<T><<<row_blocks, kThreads, 0, st>>>(
       static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d);
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
-  const size_t smem = (size_t)kWarps * 2 * p.d * sizeof(float);
-  bwd_pairs_kernel<T><<<grid, kWarps * 32, smem, st>>>(
+  const size_t base = (size_t)kWarps * 2 * p.d * sizeof(float);
+  const size_t acc = (size_t)2 * (2 * (size_t)p.c) * p.d * sizeof(float);
+  const bool sacc = base + acc <= kSaccLimit;
+  const size_t smem = sacc ? base + acc : base;
+  auto kernel = sacc ? bwd_pairs_kernel<T, true> : bwd_pairs_kernel<T, false>;
+  if (smem > 48 * 1024) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  kernel<<<grid, kWarps * 32, smem, st>>>(
       static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
       static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0,
       1.0f / sqrtf((float)p.d));
