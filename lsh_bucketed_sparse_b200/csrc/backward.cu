@@ -157,6 +157,118 @@ bwd_pairs_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   }
 }
 
+// The same pairs with the window staged: the chunk's window keys (already
+// normalised) and values are copied once into padded shared-memory rows
+// (d + 1 floats, so lanes reading different rows hit different banks) and
+// every query warp of the chunk reads them there; the window's dv and dk_hat
+// sums stay in shared memory as in SACC.
+template <typename T>
+__global__ void __launch_bounds__(kWarps * 32)
+bwd_pairs_staged_kernel(const T* __restrict__ qk, const T* __restrict__ v,
+                        const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
+                        const float* __restrict__ lse, const T* __restrict__ dout,
+                        const float* __restrict__ delta, float* __restrict__ dq,
+                        float* __restrict__ dv, float* __restrict__ dkh, int L, int d, int n_h,
+                        int c, int causal, float scale) {
+  extern __shared__ float sh[];
+  const int n_c = (L + c - 1) / c;
+  const int k = (int)(blockIdx.x % n_c);
+  const int r = (int)((blockIdx.x / n_c) % n_h);
+  const size_t bh = blockIdx.x / ((size_t)n_c * n_h);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int32_t* P = perm + (bh * n_h + r) * (size_t)L;
+  const T* X = qk + bh * (size_t)L * d;
+  const T* V = v + bh * (size_t)L * d;
+  const T* G = dout + bh * (size_t)L * d;
+  const float* IN = inv_norm + bh * (size_t)L;
+  float* DQ = dq + bh * (size_t)L * d;
+  float* DV = dv + bh * (size_t)L * d;
+  float* DK = dkh + bh * (size_t)L * d;
+  const int k0 = k > 0 ? (k - 1) * c : 0, k1 = min((k + 1) * c, L), nw = k1 - k0;
+  const int dp = d + 1;                      // padded row
+  float* qs = sh + warp * 2 * d;
+  float* gs = qs + d;
+  float* ks = sh + kWarps * 2 * d;           // [2c][dp] normalised keys
+  float* vs = ks + (size_t)2 * c * dp;       // [2c][dp] values
+  float* dv_s = vs + (size_t)2 * c * dp;     // [2c][dp]
+  float* dk_s = dv_s + (size_t)2 * c * dp;   // [2c][dp]
+  int* pos_w = reinterpret_cast<int*>(dk_s + (size_t)2 * c * dp);  // [2c]
+  for (int t = threadIdx.x; t < nw * d; t += blockDim.x) {
+    const int w = t / d, e = t % d;
+    const int j = P[k0 + w];
+    ks[w * dp + e] = to_f32(X[(size_t)j * d + e]) * IN[j];
+    vs[w * dp + e] = to_f32(V[(size_t)j * d + e]);
+    dv_s[w * dp + e] = 0.f;
+    dk_s[w * dp + e] = 0.f;
+    if (e == 0) pos_w[w] = j;
+  }
+  __syncthreads();
+  constexpr int kPer = kMaxD / 32;
+
+  for (int qslot = k * c + warp; qslot < k1; qslot += kWarps) {
+    const int i = P[qslot];
+    for (int e = lane; e < d; e += 32) {
+      qs[e] = to_f32(X[(size_t)i * d + e]);
+      gs[e] = to_f32(G[(size_t)i * d + e]);
+    }
+    __syncwarp();
+    const float LSE = lse[bh * (size_t)L + i];
+    const float dl = delta[bh * (size_t)L + i];
+    float acc[kPer];
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) acc[t] = 0.f;
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+      const int w = w0 + lane;
+      const bool in_window = w < nw;
+      const int j = in_window ? pos_w[w] : 0;
+      const bool visible = in_window && !(causal && j > i);
+      float e_ij = 0.f, ds = 0.f;
+      if (visible) {
+        const float* kr = ks + w * dp;
+        const float* vr = vs + w * dp;
+        float dot = 0.f, gv = 0.f;
+        for (int e = 0; e < d; ++e) {
+          dot = fmaf(qs[e], kr[e], dot);
+          gv = fmaf(gs[e], vr[e], gv);
+        }
+        const float s = (j == i) ? kSelfScore : dot * scale;
+        e_ij = expf(s - LSE);
+        if (j != i) ds = e_ij * (gv - dl);
+        float* dvr = dv_s + w * dp;
+        float* dkr = dk_s + w * dp;
+        for (int e = 0; e < d; ++e) {
+          atomicAdd(&dvr[e], e_ij * gs[e]);
+          if (ds != 0.f) atomicAdd(&dkr[e], ds * scale * qs[e]);
+        }
+      }
+      for (int src = 0; src < 32; ++src) {
+        const float dss = __shfl_sync(0xffffffffu, ds * scale, src);
+        if (dss == 0.f) continue;
+        const float* kr = ks + (w0 + src) * dp;
+#pragma unroll
+        for (int t = 0; t < kPer; ++t) {
+          const int e = lane + 32 * t;
+          if (e < d) acc[t] = fmaf(dss, kr[e], acc[t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < kPer; ++t) {
+      const int e = lane + 32 * t;
+      if (e < d) atomicAdd(&DQ[(size_t)i * d + e], acc[t]);
+    }
+    __syncwarp();
+  }
+  __syncthreads();
+  for (int t = threadIdx.x; t < nw * d; t += blockDim.x) {
+    const int w = t / d, e = t % d;
+    const int j = pos_w[w];
+    atomicAdd(&DV[(size_t)j * d + e], dv_s[w * dp + e]);
+    const float x = dk_s[w * dp + e];
+    if (x != 0.f && IN[j] != 0.f) atomicAdd(&DK[(size_t)j * d + e], x);
+  }
+}
+
 // dqk_i += (dk_hat_i - k_hat_i (k_hat_i . dk_hat_i)) / ||qk_i||
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -189,6 +301,21 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
       static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d);
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
   const size_t base = (size_t)kWarps * 2 * p.d * sizeof(float);
+  const size_t staged = base + (size_t)4 * 2 * p.c * (p.d + 1) * sizeof(float) +
+                        (size_t)2 * p.c * sizeof(int);
+  if (staged <= kSaccLimit) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_pairs_staged_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)staged);
+    if (e != cudaSuccess) return e;
+    bwd_pairs_staged_kernel<T><<<grid, kWarps * 32, staged, st>>>(
+        static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
+        static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.d, p.n_h, p.c,
+        p.causal ? 1 : 0, 1.0f / sqrtf((float)p.d));
+    bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm,
+                                                          dkh, dqk, rows, p.d);
+    return cudaGetLastError();
+  }
   const size_t acc = (size_t)2 * (2 * (size_t)p.c) * p.d * sizeof(float);
   const bool sacc = base + acc <= kSaccLimit;
   const size_t smem = sacc ? base + acc : base;
