@@ -62,6 +62,7 @@ constexpr int kVWarp = 2 + kSoftWarps;
 constexpr int kThreads = (3 + kSoftWarps) * 32;   // qk producer, MMA, softmax, v producer
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMetaSlots = 8;
+constexpr int kMaxRounds = 8;  // rounds the duplicate correction carries per row
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 // A row whose sum of 2^(s' - ref) falls below this is redone with its exact max.
@@ -84,6 +85,7 @@ struct Params {
   __nv_bfloat16* o_rounds;
   float* lse_rounds;
   const int16_t* buckets;  // [BH, n_h, L] bucket ids for the bucket-equality mask, else null
+  const int32_t* undo;     // [BH, n_h, L] every round's undo for the duplicate correction
   unsigned int* err;
   int L, n_h, causal;
   int steps;          // ceil(L / 128) per segment
@@ -94,7 +96,7 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, p, pos, ksc, qref, bkt, xch, bars, misc, total;
+  uint32_t qk, v, p, pos, ksc, qref, bkt, chk, xch, bars, misc, total;
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
@@ -102,7 +104,7 @@ __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
   return 2 * nq + 2 * nv + 2 * kMetaSlots + 12 + 8 + 4 + 1;
 }
 
-template <int C, int D, bool BM = false>
+template <int C, int D, bool BM = false, bool DD = false>
 __host__ __device__ constexpr Layout layout(int nq, int nv, int np) {
   using K = Cfg<C, D>;
   Layout l{};
@@ -114,6 +116,8 @@ __host__ __device__ constexpr Layout layout(int nq, int nv, int np) {
   l.ksc = off;  off += kMetaSlots * kQ * 4;
   l.qref = off; off += kMetaSlots * kQ * 4;
   l.bkt = off;  off += BM ? kMetaSlots * kQ * 4 : 0;  // bucket ids (bucket-equality mask)
+  // every round's chunk index per row (duplicate correction)
+  l.chk = off;  off += DD ? kMetaSlots * kQ * kMaxRounds * 4 : 0;
   l.xch = off;  off += (2 * 2 + 2 + 2) * kQ * 4;   // partial sums [2][2], maxima [2], redo sums [2]
   l.bars = off; off += n_barriers(nq, nv) * 8;
   l.misc = off; off += 16;
@@ -241,27 +245,47 @@ struct Plan {
   bool ok;
 };
 
-template <int C, int D, bool BM = false>
+template <int C, int D, bool BM = false, bool DD = false>
 __host__ __device__ constexpr Plan make_plan() {
   constexpr uint32_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
   for (int pb = 2; pb >= 1; --pb) {
-    const uint32_t fixed = layout<C, D, BM>(0, 0, pb).total + n_barriers(6, 6) * 8;
+    const uint32_t fixed = layout<C, D, BM, DD>(0, 0, pb).total + n_barriers(6, 6) * 8;
     if (fixed >= limit) continue;
     const int tiles = (int)((limit - fixed) / Cfg<C, D>::kTile);
     if (tiles < 4 || (pb == 2 && tiles < 6)) continue;
     const int q = (tiles + 1) / 2 < 5 ? (tiles + 1) / 2 : 5;
     const int v = tiles - q < 5 ? tiles - q : 5;
-    uint32_t smem = layout<C, D, BM>(q, v, pb).total + 1024;
+    uint32_t smem = layout<C, D, BM, DD>(q, v, pb).total + 1024;
     if (smem < 116 * 1024) smem = 116 * 1024;
     return Plan{q, v, pb, smem, smem <= (uint32_t)kSmemLimit};
   }
   return Plan{0, 0, 0, 0, false};
 }
 
+// log2 of the number of rounds in which a key (its chunk index of every
+// round at `ck`) lies in the window of a query (chunk indices `cq`): rounds
+// where the query's chunk minus the key's is 0 or 1.
+__device__ __forceinline__ float dup_log2(const int* ck, const int (&cq)[kMaxRounds], int n_h) {
+  const int4 a = *reinterpret_cast<const int4*>(ck);
+  const int4 b = *reinterpret_cast<const int4*>(ck + 4);
+  const int k8[kMaxRounds] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+  int n = 0;
+#pragma unroll
+  for (int rr = 0; rr < kMaxRounds; ++rr)
+    n += (rr < n_h && (unsigned)(cq[rr] - k8[rr]) <= 1u) ? 1 : 0;
+  float l;
+  asm("lg2.approx.f32 %0, %1;" : "=f"(l) : "f"((float)max(n, 1)));
+  return l;
+}
+
 // BMASK: the bucket-equality mask variant (section 2 "LSH attention": a
 // query attends only to targets in its own hash bucket): a key whose bucket
 // in this round differs from the query's is not visible.
-template <int C, int D, bool CAUSAL, bool BMASK>
+// DEDUP: the duplicate-count correction (Appendix A "Duplicate handling"):
+// a visible key's exponent loses log2 N_ij, N_ij = the rounds r' (at most
+// kMaxRounds) with chunk_r'(i) - chunk_r'(j) in {0, 1}; each row carries its
+// chunk index of every round in the metadata ring.
+template <int C, int D, bool CAUSAL, bool BMASK, bool DEDUP>
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
                const Params p) {
@@ -269,9 +293,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  constexpr Plan PL = make_plan<C, D, BMASK>();
+  constexpr Plan PL = make_plan<C, D, BMASK, DEDUP>();
   constexpr int NQ = PL.nq, NV = PL.nv, NP = PL.np, NM = kMetaSlots;
-  constexpr Layout Ly = layout<C, D, BMASK>(NQ, NV, NP);
+  constexpr Layout Ly = layout<C, D, BMASK, DEDUP>(NQ, NV, NP);
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
   uint8_t* p_s = smem + Ly.p;
@@ -279,6 +303,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   float* ksc_s = reinterpret_cast<float*>(smem + Ly.ksc);
   float* qref_s = reinterpret_cast<float*>(smem + Ly.qref);
   int* bkt_s = reinterpret_cast<int*>(smem + Ly.bkt);
+  int* chk_s = reinterpret_cast<int*>(smem + Ly.chk);  // [NM * kQ][kMaxRounds]
   float* xl = reinterpret_cast<float*>(smem + Ly.xch);  // [2 buf][2 half][kQ]
   float* xm = xl + 4 * kQ;                              // [2 half][kQ]
   float* xl2 = xm + 2 * kQ;                             // [2 half][kQ]
@@ -399,6 +424,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         ksc_s[row] = in0[k] * p.ksc;
         qref_s[row] = in0[k] > 0.f ? p.ksc / in0[k] : 0.f;
         if (BMASK) bkt_s[row] = bk0[k];
+        if (DEDUP) {
+          const size_t ub = (size_t)c0.U.bh * p.n_h * p.L;
+#pragma unroll
+          for (int rr = 0; rr < kMaxRounds; ++rr)
+            chk_s[row * kMaxRounds + rr] =
+                (rr < p.n_h && pos0[k] != INT_MAX) ? p.undo[ub + (size_t)rr * p.L + pos0[k]] / C
+                                                   : -2;
+        }
       }
       mbar_arrive(&m_full[ms]);
 #pragma unroll
@@ -576,6 +609,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
       const int qb = BMASK ? bkt_s[cs * kQ + m] : 0;
+      int cq[kMaxRounds];
+#pragma unroll
+      for (int rr = 0; rr < kMaxRounds; ++rr)
+        cq[rr] = DEDUP ? chk_s[(cs * kQ + m) * kMaxRounds + rr] : 0;
+      // log2 N for the key in metadata row kr (0 without the correction)
+#define DUP_LOG2(kr) (DEDUP ? dup_log2(chk_s + (kr) * kMaxRounds, cq, p.n_h) : 0.f)
       const int qlim = p.causal ? qpos : INT_MAX - 1;
       const int lo = has_prev ? win_lo : max(win_lo, C);
       // metadata row of key column j0 (a multiple of 32, all in one block)
@@ -618,7 +657,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
               }
               if (BMASK) valid = valid && kba[h] == qb;
               if (!CAUSAL || BMASK) any |= valid;
-              const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
+              float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
+              if (DEDUP && valid) x -= DUP_LOG2(kb + e + h);
               pr[h] = valid ? ex2(x) : 0.f;
               la[h] += pr[h];
             }
@@ -664,7 +704,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           for (int e = 0; e < 32; ++e) {
             const int kp = pos_s[kb + e];
             if (kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e] == qb))
-              mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
+              mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e] - DUP_LOG2(kb + e));
           }
         }
         xm[half * kQ + m] = mx;
@@ -693,7 +733,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
                 const bool valid =
                     kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e + h + g] == qb);
                 pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + h + g]), ksc_s[kb + e + h + g],
-                                         -gmax))
+                                         -gmax) - DUP_LOG2(kb + e + h + g))
                               : 0.f;
                 l2 += pr[g];
               }
@@ -813,13 +853,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 
 template <int C, int D>
 cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const float* inv_norm,
-                      const int32_t* perm, const int16_t* buckets, void* o_rounds,
-                      float* lse_rounds, cudaStream_t st) {
-  constexpr Plan PL = make_plan<C, D, false>();
-  constexpr Plan PLM = make_plan<C, D, true>();
+                      const int32_t* perm, const int16_t* buckets, const int32_t* undo,
+                      void* o_rounds, float* lse_rounds, cudaStream_t st) {
+  constexpr Plan PL = make_plan<C, D, false, false>();
+  constexpr Plan PLM = make_plan<C, D, true, false>();
+  constexpr Plan PLD = make_plan<C, D, false, true>();
   static_assert(PL.ok && PLM.ok, "no shared-memory plan for this (chunk, d)");
+  // the duplicate correction's chunk indices do not fit next to the rings
+  // for every (chunk, d): those take the CUDA-core kernel
+  if (undo && !PLD.ok) return cudaErrorNotSupported;
   Params p;
-  const size_t smem = buckets ? PLM.smem : PL.smem;
+  const size_t smem = undo ? PLD.smem : (buckets ? PLM.smem : PL.smem);
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;
   p.v = static_cast<const __nv_bfloat16*>(v);
@@ -828,6 +872,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   p.o_rounds = static_cast<__nv_bfloat16*>(o_rounds);
   p.lse_rounds = lse_rounds;
   p.buckets = buckets;
+  p.undo = undo;
   p.err = err;
   p.L = pr.L;
   p.n_h = pr.n_h;
@@ -860,11 +905,17 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const bool bmask = buckets != nullptr;
-  auto kernel = pr.causal ? (bmask ? attn_tc_kernel<C, D, true, true>
-                                   : attn_tc_kernel<C, D, true, false>)
-                          : (bmask ? attn_tc_kernel<C, D, false, true>
-                                   : attn_tc_kernel<C, D, false, false>);
+  const bool bmask = buckets != nullptr, dedup = undo != nullptr;
+  // (with no plan for the correction, its instantiations are never launched:
+  // they fall back to the plain kernel's symbol and are excluded above)
+  constexpr bool kDD = PLD.ok;
+  auto kernel =
+      pr.causal ? (dedup ? attn_tc_kernel<C, D, true, false, kDD>
+                         : (bmask ? attn_tc_kernel<C, D, true, true, false>
+                                  : attn_tc_kernel<C, D, true, false, false>))
+                : (dedup ? attn_tc_kernel<C, D, false, false, kDD>
+                         : (bmask ? attn_tc_kernel<C, D, false, true, false>
+                                  : attn_tc_kernel<C, D, false, false, false>));
   cudaError_t e = cudaFuncSetAttribute(kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -882,17 +933,21 @@ bool attn_tc_supported(const Problem& p) {
 }
 
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
-                           const int32_t* perm, const int16_t* buckets, void* o_rounds,
-                           float* lse_rounds, cudaStream_t st) {
+                           const int32_t* perm, const int16_t* buckets, const int32_t* undo,
+                           void* o_rounds, float* lse_rounds, cudaStream_t st) {
   if (!p.bucket_mask) buckets = nullptr;
+  if (!p.dedup) undo = nullptr;
+  if (buckets && undo) return cudaErrorNotSupported;  // both at once: CUDA-core kernel
+  if (undo && p.n_h > kMaxRounds) return cudaErrorNotSupported;
   if (p.c == 64 && p.d == 64)
-    return launch_cd<64, 64>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
+    return launch_cd<64, 64>(p, qk, v, inv_norm, perm, buckets, undo, o_rounds, lse_rounds, st);
   if (p.c == 64 && p.d == 128)
-    return launch_cd<64, 128>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
+    return launch_cd<64, 128>(p, qk, v, inv_norm, perm, buckets, undo, o_rounds, lse_rounds, st);
   if (p.c == 128 && p.d == 64)
-    return launch_cd<128, 64>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
+    return launch_cd<128, 64>(p, qk, v, inv_norm, perm, buckets, undo, o_rounds, lse_rounds, st);
   if (p.c == 128 && p.d == 128)
-    return launch_cd<128, 128>(p, qk, v, inv_norm, perm, buckets, o_rounds, lse_rounds, st);
+    return launch_cd<128, 128>(p, qk, v, inv_norm, perm, buckets, undo, o_rounds, lse_rounds,
+                               st);
   return cudaErrorNotSupported;
 }
 

@@ -77,8 +77,8 @@ cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v
                                  float* lse_rounds, cudaStream_t st);
 bool attn_tc_supported(const Problem& p);
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
-                           const int32_t* perm, const int16_t* buckets, void* o_rounds,
-                           float* lse_rounds, cudaStream_t st);
+                           const int32_t* perm, const int16_t* buckets, const int32_t* undo,
+                           void* o_rounds, float* lse_rounds, cudaStream_t st);
 
 // ---- stage 4: combine ------------------------------------------------------
 cudaError_t launch_combine(const Problem& p, const void* o_rounds, const float* lse_rounds,

@@ -119,15 +119,18 @@ lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort launch");
 }
 
-// The duplicate-count correction runs on the CUDA-core kernel only; the
-// bucket-equality mask on both.
+// The variants run on the tensor-core kernel where it takes them (the
+// duplicate correction for n_h <= 8, not together with the bucket mask),
+// else on the CUDA-core kernel.
 lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                     const int32_t* perm, const int32_t* undo, const int16_t* buckets,
                     void* o_r, float* lse_r, cudaStream_t st) {
-  cudaError_t e =
-      (!p.portable && !p.dedup && attn_tc_supported(p))
-          ? launch_attn_tc(p, qk, v, inv_norm, perm, buckets, o_r, lse_r, st)
-          : launch_attn_portable(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st);
+  const bool tc = !p.portable && attn_tc_supported(p) &&
+                  !(p.dedup && (p.bucket_mask || p.n_h > 8));
+  cudaError_t e = tc ? launch_attn_tc(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st)
+                     : cudaErrorNotSupported;
+  if (e == cudaErrorNotSupported)  // a shape the tensor-core kernel does not plan for
+    e = launch_attn_portable(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
 }
 

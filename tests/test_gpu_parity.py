@@ -337,6 +337,13 @@ DEDUP = [
             n_buckets=4, chunk_len=32, causal=False),
     W.small("dedup-f32-causal", heads=1, seq_len=256, n_hashes=3, n_buckets=8,
             dtype=torch.float32),
+    # the tensor-core attention's correction: (c, d) = (128, 64), and (64, 128)
+    # non-causal with a short last chunk; more than 8 rounds fall back
+    W.small("dedup-tc-c128-d64", heads=2, seq_len=1024, n_hashes=4, n_buckets=8,
+            chunk_len=128),
+    W.small("dedup-tc-c64-d128-noncausal", heads=2, seq_len=1000, d_k=128, n_hashes=3,
+            n_buckets=8, causal=False),
+    W.small("dedup-nine-rounds", heads=1, seq_len=512, n_hashes=9, n_buckets=8),
 ]
 
 
