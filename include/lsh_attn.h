@@ -55,7 +55,7 @@ extern "C" {
 typedef enum lsh_status {
   LSH_OK = 0,
   LSH_ERR_INVALID_ARG = 1,     /* null/misaligned pointer, bad size or flag */
-  LSH_ERR_UNSUPPORTED = 2,     /* valid request this build cannot serve    */
+  LSH_ERR_UNSUPPORTED = 2,     /* valid request this library cannot serve  */
   LSH_ERR_WORKSPACE = 3,       /* workspace or staging buffer too small     */
   LSH_ERR_CUDA = 4,            /* a CUDA launch or copy failed              */
   LSH_ERR_DEVICE_TIMEOUT = 5   /* a kernel's bounded wait ran out           */

@@ -1,6 +1,6 @@
 // Backward of the forward pass with the hash and the sort held fixed (the
-// hash is piecewise constant, so no gradient flows through bucket ids; the
-// survey's "next" row f3).  "Reformer: The Efficient Transformer", section 2
+// hash is piecewise constant, so no gradient flows through bucket ids).
+// "Reformer: The Efficient Transformer", section 2
 // "LSH attention" and Appendix A define the forward; its gradient follows
 // from the multiset form of the combined output,
 //   out_i = sum_r sum_{j in W_r(i)} exp(s_ij - LSE_i) v_j,

@@ -339,7 +339,7 @@ def token_rounds(x, v, perm, undo, chunk_len, causal, i):
 
 
 # ---------------------------------------------------------------------------
-# 6. Backward (the survey's "next" row f3; no gradient through hash or sort)
+# 6. Backward (hash and sort held fixed: no gradient through bucket ids)
 # ---------------------------------------------------------------------------
 def backward_head(x, v, perm, chunk_len: int, causal: bool, dout):
     """Gradients of out w.r.t. the shared qk and v of one (batch, head), with
