@@ -244,7 +244,10 @@ LSH_ATTN_API lsh_status lsh_attn_backward(const lsh_shape* shape, const void* qk
  * waits for all of it, so the caller synchronises `stream` before reading
  * out_host / lse_host.  Calls on one device enqueue one at a time (a mutex
  * guards the shared streams).  Host buffers should be page-locked for the
- * copies to overlap.
+ * copies to overlap.  On an error after the first copy was queued, `stream`
+ * still waits for everything already queued (which reads and writes the
+ * caller's buffers), so synchronise it before freeing them; out_host and
+ * lse_host are then undefined.
  *   device_buffer: caller-owned device memory of at least
  *   lsh_attn_forward_host_device_bytes() bytes, 256-byte aligned; it holds the
  *   device copies of the inputs and outputs plus the workspace.

@@ -252,6 +252,62 @@ cudaMemPool_t scratch_pool(int dev) {
   return g_pool[dev];
 }
 
+// Queues every group's copy-in, forward pass and copy-out on the pipe's
+// streams (host_pipe's comment gives the overlap).
+lsh_status host_groups(const Problem& p, const HostStaging& h, HostPipe* hp, int G,
+                       size_t row_in, size_t row_lse, const void* qk_host, const void* v_host,
+                       const void* rotations_host, void* out_host, float* lse_host, char* base) {
+  cudaError_t e;
+  if (h.rot_bytes &&
+      (e = cudaMemcpyAsync(base + h.rot, rotations_host, h.rot_bytes, cudaMemcpyHostToDevice,
+                           hp->in)))
+    return cuda_fail(e, "copy rotations to device");
+  const int BH = p.BH();
+  for (int g = 0; g < G; ++g) {
+    const int b0 = (int)((long long)BH * g / G), b1 = (int)((long long)BH * (g + 1) / G);
+    const size_t in_off = (size_t)b0 * row_in, in_len = (size_t)(b1 - b0) * row_in;
+    const size_t l_off = (size_t)b0 * row_lse, l_len = (size_t)(b1 - b0) * row_lse;
+    // one cudaMemcpyAsync per tensor slice
+    if ((e = cudaMemcpyAsync(base + h.qk + in_off, static_cast<const char*>(qk_host) + in_off,
+                             in_len, cudaMemcpyHostToDevice, hp->in)))
+      return cuda_fail(e, "copy qk to device");
+    if ((e = cudaMemcpyAsync(base + h.v + in_off, static_cast<const char*>(v_host) + in_off,
+                             in_len, cudaMemcpyHostToDevice, hp->in)))
+      return cuda_fail(e, "copy v to device");
+    if ((e = cudaEventRecord(hp->in_done[g], hp->in))) return cuda_fail(e, "record copy-in");
+    if ((e = cudaStreamWaitEvent(hp->comp, hp->in_done[g], 0))) return cuda_fail(e, "wait copy-in");
+    Problem pg = p;
+    pg.B = 1;
+    pg.H = b1 - b0;
+    CHECK(forward_body(pg, base + h.qk + in_off, base + h.v + in_off,
+                       h.rot_bytes ? base + h.rot : nullptr, base + h.out + in_off,
+                       reinterpret_cast<float*>(base + h.lse + l_off), base + h.ws, hp->comp));
+    if ((e = cudaEventRecord(hp->comp_done[g], hp->comp))) return cuda_fail(e, "record compute");
+    if ((e = cudaStreamWaitEvent(hp->out, hp->comp_done[g], 0))) return cuda_fail(e, "wait compute");
+    if ((e = cudaMemcpyAsync(static_cast<char*>(out_host) + in_off, base + h.out + in_off, in_len,
+                             cudaMemcpyDeviceToHost, hp->out)))
+      return cuda_fail(e, "copy out to host");
+    if ((e = cudaMemcpyAsync(reinterpret_cast<char*>(lse_host) + l_off, base + h.lse + l_off,
+                             l_len, cudaMemcpyDeviceToHost, hp->out)))
+      return cuda_fail(e, "copy lse to host");
+  }
+  return LSH_OK;
+}
+
+// Makes `st` wait for everything queued on the three streams.  Each stream
+// gets its own event record, so a stream whose queue ended early (a failed
+// group) is joined as well; the first error is returned after all three.
+cudaError_t join_pipe(HostPipe* hp, cudaStream_t st) {
+  cudaError_t first = cudaSuccess;
+  const cudaStream_t streams[3] = {hp->in, hp->comp, hp->out};
+  for (cudaStream_t s : streams) {
+    cudaError_t e = cudaEventRecord(hp->out_done, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(st, hp->out_done, 0);
+    if (e != cudaSuccess && first == cudaSuccess) first = e;
+  }
+  return first;
+}
+
 }  // namespace
 
 unsigned int* device_error_word() {
@@ -430,43 +486,14 @@ lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void* qk_host,
   if ((e = cudaStreamWaitEvent(hp->in, hp->start, 0))) return cuda_fail(e, "wait start");
   if ((e = cudaStreamWaitEvent(hp->comp, hp->start, 0))) return cuda_fail(e, "wait start");
   if ((e = cudaStreamWaitEvent(hp->out, hp->start, 0))) return cuda_fail(e, "wait start");
-  if (h.rot_bytes &&
-      (e = cudaMemcpyAsync(base + h.rot, rotations_host, h.rot_bytes, cudaMemcpyHostToDevice,
-                           hp->in)))
-    return cuda_fail(e, "copy rotations to device");
-  for (int g = 0; g < G; ++g) {
-    const int b0 = (int)((long long)BH * g / G), b1 = (int)((long long)BH * (g + 1) / G);
-    const size_t in_off = (size_t)b0 * row_in, in_len = (size_t)(b1 - b0) * row_in;
-    const size_t l_off = (size_t)b0 * row_lse, l_len = (size_t)(b1 - b0) * row_lse;
-    // one cudaMemcpyAsync per tensor slice
-    if ((e = cudaMemcpyAsync(base + h.qk + in_off, static_cast<const char*>(qk_host) + in_off,
-                             in_len, cudaMemcpyHostToDevice, hp->in)))
-      return cuda_fail(e, "copy qk to device");
-    if ((e = cudaMemcpyAsync(base + h.v + in_off, static_cast<const char*>(v_host) + in_off,
-                             in_len, cudaMemcpyHostToDevice, hp->in)))
-      return cuda_fail(e, "copy v to device");
-    if ((e = cudaEventRecord(hp->in_done[g], hp->in))) return cuda_fail(e, "record copy-in");
-    if ((e = cudaStreamWaitEvent(hp->comp, hp->in_done[g], 0))) return cuda_fail(e, "wait copy-in");
-    Problem pg = p;
-    pg.B = 1;
-    pg.H = b1 - b0;
-    CHECK(forward_body(pg, base + h.qk + in_off, base + h.v + in_off,
-                       h.rot_bytes ? base + h.rot : nullptr, base + h.out + in_off,
-                       reinterpret_cast<float*>(base + h.lse + l_off), base + h.ws, hp->comp));
-    if ((e = cudaEventRecord(hp->comp_done[g], hp->comp))) return cuda_fail(e, "record compute");
-    if ((e = cudaStreamWaitEvent(hp->out, hp->comp_done[g], 0))) return cuda_fail(e, "wait compute");
-    if ((e = cudaMemcpyAsync(static_cast<char*>(out_host) + in_off, base + h.out + in_off, in_len,
-                             cudaMemcpyDeviceToHost, hp->out)))
-      return cuda_fail(e, "copy out to host");
-    if ((e = cudaMemcpyAsync(reinterpret_cast<char*>(lse_host) + l_off, base + h.lse + l_off,
-                             l_len, cudaMemcpyDeviceToHost, hp->out)))
-      return cuda_fail(e, "copy lse to host");
-  }
-  // The caller's stream continues once the last copy-out is done (which
-  // follows every compute and copy-in through the events above).
-  if ((e = cudaEventRecord(hp->out_done, hp->out))) return cuda_fail(e, "record done");
-  if ((e = cudaStreamWaitEvent(st, hp->out_done, 0))) return cuda_fail(e, "join stream");
-  return LSH_OK;
+  const lsh_status r = host_groups(p, h, hp, G, row_in, row_lse, qk_host, v_host,
+                                   rotations_host, out_host, lse_host, base);
+  // The caller's stream continues once all three streams are done, on
+  // success and on failure alike: the copies and kernels already queued
+  // use the caller's buffers, which must stay alive until they finish.
+  const cudaError_t je = join_pipe(hp, st);
+  if (r != LSH_OK) return r;
+  return je == cudaSuccess ? LSH_OK : cuda_fail(je, "join stream");
 }
 
 lsh_status lsh_attn_backward_workspace_size(const lsh_shape* shape, size_t* bytes) {
