@@ -132,14 +132,55 @@ def _ptr(t: Optional[torch.Tensor]):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _cuda(t: torch.Tensor, name: str, dtype=None):
+def _cuda(t: torch.Tensor, name: str, dtype=None, shape=None, like=None):
+    """Checks a tensor argument before its pointer reaches the library, which
+    sees only pointers and so cannot check extents: a CUDA tensor, contiguous,
+    of ``dtype`` and ``shape`` when given, on ``like``'s device when given."""
     if not isinstance(t, torch.Tensor) or not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if dtype is not None and t.dtype != dtype:
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if like is not None and t.device != like.device:
+        raise ValueError(f"{name} is on {t.device}, expected {like.device}")
     return t
+
+
+def _host(t: torch.Tensor, name: str, dtype, shape):
+    if not isinstance(t, torch.Tensor) or t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _qk(qk):
+    _cuda(qk, "qk")
+    if qk.dim() != 4:
+        raise ValueError(f"qk must be [B, H, L, d], got shape {tuple(qk.shape)}")
+    return qk.shape
+
+
+def _rot_shape(n_hashes, d, n_buckets, kmeans):
+    """rotations [n_h, d, n_b/2] (the random rotations), or the centroids
+    [n_h, d, n_b] of the routing-style assignment."""
+    return (n_hashes, d, n_buckets if kmeans else n_buckets // 2)
+
+
+def _rotations(rotations, qk, n_hashes, n_buckets, kmeans):
+    B, H, L, d = qk.shape
+    if n_buckets == 1 and not kmeans:
+        if rotations is not None:
+            raise ValueError("rotations must be None when n_buckets == 1")
+        return
+    if rotations is None:
+        raise ValueError("rotations is required when n_buckets > 1")
+    _cuda(rotations, "rotations", qk.dtype, _rot_shape(n_hashes, d, n_buckets, kmeans), qk)
 
 
 def _stream(stream):
@@ -159,13 +200,12 @@ def lsh_attn_hash(qk, rotations, n_buckets, n_hashes=None, *, portable=False, km
                   stream=None):
     """Stage 1.  qk [B,H,L,d]; rotations [n_h,d,n_b/2] (None when n_b == 1).
     Returns (buckets int16 [B,H,n_h,L], inv_norm float32 [B,H,L])."""
-    _cuda(qk, "qk")
-    if rotations is not None:
-        _cuda(rotations, "rotations", qk.dtype)
+    B, H, L, d = _qk(qk)
+    if rotations is not None and rotations.dim() == 3:
         n_hashes = rotations.shape[0]
     if n_hashes is None:
         n_hashes = 1
-    B, H, L, d = qk.shape
+    _rotations(rotations, qk, n_hashes, n_buckets, kmeans)
     shp = _shape_of(qk, n_hashes, n_buckets, 1, False, portable, kmeans=kmeans)
     buckets = torch.empty(B, H, n_hashes, L, dtype=torch.int16, device=qk.device)
     inv_norm = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
@@ -178,6 +218,8 @@ def lsh_attn_sort(buckets, n_buckets, *, want_undo=True, want_counts=False, stre
     """Stage 2.  buckets int16 [B,H,n_h,L].  Returns (perm, undo, counts); undo and
     counts are None unless asked for."""
     _cuda(buckets, "buckets", torch.int16)
+    if buckets.dim() != 4:
+        raise ValueError(f"buckets must be [B, H, n_h, L], got shape {tuple(buckets.shape)}")
     B, H, n_h, L = buckets.shape
     shp = make_shape(B, H, L, 8, n_h, n_buckets, 1, False, F32)
     perm = torch.empty(B, H, n_h, L, dtype=torch.int32, device=buckets.device)
@@ -189,14 +231,22 @@ def lsh_attn_sort(buckets, n_buckets, *, want_undo=True, want_counts=False, stre
     return perm, undo, counts
 
 
+def _stage3_args(qk, v, inv_norm, perm):
+    """qk and v [B,H,L,d], inv_norm [B,H,L], perm [B,H,n_h,L]; returns n_h."""
+    B, H, L, d = _qk(qk)
+    _cuda(v, "v", qk.dtype, qk.shape, qk)
+    _cuda(inv_norm, "inv_norm", torch.float32, (B, H, L), qk)
+    _cuda(perm, "perm", torch.int32, None, qk)
+    if perm.dim() != 4 or (perm.shape[0], perm.shape[1], perm.shape[3]) != (B, H, L):
+        raise ValueError(f"perm must be [{B}, {H}, n_h, {L}], got shape {tuple(perm.shape)}")
+    return perm.shape[2]
+
+
 def lsh_attn_chunked_fwd(qk, v, inv_norm, perm, chunk_len, causal, *, n_buckets=2,
                          portable=False, stream=None):
     """Stage 3.  Returns (o_rounds [B,H,n_h,L,d] in qk's dtype, lse_rounds f32 [B,H,n_h,L])."""
-    _cuda(qk, "qk")
-    _cuda(v, "v", qk.dtype)
-    _cuda(inv_norm, "inv_norm", torch.float32)
-    _cuda(perm, "perm", torch.int32)
-    B, H, n_h, L = perm.shape
+    n_h = _stage3_args(qk, v, inv_norm, perm)
+    B, H, L, d = qk.shape
     shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, portable)
     o_r = torch.empty(B, H, n_h, L, qk.shape[-1], dtype=qk.dtype, device=qk.device)
     lse_r = torch.empty(B, H, n_h, L, dtype=torch.float32, device=qk.device)
@@ -211,15 +261,12 @@ def lsh_attn_chunked_fwd_ex(qk, v, inv_norm, perm, chunk_len, causal, *, undo=No
     (every round's [B,H,n_h,L] int32, from lsh_attn_sort) is given, the
     bucket-equality mask when ``buckets`` ([B,H,n_h,L] int16) is given.
     Returns (o_rounds, lse_rounds)."""
-    _cuda(qk, "qk")
-    _cuda(v, "v", qk.dtype)
-    _cuda(inv_norm, "inv_norm", torch.float32)
-    _cuda(perm, "perm", torch.int32)
+    n_h = _stage3_args(qk, v, inv_norm, perm)
+    B, H, L, d = qk.shape
     if undo is not None:
-        _cuda(undo, "undo", torch.int32)
+        _cuda(undo, "undo", torch.int32, perm.shape, qk)
     if buckets is not None:
-        _cuda(buckets, "buckets", torch.int16)
-    B, H, n_h, L = perm.shape
+        _cuda(buckets, "buckets", torch.int16, perm.shape, qk)
     shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, False, undo is not None,
                     buckets is not None)
     o_r = torch.empty(B, H, n_h, L, qk.shape[-1], dtype=qk.dtype, device=qk.device)
@@ -233,13 +280,27 @@ def lsh_attn_chunked_fwd_ex(qk, v, inv_norm, perm, chunk_len, causal, *, undo=No
 def lsh_attn_combine(o_rounds, lse_rounds, *, stream=None):
     """Stage 4.  Returns (out [B,H,L,d], lse f32 [B,H,L])."""
     _cuda(o_rounds, "o_rounds")
-    _cuda(lse_rounds, "lse_rounds", torch.float32)
+    if o_rounds.dim() != 5:
+        raise ValueError(f"o_rounds must be [B, H, n_h, L, d], got shape {tuple(o_rounds.shape)}")
     B, H, n_h, L, d = o_rounds.shape
+    _cuda(lse_rounds, "lse_rounds", torch.float32, (B, H, n_h, L), o_rounds)
     shp = make_shape(B, H, L, d, n_h, 2, 1, False, o_rounds.dtype)
     out = torch.empty(B, H, L, d, dtype=o_rounds.dtype, device=o_rounds.device)
     lse = torch.empty(B, H, L, dtype=torch.float32, device=o_rounds.device)
     _check(lib().lsh_attn_combine(ctypes.byref(shp), _ptr(o_rounds), _ptr(lse_rounds), _ptr(out),
                                   _ptr(lse), _stream(stream)))
+    return out, lse
+
+
+def _outputs(qk, out, lse):
+    """out [B,H,L,d] in qk's dtype and lse f32 [B,H,L]: checked, or allocated."""
+    B, H, L, d = qk.shape
+    if out is None:
+        out = torch.empty_like(qk)
+    if lse is None:
+        lse = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
+    _cuda(out, "out", qk.dtype, qk.shape, qk)
+    _cuda(lse, "lse", torch.float32, (B, H, L), qk)
     return out, lse
 
 
@@ -254,20 +315,16 @@ def lsh_attn_forward(qk, v, rotations, n_hashes, n_buckets, chunk_len, causal, *
                      bucket_mask=False, kmeans=False, stream=None):
     """The fused pass.  Returns (out [B,H,L,d], lse f32 [B,H,L]).  ``workspace`` (a
     uint8 CUDA tensor) can be passed in to avoid an allocation per call."""
-    _cuda(qk, "qk")
-    _cuda(v, "v", qk.dtype)
-    if rotations is not None:
-        _cuda(rotations, "rotations", qk.dtype)
-    B, H, L, d = qk.shape
+    B, H, L, d = _qk(qk)
+    _cuda(v, "v", qk.dtype, qk.shape, qk)
+    _rotations(rotations, qk, n_hashes, n_buckets, kmeans)
     shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable, dedup, bucket_mask,
                     kmeans)
     need = lsh_attn_forward_workspace_size(shp)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=qk.device)
-    if out is None:
-        out = torch.empty_like(qk)
-    if lse is None:
-        lse = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
+    _cuda(workspace, "workspace", None, None, qk)
+    out, lse = _outputs(qk, out, lse)
     _check(lib().lsh_attn_forward(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(rotations),
                                   _ptr(out), _ptr(lse), _ptr(workspace),
                                   ctypes.c_size_t(workspace.numel()), _stream(stream)))
@@ -284,10 +341,19 @@ def lsh_attn_forward_host(shape: Shape, qk_host, v_host, rot_host, out_host, lse
                           device_buffer, *, stream=None):
     """Forward pass from host tensors (ideally pinned): enqueues the copies in,
     the pass and the copies out on ``stream``; the caller synchronises."""
-    for name, t in (("qk_host", qk_host), ("v_host", v_host), ("out_host", out_host),
-                    ("lse_host", lse_host)):
-        if t.is_cuda or not t.is_contiguous():
-            raise ValueError(f"{name} must be a contiguous host tensor")
+    dt = torch.float32 if shape.dtype == F32 else torch.bfloat16
+    x_shape = (shape.batch, shape.heads, shape.seq_len, shape.d_k)
+    for name, t in (("qk_host", qk_host), ("v_host", v_host), ("out_host", out_host)):
+        _host(t, name, dt, x_shape)
+    _host(lse_host, "lse_host", torch.float32, x_shape[:3])
+    kmeans = bool(shape.flags & FLAG_KMEANS)
+    if shape.n_buckets > 1 or kmeans:
+        if rot_host is None:
+            raise ValueError("rot_host is required when n_buckets > 1")
+        _host(rot_host, "rot_host", dt,
+              _rot_shape(shape.n_hashes, shape.d_k, shape.n_buckets, kmeans))
+    elif rot_host is not None:
+        raise ValueError("rot_host must be None when n_buckets == 1")
     _cuda(device_buffer, "device_buffer")
     _check(lib().lsh_attn_forward_host(
         ctypes.byref(shape), _ptr(qk_host), _ptr(v_host), _ptr(rot_host), _ptr(out_host),
@@ -305,16 +371,11 @@ def lsh_attn_forward_noalloc(qk, v, rotations, n_hashes, n_buckets, chunk_len, c
     device, so calls must not overlap on the GPU; larger problems raise
     LshError(LSH_ERR_WORKSPACE).  (This Python wrapper still allocates ``out``
     and ``lse`` with torch when they are not passed in.)"""
-    _cuda(qk, "qk")
-    _cuda(v, "v", qk.dtype)
-    if rotations is not None:
-        _cuda(rotations, "rotations", qk.dtype)
-    B, H, L, d = qk.shape
+    B, H, L, d = _qk(qk)
+    _cuda(v, "v", qk.dtype, qk.shape, qk)
+    _rotations(rotations, qk, n_hashes, n_buckets, False)
     shp = _shape_of(qk, n_hashes, n_buckets, chunk_len, causal, portable)
-    if out is None:
-        out = torch.empty_like(qk)
-    if lse is None:
-        lse = torch.empty(B, H, L, dtype=torch.float32, device=qk.device)
+    out, lse = _outputs(qk, out, lse)
     _check(lib().lsh_attn_forward_noalloc(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(rotations),
                                           _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
@@ -336,18 +397,16 @@ def lsh_attn_backward(qk, v, inv_norm, perm, out, lse, dout, chunk_len, causal, 
     """Gradients of out w.r.t. qk and v with the buckets and sort held fixed.
     perm [B,H,n_h,L] and inv_norm from stages 1-2, out and lse from the
     forward.  Returns (dqk, dv), float32 [B,H,L,d]."""
-    _cuda(qk, "qk")
-    _cuda(v, "v", qk.dtype)
-    _cuda(inv_norm, "inv_norm", torch.float32)
-    _cuda(perm, "perm", torch.int32)
-    _cuda(out, "out", qk.dtype)
-    _cuda(lse, "lse", torch.float32)
-    _cuda(dout, "dout", qk.dtype)
-    B, H, n_h, L = perm.shape
+    n_h = _stage3_args(qk, v, inv_norm, perm)
+    B, H, L, d = qk.shape
+    _cuda(out, "out", qk.dtype, qk.shape, qk)
+    _cuda(lse, "lse", torch.float32, (B, H, L), qk)
+    _cuda(dout, "dout", qk.dtype, qk.shape, qk)
     shp = _shape_of(qk, n_h, n_buckets, chunk_len, causal, False)
     need = lsh_attn_backward_workspace_size(shp)
     if workspace is None:
         workspace = torch.empty(need, dtype=torch.uint8, device=qk.device)
+    _cuda(workspace, "workspace", None, None, qk)
     dqk = torch.empty(qk.shape, dtype=torch.float32, device=qk.device)
     dv = torch.empty(v.shape, dtype=torch.float32, device=qk.device)
     _check(lib().lsh_attn_backward(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(inv_norm),

@@ -114,3 +114,28 @@ def test_binding_fails_loudly_without_gpu_tensors():
     with pytest.raises(ValueError):
         lsh.lsh_attn_forward(torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16),
                              torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16), None, 1, 1, 64, True)
+
+
+def test_binding_checks_host_tensor_shapes_before_any_copy():
+    # The library sees only pointers, so the binding checks every extent: a
+    # host tensor of the wrong shape, dtype or a missing rotation table raises
+    # before the device buffer is even looked at (here it is not a CUDA tensor).
+    import torch
+    shp = lsh.make_shape(1, 2, 128, 64, 2, 16, 64, True, torch.bfloat16)
+    x = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16)
+    rot = torch.zeros(2, 64, 8, dtype=torch.bfloat16)
+    lse = torch.zeros(1, 2, 128, dtype=torch.float32)
+    cases = [
+        (x, x, rot, x, torch.zeros(1, 2, 64, dtype=torch.float32)),    # lse too short
+        (x, x[:, :1].contiguous(), rot, x, lse),                       # v has one head
+        (x, x, torch.zeros(2, 64, 16, dtype=torch.bfloat16), x, lse),  # rotations n_b wide
+        (x, x, None, x, lse),                                          # rotations missing
+        (x, x, rot, torch.zeros(1, 2, 128, 64), lse),                  # out in float32
+    ]
+    for qk_h, v_h, rot_h, out_h, lse_h in cases:
+        with pytest.raises((ValueError, TypeError)) as ei:
+            lsh.lsh_attn_forward_host(shp, qk_h, v_h, rot_h, out_h, lse_h, "not a tensor")
+        assert "device_buffer" not in str(ei.value)
+    km = lsh.make_shape(1, 2, 128, 64, 2, 16, 64, True, torch.bfloat16, kmeans=True)
+    with pytest.raises(ValueError, match="rot_host"):  # centroids are [n_h, d, n_b]
+        lsh.lsh_attn_forward_host(km, x, x, rot, x, lse, "not a tensor")

@@ -568,3 +568,37 @@ def test_backward_matches_oracle(wl):
             assert err[~alone].max() <= tol, f"{name} head {h}: {err[~alone].max():.3e}"
             if alone.any():
                 assert err[alone].max() <= max(tol, 1e-2), f"{name} head {h} (alone)"
+
+
+def test_binding_rejects_mismatched_device_tensors():
+    # The library sees only pointers; the binding must refuse every tensor
+    # whose extent disagrees with qk's before a pointer reaches a kernel.
+    wl = W.small("shapes", heads=2, seq_len=256, n_hashes=2, n_buckets=16)
+    qk, v, rot = [t.to(DEV) for t in W.make_inputs(wl)]
+    B, H, L, d = qk.shape
+    bad_calls = [
+        lambda: lsh.lsh_attn_forward(qk, v[:, :1].contiguous(), rot, 2, 16, 64, True),
+        lambda: lsh.lsh_attn_forward(qk, v, rot[:1].contiguous(), 2, 16, 64, True),
+        lambda: lsh.lsh_attn_forward(qk, v, rot, 2, 32, 64, True),  # rot is n_b/2 = 8 wide
+        lambda: lsh.lsh_attn_forward(qk, v, None, 2, 16, 64, True),
+        lambda: lsh.lsh_attn_forward(qk, v, rot, 2, 16, 64, True,
+                                     out=torch.empty(B, H, L // 2, d, dtype=qk.dtype, device=DEV)),
+        lambda: lsh.lsh_attn_forward(qk, v, rot, 2, 16, 64, True,
+                                     lse=torch.empty(B, H, L, dtype=torch.bfloat16, device=DEV)),
+        lambda: lsh.lsh_attn_hash(qk, rot, 16, 2, kmeans=True),  # centroids are n_b wide
+        lambda: lsh.lsh_attn_forward_noalloc(qk, v[..., :32].contiguous(), rot, 2, 16, 64, True),
+    ]
+    b, inv = lsh.lsh_attn_hash(qk, rot, 16, 2)
+    perm, undo, _ = lsh.lsh_attn_sort(b, 16)
+    bad_calls += [
+        lambda: lsh.lsh_attn_chunked_fwd(qk, v, inv, perm[..., :128].contiguous(), 64, True),
+        lambda: lsh.lsh_attn_chunked_fwd(qk, v, inv[:, :1].contiguous(), perm, 64, True),
+        lambda: lsh.lsh_attn_chunked_fwd_ex(qk, v, inv, perm, 64, True,
+                                            undo=undo[:, :, :1].contiguous()),
+        lambda: lsh.lsh_attn_combine(torch.empty(B, H, 2, L, d, dtype=qk.dtype, device=DEV),
+                                     torch.empty(B, H, 2, L // 2, device=DEV)),
+    ]
+    for i, call in enumerate(bad_calls):
+        with pytest.raises((ValueError, TypeError)):
+            call()
+    lsh.lsh_attn_device_check()
