@@ -239,7 +239,8 @@ LSH_ATTN_API lsh_status lsh_attn_backward(const lsh_shape* shape, const void* qk
  * device, runs the forward pass, and copies out and lse back.  The (batch,
  * head) pairs are independent, so they go in up to 8 groups through three
  * library-owned streams (copy in, compute, copy out): a group's inputs cross
- * PCIe while the previous group computes and the one before it copies back.
+ * PCIe while the previous group computes and the one before it copies back;
+ * a group's qk crosses before its v, and its hash and sort start on qk alone.
  * The work starts after what is already queued on `stream`, and `stream`
  * waits for all of it, so the caller synchronises `stream` before reading
  * out_host / lse_host.  Calls on one device enqueue one at a time (a mutex

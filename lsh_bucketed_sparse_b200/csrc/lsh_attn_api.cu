@@ -159,21 +159,52 @@ Workspace workspace_layout(const Problem& p) {
   return w;
 }
 
-lsh_status forward_body(const Problem& p, const void* qk, const void* v, const void* rot,
-                        void* out, float* lse, void* ws, cudaStream_t st) {
+namespace {
+
+// The forward pass in two halves over one workspace: hash and sort read only
+// qk, so a caller whose v arrives later can start them first.
+struct WsPtrs {
+  int16_t* buckets;
+  float* inv_norm;
+  int32_t* perm;
+  int32_t* undo;
+  void* o_r;
+  float* lse_r;
+  void* sort_scratch;
+};
+
+WsPtrs ws_ptrs(const Problem& p, void* ws) {
   const Workspace w = workspace_layout(p);
   char* base = static_cast<char*>(ws);
-  int16_t* buckets = reinterpret_cast<int16_t*>(base + w.buckets);
-  float* inv_norm = reinterpret_cast<float*>(base + w.inv_norm);
-  int32_t* perm = reinterpret_cast<int32_t*>(base + w.perm);
-  void* o_r = base + w.o_rounds;
-  float* lse_r = reinterpret_cast<float*>(base + w.lse_rounds);
-  CHECK(run_hash(p, qk, rot, buckets, inv_norm, st));
-  int32_t* undo = p.dedup ? reinterpret_cast<int32_t*>(base + w.undo) : nullptr;
-  CHECK(run_sort(p, buckets, perm, undo, nullptr, base + w.sort_scratch, st));
-  CHECK(run_attn(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st));
-  CHECK(run_combine(p, o_r, lse_r, out, lse, st));
-  return LSH_OK;
+  return {reinterpret_cast<int16_t*>(base + w.buckets),
+          reinterpret_cast<float*>(base + w.inv_norm),
+          reinterpret_cast<int32_t*>(base + w.perm),
+          p.dedup ? reinterpret_cast<int32_t*>(base + w.undo) : nullptr,
+          base + w.o_rounds,
+          reinterpret_cast<float*>(base + w.lse_rounds),
+          base + w.sort_scratch};
+}
+
+lsh_status forward_hash_sort(const Problem& p, const void* qk, const void* rot, void* ws,
+                             cudaStream_t st) {
+  const WsPtrs w = ws_ptrs(p, ws);
+  CHECK(run_hash(p, qk, rot, w.buckets, w.inv_norm, st));
+  return run_sort(p, w.buckets, w.perm, w.undo, nullptr, w.sort_scratch, st);
+}
+
+lsh_status forward_attend_combine(const Problem& p, const void* qk, const void* v, void* out,
+                                  float* lse, void* ws, cudaStream_t st) {
+  const WsPtrs w = ws_ptrs(p, ws);
+  CHECK(run_attn(p, qk, v, w.inv_norm, w.perm, w.undo, w.buckets, w.o_r, w.lse_r, st));
+  return run_combine(p, w.o_r, w.lse_r, out, lse, st);
+}
+
+}  // namespace
+
+lsh_status forward_body(const Problem& p, const void* qk, const void* v, const void* rot,
+                        void* out, float* lse, void* ws, cudaStream_t st) {
+  CHECK(forward_hash_sort(p, qk, rot, ws, st));
+  return forward_attend_combine(p, qk, v, out, lse, ws, st);
 }
 
 namespace {
@@ -204,10 +235,12 @@ HostStaging host_layout(const Problem& p) {
 // through three streams: copies in, compute, copies out.  Group g's inputs
 // cross PCIe while group g-1 is computed and group g-2's outputs come back;
 // the compute stream runs the groups in order, so one workspace serves all.
+// A group's qk is copied before its v, and its hash and sort (which read only
+// qk) start as soon as qk has arrived.
 constexpr int kMaxGroups = 8;
 struct HostPipe {
   cudaStream_t in, comp, out;
-  cudaEvent_t start, in_done[kMaxGroups], comp_done[kMaxGroups], out_done;
+  cudaEvent_t start, qk_done[kMaxGroups], in_done[kMaxGroups], comp_done[kMaxGroups], out_done;
   bool ok;
 };
 HostPipe g_pipe[kMaxDevices];
@@ -223,7 +256,8 @@ HostPipe* host_pipe(int dev) {
            cudaEventCreateWithFlags(&h.start, cudaEventDisableTiming) == cudaSuccess &&
            cudaEventCreateWithFlags(&h.out_done, cudaEventDisableTiming) == cudaSuccess;
     for (int g = 0; h.ok && g < kMaxGroups; ++g)
-      h.ok = cudaEventCreateWithFlags(&h.in_done[g], cudaEventDisableTiming) == cudaSuccess &&
+      h.ok = cudaEventCreateWithFlags(&h.qk_done[g], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&h.in_done[g], cudaEventDisableTiming) == cudaSuccess &&
              cudaEventCreateWithFlags(&h.comp_done[g], cudaEventDisableTiming) == cudaSuccess;
   });
   return g_pipe[dev].ok ? &g_pipe[dev] : nullptr;
@@ -271,17 +305,23 @@ lsh_status host_groups(const Problem& p, const HostStaging& h, HostPipe* hp, int
     if ((e = cudaMemcpyAsync(base + h.qk + in_off, static_cast<const char*>(qk_host) + in_off,
                              in_len, cudaMemcpyHostToDevice, hp->in)))
       return cuda_fail(e, "copy qk to device");
+    if ((e = cudaEventRecord(hp->qk_done[g], hp->in))) return cuda_fail(e, "record copy-in");
     if ((e = cudaMemcpyAsync(base + h.v + in_off, static_cast<const char*>(v_host) + in_off,
                              in_len, cudaMemcpyHostToDevice, hp->in)))
       return cuda_fail(e, "copy v to device");
     if ((e = cudaEventRecord(hp->in_done[g], hp->in))) return cuda_fail(e, "record copy-in");
-    if ((e = cudaStreamWaitEvent(hp->comp, hp->in_done[g], 0))) return cuda_fail(e, "wait copy-in");
     Problem pg = p;
     pg.B = 1;
     pg.H = b1 - b0;
-    CHECK(forward_body(pg, base + h.qk + in_off, base + h.v + in_off,
-                       h.rot_bytes ? base + h.rot : nullptr, base + h.out + in_off,
-                       reinterpret_cast<float*>(base + h.lse + l_off), base + h.ws, hp->comp));
+    // (the rotations were queued on the same stream before the first qk)
+    if ((e = cudaStreamWaitEvent(hp->comp, hp->qk_done[g], 0))) return cuda_fail(e, "wait copy-in");
+    CHECK(forward_hash_sort(pg, base + h.qk + in_off, h.rot_bytes ? base + h.rot : nullptr,
+                            base + h.ws, hp->comp));
+    if ((e = cudaStreamWaitEvent(hp->comp, hp->in_done[g], 0))) return cuda_fail(e, "wait copy-in");
+    CHECK(forward_attend_combine(pg, base + h.qk + in_off, base + h.v + in_off,
+                                 base + h.out + in_off,
+                                 reinterpret_cast<float*>(base + h.lse + l_off), base + h.ws,
+                                 hp->comp));
     if ((e = cudaEventRecord(hp->comp_done[g], hp->comp))) return cuda_fail(e, "record compute");
     if ((e = cudaStreamWaitEvent(hp->out, hp->comp_done[g], 0))) return cuda_fail(e, "wait compute");
     if ((e = cudaMemcpyAsync(static_cast<char*>(out_host) + in_off, base + h.out + in_off, in_len,
