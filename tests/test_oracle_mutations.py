@@ -1,10 +1,14 @@
 """Each plausible mistake, planted in the oracle on the CPU, must fail a pin.
 
 The mutations are applied with monkeypatch to a copy of one oracle function;
-the pin that should catch it is run and must raise.
+the pin that should catch it is run and must raise.  A mistake inside a
+longer function is planted by editing one line of that function's own source
+and compiling the result in the oracle's namespace.
 """
 
+import inspect
 import math
+import textwrap
 
 import numpy as np
 import pytest
@@ -87,3 +91,63 @@ def test_pin_catches_wrong_self_constant(monkeypatch):
     monkeypatch.setattr(O, "SELF_SCORE", -1e5 + 0.5)
     with pytest.raises(AssertionError):
         P.test_attention_golden_tiny()
+
+
+def _source_mutant(name, old, new):
+    """The oracle function ``name`` with its one occurrence of ``old``
+    replaced by ``new``, compiled against the oracle module's globals."""
+    src = textwrap.dedent(inspect.getsource(getattr(O, name)))
+    assert src.count(old) == 1, (name, old)
+    ns = dict(vars(O))
+    exec(compile(src.replace(old, new), f"<mutant of {name}>", "exec"), ns)
+    return ns[name]
+
+
+SOURCE_CASES = [
+    # the short last chunk of a ragged length is dropped
+    ("attend_round", "n_c = -(-L // c)", "n_c = L // c",
+     lambda: P.test_brute_force_small(20, 8, 4, 2, True)),
+    # causal mask pointing the wrong way (a key in the past is hidden)
+    ("attend_round", "np.where(kp > qp, -np.inf, s)", "np.where(kp < qp, -np.inf, s)",
+     lambda: P.test_brute_force_small(16, 4, 4, 2, True)),
+    # the bucket-equality mask is never applied
+    ("attend_round", "if bucket_r is not None:", "if False:", P.test_bucket_mask_brute_force),
+    # the duplicate count ignores the look-back chunk
+    ("duplicate_counts", "(diff == 0) | (diff == 1)", "(diff == 0)", P.test_dedup_gives_set_union),
+    # the routing-style assignment takes |x . mu| like the rotation hash
+    ("kmeans_head", "np.argmax(p, axis=1)", "np.argmax(np.abs(p), axis=1)",
+     P.test_kmeans_with_plus_minus_rotation_is_the_lsh_hash),
+    # ... or the smallest dot product
+    ("kmeans_head", "np.argmax(p, axis=1)", "np.argmin(p, axis=1)",
+     P.test_kmeans_picks_the_largest_coordinate_with_basis_centroids),
+    # the margin is taken against the smallest entry, not the runner-up
+    ("hash_head", "top2[:, 1] - top2[:, 0]", "top2[:, 1] - z.min(axis=1)", P.test_hash_golden_tiny),
+    # no gradient through the key normalisation
+    ("backward_head", "X / torch.where(norm > 0, norm, 1.0)[:, None]",
+     "X.detach() / torch.where(norm > 0, norm, 1.0).detach()[:, None]",
+     lambda: P.test_backward_matches_finite_differences(False)),
+    # the causal mask left out of the backward's forward
+    ("backward_head", "if causal:", "if False:",
+     lambda: P.test_backward_matches_finite_differences(True)),
+    # combine weights normalised over positions instead of rounds
+    ("backward_head", "torch.softmax(Lr, dim=0)", "torch.softmax(Lr, dim=1)",
+     P.test_backward_of_v_is_the_attention_transpose),
+]
+
+
+@pytest.mark.filterwarnings("ignore::RuntimeWarning")  # a mutant may divide by zero
+@pytest.mark.parametrize("name,old,new,pin", SOURCE_CASES,
+                         ids=[f"{c[0]}-{i}" for i, c in enumerate(SOURCE_CASES)])
+def test_pin_catches_source_mutation(monkeypatch, name, old, new, pin):
+    monkeypatch.setattr(O, name, _source_mutant(name, old, new))
+    with pytest.raises(AssertionError):
+        pin()
+
+
+def test_source_mutant_without_change_passes(monkeypatch):
+    # The mutation harness itself leaves a function intact when nothing is
+    # replaced: the recompiled copy must still satisfy its pins.
+    monkeypatch.setattr(O, "attend_round", _source_mutant("attend_round", "n_c = -(-L // c)",
+                                                          "n_c = -(-L // c)"))
+    P.test_brute_force_small(20, 8, 4, 2, True)
+    P.test_bucket_mask_brute_force()
