@@ -13,12 +13,14 @@
 // The self pair's score is the constant -1e5 (no gradient to qk), and a key
 // of zero norm has k_hat = 0 and passes no gradient through the key.
 //
-// CUDA cores, float32: one CTA per (b*h, round, chunk), one warp per query
-// (the forward's CUDA-core layout); dv, dq and dk_hat are accumulated with
-// float32 atomics, so the summation order (and the last bits) can change
-// from run to run.  When the window's dv and dk_hat rows fit in shared
-// memory (SACC), the CTA sums its queries' contributions there and adds each
-// window row to global memory once.
+// CUDA cores, float32, one CTA per (b*h, round, chunk); dv, dq and dk_hat
+// are accumulated across CTAs with float32 atomics, so the summation order
+// (and the last bits) can change from run to run.  For c = 64 and d = 64 the
+// chunk's pairs run as register tiles (bwd_pairs_tiled_kernel).  Other shapes
+// take one warp per query (the forward's CUDA-core layout): when the window's
+// keys, values and sums fit in shared memory the CTA stages them there
+// (bwd_pairs_staged_kernel), else it keeps only the sums there (SACC) or
+// adds every pair's terms to global memory.
 #include "common.cuh"
 #include "internal.h"
 
@@ -269,6 +271,198 @@ bwd_pairs_staged_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   }
 }
 
+// The pairs of one chunk for c = 64 and d = 64 as register tiles.  The
+// chunk's queries (qk and dout rows) and its window's keys (normalised) and
+// values are staged once in shared memory; the chunk's products then run on
+// CUDA cores with each thread holding a tile of the result in registers:
+//   S = Q K_hat^T and dP = dout V^T        64 x 128, 4 x 8 per thread
+//   P = exp(S/sqrt(d) - LSE), dS = P (dP - delta)/sqrt(d), masks applied
+//   dV = P^T dout and dK_hat = dS^T Q      128 x 64, 8 x 4 per thread
+//   dQ = dS K_hat                          64 x 64, 4 x 4 per thread
+// and the CTA adds each row of dV, dK_hat and dQ to global memory once, in
+// 16-byte vector atomics.  Missing rows (a short last chunk, the first
+// chunk's absent look-back) are zeros with position -1: never visible.
+namespace tiled {
+constexpr int C = 64, D = 64, NW = 2 * C, kTileThreads = 256;
+constexpr int kKt = NW + 1;   // row of the transposed keys and values [D][NW + 1]
+constexpr int kPs = NW + 16;  // row of P and dS [C][NW + 16]
+constexpr int oQ = 0, oG = oQ + C * D, oKt = oG + C * D, oVt = oKt + D * kKt,
+              oP = oVt + D * kKt, oDS = oP + C * kPs, oLse = oDS + C * kPs, oDl = oLse + C,
+              oPq = oDl + C, oPk = oPq + C, kFloats = oPk + NW;
+constexpr size_t kSmem = (size_t)kFloats * sizeof(float);
+static_assert(NW * D <= D * kKt, "the row-major keys reuse the values' buffer");
+static_assert(oG % 4 == 0 && oVt % 4 == 0, "float4 rows");
+static_assert(kTileThreads == 16 * 16 && C == 4 * 16 && NW == 8 * 16 && D == 4 * 16, "tiling");
+}  // namespace tiled
+
+template <typename T>
+__global__ void __launch_bounds__(tiled::kTileThreads, 1)
+bwd_pairs_tiled_kernel(const T* __restrict__ qk, const T* __restrict__ v,
+                       const float* __restrict__ inv_norm, const int32_t* __restrict__ perm,
+                       const float* __restrict__ lse, const T* __restrict__ dout,
+                       const float* __restrict__ delta, float* __restrict__ dq,
+                       float* __restrict__ dv, float* __restrict__ dkh, int L, int n_h,
+                       int causal, float scale) {
+  using namespace tiled;
+  extern __shared__ float4 sh4[];
+  float* sh = reinterpret_cast<float*>(sh4);
+  float* Qs = sh + oQ;    // [C][D] query rows of qk
+  float* Gs = sh + oG;    // [C][D] query rows of dout
+  float* Kt = sh + oKt;   // [D][kKt] normalised keys, transposed
+  float* Vt = sh + oVt;   // [D][kKt] values, transposed; later the keys row-major
+  float* Ps = sh + oP;    // [C][kPs]
+  float* DSs = sh + oDS;  // [C][kPs], already divided by sqrt(d)
+  float* lse_q = sh + oLse;
+  float* dl_q = sh + oDl;
+  int* pos_q = reinterpret_cast<int*>(sh + oPq);
+  int* pos_k = reinterpret_cast<int*>(sh + oPk);
+  const int n_c = (L + C - 1) / C;
+  const int k = (int)(blockIdx.x % n_c);
+  const int r = (int)((blockIdx.x / n_c) % n_h);
+  const size_t bh = blockIdx.x / ((size_t)n_c * n_h);
+  const int tid = threadIdx.x;
+  const int32_t* P = perm + (bh * n_h + r) * (size_t)L;
+  const T* X = qk + bh * (size_t)L * D;
+  const T* V = v + bh * (size_t)L * D;
+  const T* G = dout + bh * (size_t)L * D;
+  const float* IN = inv_norm + bh * (size_t)L;
+  float* DQ = dq + bh * (size_t)L * D;
+  float* DV = dv + bh * (size_t)L * D;
+  float* DK = dkh + bh * (size_t)L * D;
+  const int q0 = k * C, nq = min(C, L - q0);
+  const int k0 = k > 0 ? q0 - C : 0, nw = min(q0 + C, L) - k0;
+
+  if (tid < C) {
+    const int i = tid < nq ? P[q0 + tid] : -1;
+    pos_q[tid] = i;
+    lse_q[tid] = i >= 0 ? lse[bh * (size_t)L + i] : 0.f;
+    dl_q[tid] = i >= 0 ? delta[bh * (size_t)L + i] : 0.f;
+  }
+  if (tid < NW) pos_k[tid] = tid < nw ? P[k0 + tid] : -1;
+  __syncthreads();
+  for (int idx = tid; idx < C * D; idx += kTileThreads) {
+    const int i = pos_q[idx / D], e = idx % D;
+    Qs[idx] = i >= 0 ? to_f32(X[(size_t)i * D + e]) : 0.f;
+    Gs[idx] = i >= 0 ? to_f32(G[(size_t)i * D + e]) : 0.f;
+  }
+  for (int idx = tid; idx < NW * D; idx += kTileThreads) {
+    const int w = idx / D, e = idx % D, j = pos_k[w];
+    Kt[e * kKt + w] = j >= 0 ? to_f32(X[(size_t)j * D + e]) * IN[j] : 0.f;
+    Vt[e * kKt + w] = j >= 0 ? to_f32(V[(size_t)j * D + e]) : 0.f;
+  }
+  __syncthreads();
+
+  {  // S, dP -> P, dS: rows m = mq + 16a, columns w = kw + 16b
+    const int mq = tid >> 4, kw = tid & 15;
+    float s[4][8], gp[4][8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int b = 0; b < 8; ++b) s[a][b] = gp[a][b] = 0.f;
+#pragma unroll 2
+    for (int e = 0; e < D; ++e) {
+      float qv[4], gv[4], kv[8], vv[8];
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        qv[a] = Qs[(mq + 16 * a) * D + e];
+        gv[a] = Gs[(mq + 16 * a) * D + e];
+      }
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        kv[b] = Kt[e * kKt + kw + 16 * b];
+        vv[b] = Vt[e * kKt + kw + 16 * b];
+      }
+#pragma unroll
+      for (int a = 0; a < 4; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+          s[a][b] = fmaf(qv[a], kv[b], s[a][b]);
+          gp[a][b] = fmaf(gv[a], vv[b], gp[a][b]);
+        }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int m = mq + 16 * a, i = pos_q[m];
+      const float LSE = lse_q[m], dl = dl_q[m];
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const int w = kw + 16 * b, j = pos_k[w];
+        float pv = 0.f, ds = 0.f;
+        if (i >= 0 && j >= 0 && !(causal && j > i)) {
+          pv = expf((j == i ? kSelfScore : s[a][b] * scale) - LSE);
+          if (j != i) ds = pv * (gp[a][b] - dl) * scale;
+        }
+        Ps[m * kPs + w] = pv;
+        DSs[m * kPs + w] = ds;
+      }
+    }
+  }
+  __syncthreads();
+  float* Kr = Vt;  // [NW][D] normalised keys, row-major (the values are done)
+  for (int idx = tid; idx < NW * D; idx += kTileThreads) Kr[idx] = Kt[(idx % D) * kKt + idx / D];
+  __syncthreads();
+
+  {  // dV = P^T dout, dK_hat = dS^T Q: rows w = kw + 16b, columns 4 eq .. 4 eq + 3
+    const int kw = tid & 15, eq = tid >> 4;
+    float av[8][4], ak[8][4];
+#pragma unroll
+    for (int b = 0; b < 8; ++b)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) av[b][t] = ak[b][t] = 0.f;
+#pragma unroll 2
+    for (int m = 0; m < C; ++m) {
+      const float4 g4 = *reinterpret_cast<const float4*>(Gs + m * D + 4 * eq);
+      const float4 x4 = *reinterpret_cast<const float4*>(Qs + m * D + 4 * eq);
+      const float gq[4] = {g4.x, g4.y, g4.z, g4.w}, xq[4] = {x4.x, x4.y, x4.z, x4.w};
+#pragma unroll
+      for (int b = 0; b < 8; ++b) {
+        const float pb = Ps[m * kPs + kw + 16 * b], db = DSs[m * kPs + kw + 16 * b];
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          av[b][t] = fmaf(pb, gq[t], av[b][t]);
+          ak[b][t] = fmaf(db, xq[t], ak[b][t]);
+        }
+      }
+    }
+#pragma unroll
+    for (int b = 0; b < 8; ++b) {
+      const int j = pos_k[kw + 16 * b];
+      if (j < 0) continue;
+      atomicAdd(reinterpret_cast<float4*>(DV + (size_t)j * D + 4 * eq),
+                make_float4(av[b][0], av[b][1], av[b][2], av[b][3]));
+      atomicAdd(reinterpret_cast<float4*>(DK + (size_t)j * D + 4 * eq),
+                make_float4(ak[b][0], ak[b][1], ak[b][2], ak[b][3]));
+    }
+  }
+  {  // dQ = dS K_hat: rows m = mq + 16a, columns 4 eq .. 4 eq + 3
+    const int eq = tid & 15, mq = tid >> 4;
+    float aq[4][4];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int t = 0; t < 4; ++t) aq[a][t] = 0.f;
+#pragma unroll 4
+    for (int w = 0; w < NW; ++w) {
+      const float4 k4 = *reinterpret_cast<const float4*>(Kr + w * D + 4 * eq);
+#pragma unroll
+      for (int a = 0; a < 4; ++a) {
+        const float d_ = DSs[(mq + 16 * a) * kPs + w];
+        aq[a][0] = fmaf(d_, k4.x, aq[a][0]);
+        aq[a][1] = fmaf(d_, k4.y, aq[a][1]);
+        aq[a][2] = fmaf(d_, k4.z, aq[a][2]);
+        aq[a][3] = fmaf(d_, k4.w, aq[a][3]);
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 4; ++a) {
+      const int i = pos_q[mq + 16 * a];
+      if (i < 0) continue;
+      atomicAdd(reinterpret_cast<float4*>(DQ + (size_t)i * D + 4 * eq),
+                make_float4(aq[a][0], aq[a][1], aq[a][2], aq[a][3]));
+    }
+  }
+}
+
 // dqk_i += (dk_hat_i - k_hat_i (k_hat_i . dk_hat_i)) / ||qk_i||
 template <typename T>
 __global__ void __launch_bounds__(kThreads)
@@ -300,6 +494,19 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
   bwd_prep_kernel<T><<<row_blocks, kThreads, 0, st>>>(
       static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d);
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
+  if (p.c == tiled::C && p.d == tiled::D) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_pairs_tiled_kernel<T>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)tiled::kSmem);
+    if (e != cudaSuccess) return e;
+    bwd_pairs_tiled_kernel<T><<<grid, tiled::kTileThreads, tiled::kSmem, st>>>(
+        static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
+        static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.n_h, p.causal ? 1 : 0,
+        1.0f / sqrtf((float)p.d));
+    bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm,
+                                                          dkh, dqk, rows, p.d);
+    return cudaGetLastError();
+  }
   const size_t base = (size_t)kWarps * 2 * p.d * sizeof(float);
   const size_t staged = base + (size_t)4 * 2 * p.c * (p.d + 1) * sizeof(float) +
                         (size_t)2 * p.c * sizeof(int);

@@ -529,6 +529,11 @@ BWD = [
     W.small("bwd-bf16-noncausal-d128", heads=1, seq_len=256, d_k=128, n_hashes=3,
             n_buckets=16, chunk_len=32, causal=False),
     W.small("bwd-bf16-causal-short-chunk", heads=2, seq_len=300, n_hashes=2, n_buckets=16),
+    # c = 64, d = 64 take the register-tiled kernel: several (batch, head)
+    # pairs without the causal mask, and one short chunk alone
+    W.small("bwd-bf16-noncausal-tiled", batch=2, heads=2, seq_len=512, n_hashes=4,
+            n_buckets=16, causal=False),
+    W.small("bwd-bf16-one-short-chunk", heads=1, seq_len=40, n_hashes=2, n_buckets=4),
     # windows too large to stage: sums in shared memory (c = 128, d = 64), and
     # straight float32 atomics (c = 128, d = 128)
     W.small("bwd-bf16-c128-d64", heads=1, seq_len=512, n_hashes=2, n_buckets=8,
