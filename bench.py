@@ -63,6 +63,24 @@ def peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
+def window_pairs(wl):
+    """(query, key) pairs of every window: per (batch, head) and round, chunk
+    k's n_q queries meet the n_w keys of chunks k-1 and k (the first chunk
+    only itself; the last chunk may be short)."""
+    L, c = wl.seq_len, wl.chunk_len
+    per_round = 0
+    for k in range(-(-L // c)):
+        nq = min(c, L - k * c)
+        nw = min((k + 1) * c, L) - (k - 1) * c if k > 0 else nq
+        per_round += nq * nw
+    return wl.batch * wl.heads * wl.n_hashes * per_round
+
+
+# fp32 lanes per SM of a B200 (4 partitions x 32) for the CUDA-core roofline
+FP32_LANES_PER_SM = 128
+N_SMS = 148
+
+
 def stage_model(wl):
     """Algorithmic bytes (HBM) and FLOPs per launch of each stage."""
     BH, L, d, n_h, half, c = wl.batch * wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, \
@@ -322,15 +340,30 @@ def run_backward(args, wl):
         clocks.stop()
     lsh.lsh_attn_device_check()
     ms_per_step = ms / args.steps
+    clk = clocks.summary()
+    # Algorithmic work: five d-long products per window pair (S, dP, dV, dK_hat,
+    # dQ), 2 FLOPs per multiply-add, against the fp32 CUDA-core rate at the
+    # clock the samples saw (nominal maximum when none were taken).
+    flops = 10.0 * wl.d_k * window_pairs(wl)
+    mhz = clk.get("sm_max_mhz") or 1965.0
+    peak = N_SMS * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+    achieved = flops / (ms_per_step / 1e3) / 1e12
     print(json.dumps({
-        "metric": METRIC, "value": wl.tokens / (ms_per_step / 1e3), "unit": UNIT, "n_gpus": 1,
+        "metric": "LSH-attention bwd tokens/s (d qk, d v; hash and sort held fixed)",
+        "value": wl.tokens / (ms_per_step / 1e3), "unit": UNIT, "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f32 (gradients)", "data": "synthetic",
         "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
                        variant="backward: d qk, d v of out with the hash and sort held fixed "
-                               "(CUDA cores, float32 atomics)"),
-        "clocks": clocks.summary(), "gpu_launches": 3 * args.steps}), flush=True)
+                               "(CUDA cores: register tiles for c = 64, d = 64, else a warp "
+                               "per query; float32 atomics)"),
+        "roofline": {"kernel": "backward pairs", "bound": "alu", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{N_SMS} SMs x {FP32_LANES_PER_SM} fp32 lanes x 2 FLOPs x "
+                                    f"{mhz:.0f} MHz (unit counts and clock, not measured)",
+                     "algorithmic_flops": flops, "window_pairs": window_pairs(wl)},
+        "clocks": clk, "gpu_launches": 3 * args.steps}), flush=True)
     return 0
 
 
