@@ -230,26 +230,31 @@ def max_over_ranks(x, world):
 
 
 # ---------------------------------------------------------- CPU baseline --
-def oracle_sample(wl, rounds):
-    """Time the oracle (as it stands) on one (batch, head) and ``rounds`` hashing
-    rounds of the workload: hash, sort, chunked attention, combine.  Returns
-    (seconds, tokens-equivalent of the full workload processed)."""
+def oracle_sample(wl, rounds, heads=1, inputs=None):
+    """Time the oracle (as it stands) on the first ``heads`` (batch, head)
+    pairs and ``rounds`` hashing rounds of each: hash, sort, chunked
+    attention, combine.  Returns (seconds, tokens-equivalent of the full
+    workload processed)."""
     import numpy as np
     from oracle import lsh_oracle as O
-    qk, v, rot = W.make_inputs(wl)
-    x = O.as_f64(qk[0, 0])
-    vv = O.as_f64(v[0, 0])
+    qk, v, rot = W.make_inputs(wl) if inputs is None else inputs
+    rounds = min(rounds, wl.n_hashes)
+    heads = min(heads, wl.batch * wl.heads)
     R = O.as_f64(rot[:rounds]) if rot is not None else None
-    t0 = time.perf_counter()
-    b, _ = O.hash_head(x, R, wl.n_buckets)
-    perm, _ = O.sort_head(b)
-    o = np.empty((rounds, wl.seq_len, wl.d_k))
-    lse = np.empty((rounds, wl.seq_len))
-    for r in range(rounds):
-        o[r], lse[r] = O.attend_round(x, vv, perm[r], wl.chunk_len, wl.causal)
-    O.combine_head(o, lse)
-    dt = time.perf_counter() - t0
-    frac = rounds / (wl.n_hashes * wl.batch * wl.heads)  # share of the whole workload
+    dt = 0.0
+    for h in range(heads):
+        x = O.as_f64(qk.reshape(-1, wl.seq_len, wl.d_k)[h])
+        vv = O.as_f64(v.reshape(-1, wl.seq_len, wl.d_k)[h])
+        t0 = time.perf_counter()
+        b, _ = O.hash_head(x, R, wl.n_buckets)
+        perm, _ = O.sort_head(b)
+        o = np.empty((rounds, wl.seq_len, wl.d_k))
+        lse = np.empty((rounds, wl.seq_len))
+        for r in range(rounds):
+            o[r], lse[r] = O.attend_round(x, vv, perm[r], wl.chunk_len, wl.causal)
+        O.combine_head(o, lse)
+        dt += time.perf_counter() - t0
+    frac = heads * rounds / (wl.n_hashes * wl.batch * wl.heads)  # share of the workload
     return dt, wl.tokens * frac
 
 
@@ -263,12 +268,15 @@ def cpu_threads():
     return int(n)
 
 
-def cpu_baseline(wl, rounds):
-    dt, toks = oracle_sample(wl, rounds)
+def cpu_baseline(wl, rounds, heads):
+    rounds = min(rounds, wl.n_hashes)
+    heads = min(heads, wl.batch * wl.heads)
+    dt, toks = oracle_sample(wl, rounds, heads)
     return {"value": toks / dt, "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
-            "sample": f"one (batch, head) of {wl.name}, {rounds} of {wl.n_hashes} hashing "
-                      f"rounds, full length: hash, sort, chunked attention, combine in "
-                      f"float64 numpy; {dt:.2f} s, scaled to the whole workload",
+            "sample": f"{heads} of {wl.batch * wl.heads} (batch, head) pairs of {wl.name}, "
+                      f"{rounds} of {wl.n_hashes} hashing rounds each, full length: hash, sort, "
+                      f"chunked attention, combine in float64 numpy; {dt:.2f} s, scaled to "
+                      f"the whole workload",
             "seconds": dt, "host_cpus": len(os.sched_getaffinity(0))}
 
 
@@ -422,8 +430,11 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=W.HEADLINE.name, choices=list(W.BY_NAME))
-    ap.add_argument("--cpu-rounds", type=int, default=2,
-                    help="hashing rounds of one head the CPU baseline times")
+    ap.add_argument("--cpu-rounds", type=int, default=8,
+                    help="hashing rounds of each sampled head the CPU baseline times")
+    ap.add_argument("--cpu-heads", type=int, default=2,
+                    help="(batch, head) pairs the CPU baseline times (about 10 s on 16 "
+                         "threads for the long-text workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dedup", action="store_true",
                     help="the pass with the duplicate-count correction (CUDA-core attention); "
@@ -570,7 +581,7 @@ def main(argv=None):
     cpu = None
     variant = args.dedup or args.bucket_mask or args.kmeans
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
-        cpu = cpu_baseline(wl, args.cpu_rounds)
+        cpu = cpu_baseline(wl, args.cpu_rounds, args.cpu_heads)
 
     if rank == 0:
         line = {
