@@ -437,14 +437,14 @@ def main(argv=None):
                          "threads for the long-text workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--dedup", action="store_true",
-                    help="the pass with the duplicate-count correction (CUDA-core attention); "
-                         "a separate measurement, not the headline")
+                    help="the pass with the duplicate-count correction; a separate "
+                         "measurement, not the headline")
     ap.add_argument("--bucket-mask", action="store_true",
-                    help="the pass with the bucket-equality mask (CUDA-core attention); a "
-                         "separate measurement, not the headline")
+                    help="the pass with the bucket-equality mask; a separate measurement, not "
+                         "the headline")
     ap.add_argument("--kmeans", action="store_true",
-                    help="routing-style assignment to n_buckets centroids (CUDA-core hash) "
-                         "instead of the random-rotation hash; a separate measurement")
+                    help="routing-style assignment to n_buckets centroids instead of the "
+                         "random-rotation hash; a separate measurement")
     ap.add_argument("--backward", action="store_true",
                     help="time the backward pass (hash and sort fixed) on the workload; a "
                          "separate measurement, not the headline")
