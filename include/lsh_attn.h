@@ -18,8 +18,11 @@
  * --------------------------------
  *  - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent)
  *    unless the name ends in _host.  The caller owns every buffer, including
- *    the workspace; the library never allocates, frees or keeps a pointer
- *    after a call returns.
+ *    the workspace, and the library keeps no pointer after a call returns.
+ *    The library allocates nothing for the caller's data; the three places
+ *    where it holds device resources of its own are stated at their calls:
+ *    lsh_attn_sort's scratch pool, lsh_attn_forward_host's streams and
+ *    events, and lsh_attn_forward_noalloc's built-in scratch.
  *  - Every device pointer must be 16-byte aligned.  Tensors are dense,
  *    row-major, last dimension fastest.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
@@ -31,8 +34,9 @@
  *    has the CUDA message).
  *  - Shapes (see lsh_shape): B batch, H heads, L seq_len, d d_k,
  *    n_h n_hashes, n_b n_buckets, c chunk_len.
- *  - The library keeps no state between calls except one device word that
- *    records a kernel's bounded wait running out (see lsh_attn_device_check).
+ *  - Besides those resources, the library keeps no state between calls
+ *    except one device word that records a kernel's bounded wait running out
+ *    (see lsh_attn_device_check).
  */
 #ifndef LSH_ATTN_H_
 #define LSH_ATTN_H_
@@ -72,22 +76,26 @@ typedef enum lsh_dtype {
                                   cross-checking the two kernel families   */
 #define LSH_FLAG_DEDUP 2u      /* duplicate-count correction ("Reformer: The
                                   Efficient Transformer", Appendix A "Multi-
-                                  round LSH attention"): a key that falls in
-                                  a query's window in N rounds has log N
+                                  round LSH attention", its "Duplicate
+                                  handling" item): a key that falls in a
+                                  query's window in N rounds has log N
                                   subtracted from its score in each of them,
                                   so the combined output weighs every
                                   distinct key once.  N counts the rounds r
                                   with chunk(undo_r[i]) - chunk(undo_r[j]) in
-                                  {0, 1}.  Runs on the CUDA-core attention
-                                  kernel; the stage call is
-                                  lsh_attn_chunked_fwd_ex.                 */
+                                  {0, 1}.  Runs on the tensor-core attention
+                                  for n_h <= 8 where it has a plan for the
+                                  (c, d) pair, else on the CUDA-core kernel;
+                                  the stage call is lsh_attn_chunked_fwd_ex. */
 #define LSH_FLAG_BUCKET_MASK 4u /* bucket-equality mask (section 2 "LSH
                                   attention": a query attends only to
                                   targets in its own hash bucket): inside a
                                   window, keys whose bucket in that round
                                   differs from the query's are not attended.
-                                  Runs on the CUDA-core attention kernel;
-                                  the stage call is lsh_attn_chunked_fwd_ex. */
+                                  Runs on the tensor-core attention (on the
+                                  CUDA-core kernel together with
+                                  LSH_FLAG_DEDUP); the stage call is
+                                  lsh_attn_chunked_fwd_ex.                 */
 #define LSH_FLAG_KMEANS 8u     /* routing-style bucket assignment (the pages
                                   name online k-means for the Routing
                                   Transformer): `rotations` holds centroids
@@ -106,7 +114,8 @@ typedef struct lsh_shape {
   int32_t seq_len;     /* L >= 1, < 2^31 / n_h                                */
   int32_t d_k;         /* d: 8..256, a multiple of 8                         */
   int32_t n_hashes;    /* n_h >= 1 hashing rounds                            */
-  int32_t n_buckets;   /* n_b: 1, or even with 2 <= n_b <= 32768             */
+  int32_t n_buckets;   /* n_b: 1, or even with 2 <= n_b <= 32768; any value
+                          in [2, 32768] with LSH_FLAG_KMEANS                 */
   int32_t chunk_len;   /* c >= 1; when c does not divide L the last chunk of
                           the sorted order holds the L mod c remaining slots */
   int32_t causal;      /* 0 or 1                                             */
