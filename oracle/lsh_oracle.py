@@ -51,6 +51,13 @@ Readings where the pages are silent (each is also listed in the design notes):
   * the duplicate-count correction of Appendix A is off unless asked for
     (``dedup=True`` subtracts log N_ij, N_ij = number of rounds whose window
     of query i contains key j).
+
+Parity unpinned (by the pages): the self score -1e5, the 1/sqrt(d_k) scale,
+the first chunk's missing look-back and the absence of a bucket mask are
+readings, not facts the pages state; the tests fix them only through
+hand-worked fixtures and brute forces that take the same readings.  Every
+function here is otherwise pinned by tests that do not reuse its code
+(closed forms, brute force, invariants, finite differences).
 """
 
 from __future__ import annotations
