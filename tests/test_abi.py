@@ -139,3 +139,60 @@ def test_binding_checks_host_tensor_shapes_before_any_copy():
     km = lsh.make_shape(1, 2, 128, 64, 2, 16, 64, True, torch.bfloat16, kmeans=True)
     with pytest.raises(ValueError, match="rot_host"):  # centroids are [n_h, d, n_b]
         lsh.lsh_attn_forward_host(km, x, x, rot, x, lse, "not a tensor")
+
+
+def _flags(shp, flags):
+    shp.flags = flags
+    return shp
+
+
+def test_backward_validates_before_launching(L):
+    shp = shape()
+    need = lsh.lsh_attn_backward_workspace_size(shp)
+    assert need >= 2 * 256 * (4 + 64 * 4)  # delta and dk_hat, float32
+
+    def bwd(s=shp, ws=FAKE, ws_bytes=need, dout=FAKE):
+        return L.lsh_attn_backward(ctypes.byref(s), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, dout,
+                                   FAKE, FAKE, ws, ws_bytes, STREAM)
+    assert bwd(s=_flags(shape(), lsh.FLAG_DEDUP)) == 2          # variants: unsupported
+    assert bwd(dout=None) == 1
+    assert bwd(ws=ctypes.c_void_p((1 << 20) + 16)) == 1          # not 256-aligned
+    assert bwd(ws_bytes=need - 1) == 3
+
+
+def test_variant_stage_call_needs_its_inputs(L):
+    ded = _flags(shape(), lsh.FLAG_DEDUP)
+    msk = _flags(shape(), lsh.FLAG_BUCKET_MASK)
+    # the plain stage call refuses variant flags
+    assert L.lsh_attn_chunked_fwd(ctypes.byref(ded), FAKE, FAKE, FAKE, FAKE, FAKE, FAKE,
+                                  STREAM) == 1
+    assert b"_ex" in L.lsh_attn_last_error()
+    # the _ex call needs undo for the correction and buckets for the mask
+    assert L.lsh_attn_chunked_fwd_ex(ctypes.byref(ded), FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                                     FAKE, STREAM) == 1
+    assert L.lsh_attn_chunked_fwd_ex(ctypes.byref(msk), FAKE, FAKE, FAKE, FAKE, None, None, FAKE,
+                                     FAKE, STREAM) == 1
+
+
+def test_host_entry_point_validates_before_any_copy(L):
+    shp = shape()
+    need = lsh.lsh_attn_forward_host_device_bytes(shp)
+
+    def host(qk=FAKE, rot=FAKE, dev=FAKE, n=need, s=shp):
+        return L.lsh_attn_forward_host(ctypes.byref(s), qk, FAKE, rot, FAKE, FAKE, dev, n, STREAM)
+    assert host(qk=None) == 1
+    assert host(rot=None) == 1                                    # n_b > 1 needs rotations
+    assert host(s=shape(n_buckets=1)) == 1                        # n_b == 1 forbids them
+    assert host(dev=ctypes.c_void_p((1 << 20) + 16)) == 1         # not 256-aligned
+    assert host(n=need - 1) == 3
+
+
+def test_kmeans_takes_any_bucket_count_from_two(L):
+    n = ctypes.c_size_t()
+    for nb, ok in [(7, True), (2, True), (32768, True), (1, False), (32769, False)]:
+        shp = _flags(shape(n_buckets=nb), lsh.FLAG_KMEANS)
+        st = L.lsh_attn_forward_workspace_size(ctypes.byref(shp), ctypes.byref(n))
+        assert (st == 0) == ok, nb
+    # without the flag an odd count is refused
+    assert L.lsh_attn_forward_workspace_size(ctypes.byref(shape(n_buckets=7)),
+                                             ctypes.byref(n)) == 1
