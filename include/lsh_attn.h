@@ -280,10 +280,15 @@ LSH_ATTN_API lsh_status lsh_attn_forward_host(const lsh_shape* shape, const void
  * take an unpredictable time.  Same arguments and results as
  * lsh_attn_forward, minus the workspace: the intermediates live in a scratch
  * array of LSH_ATTN_NOALLOC_SCRATCH_BYTES built into the library.
- *  - The scratch occupies that much device memory on every GPU where this
- *    call has run, from the first call there until the process exits.
- *  - The first call on a device resolves the scratch's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
+ *  - The scratch occupies that much device memory on every GPU whose
+ *    context has loaded the library's device code, until the process exits.
+ *    Under lazy module loading (CUDA's default, CUDA_MODULE_LOADING=LAZY)
+ *    that is the GPUs where this call has run, from its first call there;
+ *    with CUDA_MODULE_LOADING=EAGER it is every GPU on which the process
+ *    creates a context once the library is loaded.
+ *  - The first successful call on a device resolves the scratch's device
+ *    address (cudaGetSymbolAddress) with that device current and keeps it;
+ *    a failed lookup is retried on the next call.  Make that first call
  *    before any stream capture.
  *  - Problems whose workspace (lsh_attn_forward_workspace_size) exceeds
  *    LSH_ATTN_NOALLOC_SCRATCH_BYTES are rejected with LSH_ERR_WORKSPACE
@@ -315,6 +320,12 @@ LSH_ATTN_API const char* lsh_attn_status_string(lsh_status status);
 LSH_ATTN_API const char* lsh_attn_last_error(void);
 LSH_ATTN_API lsh_status lsh_attn_device_check(void* stream);
 LSH_ATTN_API int lsh_attn_version(void);
+
+/* Number of CUDA kernels this library has launched in this process so far
+ * (every stage, variant and entry point; host-side count taken at launch).
+ * A diagnostic for benchmarks that report how many of their kernels ran in a
+ * timed region: read it before and after.  Thread-safe; never reset. */
+LSH_ATTN_API unsigned long long lsh_attn_kernel_launches(void);
 
 #ifdef __cplusplus
 }

@@ -24,7 +24,7 @@ __all__ = [
     "lsh_attn_chunked_fwd", "lsh_attn_chunked_fwd_ex", "lsh_attn_combine", "lsh_attn_forward",
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
     "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
-    "lsh_attn_backward", "lsh_attn_backward_workspace_size",
+    "lsh_attn_backward", "lsh_attn_backward_workspace_size", "lsh_attn_kernel_launches",
     "LIB_PATH", "HEADER_PATH", "NOALLOC_SCRATCH_BYTES",
     "F32", "BF16", "FLAG_PORTABLE", "FLAG_DEDUP", "FLAG_BUCKET_MASK", "FLAG_KMEANS",
 ]
@@ -78,6 +78,7 @@ _SIGS = {
     "lsh_attn_last_error": [],
     "lsh_attn_device_check": [_P],
     "lsh_attn_version": [],
+    "lsh_attn_kernel_launches": [],
 }
 
 
@@ -95,6 +96,7 @@ def lib() -> ctypes.CDLL:
             fn.restype = ctypes.c_int
         L.lsh_attn_status_string.restype = ctypes.c_char_p
         L.lsh_attn_last_error.restype = ctypes.c_char_p
+        L.lsh_attn_kernel_launches.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -379,6 +381,11 @@ def lsh_attn_forward_noalloc(qk, v, rotations, n_hashes, n_buckets, chunk_len, c
     _check(lib().lsh_attn_forward_noalloc(ctypes.byref(shp), _ptr(qk), _ptr(v), _ptr(rotations),
                                           _ptr(out), _ptr(lse), _stream(stream)))
     return out, lse
+
+
+def lsh_attn_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far (host count)."""
+    return int(lib().lsh_attn_kernel_launches())
 
 
 def lsh_attn_device_check(stream=None):

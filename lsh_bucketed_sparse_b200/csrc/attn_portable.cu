@@ -135,6 +135,7 @@ cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v
     attn_portable_kernel<float><<<grid, kWarps * 32, smem, st>>>(
         (const float*)qk, (const float*)v, inv_norm, perm, undo, buckets, (float*)o_rounds, lse_rounds, p.L,
         p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
+  note_launch();
   return cudaGetLastError();
 }
 

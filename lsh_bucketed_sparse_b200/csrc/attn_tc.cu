@@ -200,7 +200,9 @@ __device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, int u_st
 
 // Positions of sorted slots sl .. sl+3 of a segment (INT_MAX past its end).
 __device__ __forceinline__ void load_positions(const int32_t* perm, int sl, int L, int* pos) {
-  if (sl + 3 < L) {
+  // one 16-byte load where the four positions are 16-byte aligned (a segment
+  // starts on such a boundary only when L is a multiple of 4)
+  if (sl + 3 < L && (reinterpret_cast<uintptr_t>(perm + sl) & 15) == 0) {
     const int4 v = *reinterpret_cast<const int4*>(perm + sl);
     pos[0] = v.x; pos[1] = v.y; pos[2] = v.z; pos[3] = v.w;
   } else {
@@ -920,7 +922,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], p);
+  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], p); note_launch();
   return cudaGetLastError();
 }
 

@@ -492,7 +492,7 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
   const long long rows = (long long)p.BH() * p.L;
   const unsigned row_blocks = (unsigned)((rows * 32 + kThreads - 1) / kThreads);
   bwd_prep_kernel<T><<<row_blocks, kThreads, 0, st>>>(
-      static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d);
+      static_cast<const T*>(out), static_cast<const T*>(dout), delta, dqk, dv, dkh, rows, p.d); note_launch();
   const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
   if (p.c == tiled::C && p.d == tiled::D) {
     cudaError_t e = cudaFuncSetAttribute(bwd_pairs_tiled_kernel<T>,
@@ -502,9 +502,9 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
     bwd_pairs_tiled_kernel<T><<<grid, tiled::kTileThreads, tiled::kSmem, st>>>(
         static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
         static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.n_h, p.causal ? 1 : 0,
-        1.0f / sqrtf((float)p.d));
+        1.0f / sqrtf((float)p.d)); note_launch();
     bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm,
-                                                          dkh, dqk, rows, p.d);
+                                                          dkh, dqk, rows, p.d); note_launch();
     return cudaGetLastError();
   }
   const size_t base = (size_t)kWarps * 2 * p.d * sizeof(float);
@@ -518,9 +518,9 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
     bwd_pairs_staged_kernel<T><<<grid, kWarps * 32, staged, st>>>(
         static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
         static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.d, p.n_h, p.c,
-        p.causal ? 1 : 0, 1.0f / sqrtf((float)p.d));
+        p.causal ? 1 : 0, 1.0f / sqrtf((float)p.d)); note_launch();
     bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm,
-                                                          dkh, dqk, rows, p.d);
+                                                          dkh, dqk, rows, p.d); note_launch();
     return cudaGetLastError();
   }
   const size_t acc = (size_t)2 * (2 * (size_t)p.c) * p.d * sizeof(float);
@@ -535,9 +535,9 @@ cudaError_t launch_t(const Problem& p, const void* qk, const void* v, const floa
   kernel<<<grid, kWarps * 32, smem, st>>>(
       static_cast<const T*>(qk), static_cast<const T*>(v), inv_norm, perm, lse,
       static_cast<const T*>(dout), delta, dqk, dv, dkh, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0,
-      1.0f / sqrtf((float)p.d));
+      1.0f / sqrtf((float)p.d)); note_launch();
   bwd_finish_kernel<T><<<row_blocks, kThreads, 0, st>>>(static_cast<const T*>(qk), inv_norm, dkh,
-                                                        dqk, rows, p.d);
+                                                        dqk, rows, p.d); note_launch();
   return cudaGetLastError();
 }
 

@@ -127,12 +127,12 @@ void launch_t(const Problem& p, const void* o_rounds, const float* lse_rounds, v
   const T* o = static_cast<const T*>(o_rounds);
   T* y = static_cast<T*>(out);
   switch (p.n_h) {
-    case 1: combine_kernel<T, 1><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 1); break;
-    case 2: combine_kernel<T, 2><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 2); break;
-    case 4: combine_kernel<T, 4><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 4); break;
-    case 8: combine_kernel<T, 8><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 8); break;
+    case 1: combine_kernel<T, 1><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 1); note_launch(); break;
+    case 2: combine_kernel<T, 2><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 2); note_launch(); break;
+    case 4: combine_kernel<T, 4><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 4); note_launch(); break;
+    case 8: combine_kernel<T, 8><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 8); note_launch(); break;
     default:
-      combine_kernel<T, 0><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, p.n_h);
+      combine_kernel<T, 0><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, p.n_h); note_launch();
   }
 }
 

@@ -21,30 +21,33 @@ namespace {
 constexpr size_t kScratchBytes = (size_t)LSH_ATTN_NOALLOC_SCRATCH_BYTES;
 constexpr int kMaxDevices = 64;
 
-// The scratch lives in device memory of every GPU on which this library's
-// no-allocation entry point has run, from its first call there until the
-// process exits.  In host code `g_noalloc_scratch` names a host-side stand-in,
+// The scratch lives in device memory of every GPU whose context has loaded
+// this library's device code, until the process exits.  Under lazy module
+// loading (CUDA's default, CUDA_MODULE_LOADING=LAZY) that is the GPUs on
+// which a kernel of this translation unit's module has been needed, i.e.
+// where this entry point has run; with CUDA_MODULE_LOADING=EAGER it is every
+// GPU on which the process creates a context after loading the library.  In host code `g_noalloc_scratch` names a host-side stand-in,
 // not a device address: the device address comes from cudaGetSymbolAddress.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kScratchBytes];
 
-std::once_flag g_once[kMaxDevices];
-void* g_scratch[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_mutex;
+void* g_scratch[kMaxDevices];  // non-null once resolved on that device
 
-// Device address of the scratch on the current device, resolved once per
-// device with that device current.
+// Device address of the scratch on the current device, looked up with that
+// device current.  Only a successful lookup is kept: a failed one (say, a
+// transient error) is tried again on the next call.
 lsh_status scratch_for_current_device(void** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= kMaxDevices) return fail(LSH_ERR_UNSUPPORTED, "device %d", dev);
-  std::call_once(g_once[dev], [dev] {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (!g_scratch[dev]) {
     void* ptr = nullptr;
-    g_scratch_err[dev] = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-    g_scratch[dev] = g_scratch_err[dev] == cudaSuccess ? ptr : nullptr;
-  });
-  if (g_scratch_err[dev] != cudaSuccess)
-    return cuda_fail(g_scratch_err[dev], "cudaGetSymbolAddress(no-allocation scratch)");
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-allocation scratch)");
+    g_scratch[dev] = ptr;
+  }
   *out = g_scratch[dev];
   return LSH_OK;
 }

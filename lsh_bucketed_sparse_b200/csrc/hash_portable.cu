@@ -99,6 +99,7 @@ cudaError_t launch_hash_portable(const Problem& p, const void* qk, const void* r
     hash_portable_kernel<float><<<(unsigned)blocks, kWarps * 32, smem, st>>>(
         (const float*)qk, (const float*)rot, buckets, inv_norm, p.BH(), p.L, p.d, p.n_h,
         p.kmeans ? 0 : p.half(), p.kmeans ? p.n_b : 0);
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -580,7 +580,7 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
   if (e != cudaSuccess) return e;
-  kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p);
+  kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p); note_launch();
   return cudaGetLastError();
 }
 

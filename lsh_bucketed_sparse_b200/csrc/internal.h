@@ -51,6 +51,10 @@ cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
                             const float* lse, const void* dout, float* dqk, float* dv,
                             void* workspace, cudaStream_t st);
 
+// Counts one kernel launch of this library (every launch site calls it right
+// after its <<<...>>>); read through lsh_attn_kernel_launches().
+void note_launch();
+
 // Address of the device word that kernels set when a bounded wait runs out.
 // Resolved for the current device (cudaGetSymbolAddress); nullptr on error.
 unsigned int* device_error_word();
@@ -75,6 +79,12 @@ cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v
                                  const float* inv_norm, const int32_t* perm,
                                  const int32_t* undo, const int16_t* buckets, void* o_rounds,
                                  float* lse_rounds, cudaStream_t st);
+// chunks of 64 with d_k = 64 (bf16): P kept in tensor memory
+bool attn_tc64_supported(const Problem& p);
+cudaError_t launch_attn_tc64(const Problem& p, const void* qk, const void* v,
+                             const float* inv_norm, const int32_t* perm, const int16_t* buckets,
+                             const int32_t* undo, void* o_rounds, float* lse_rounds,
+                             cudaStream_t st);
 bool attn_tc_supported(const Problem& p);
 cudaError_t launch_attn_tc(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                            const int32_t* perm, const int16_t* buckets, const int32_t* undo,

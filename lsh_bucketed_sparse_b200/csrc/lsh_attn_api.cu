@@ -5,6 +5,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "internal.h"
@@ -18,7 +19,10 @@ __device__ unsigned int g_device_error_word = 0;
 
 namespace {
 thread_local char g_last_error[512] = "";
+std::atomic<unsigned long long> g_launches{0};
 }  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 lsh_status fail(lsh_status st, const char* fmt, ...) {
   va_list ap;
@@ -125,10 +129,11 @@ lsh_status run_sort(const Problem& p, const int16_t* buckets, int32_t* perm, int
 lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float* inv_norm,
                     const int32_t* perm, const int32_t* undo, const int16_t* buckets,
                     void* o_r, float* lse_r, cudaStream_t st) {
-  const bool tc = !p.portable && attn_tc_supported(p) &&
-                  !(p.dedup && (p.bucket_mask || p.n_h > 8));
-  cudaError_t e = tc ? launch_attn_tc(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st)
-                     : cudaErrorNotSupported;
+  cudaError_t e = cudaErrorNotSupported;
+  if (!p.portable && attn_tc64_supported(p))
+    e = launch_attn_tc64(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st);
+  else if (!p.portable && attn_tc_supported(p) && !(p.dedup && (p.bucket_mask || p.n_h > 8)))
+    e = launch_attn_tc(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st);
   if (e == cudaErrorNotSupported)  // a shape the tensor-core kernel does not plan for
     e = launch_attn_portable(p, qk, v, inv_norm, perm, undo, buckets, o_r, lse_r, st);
   return e == cudaSuccess ? LSH_OK : cuda_fail(e, "chunked attention launch");
@@ -604,5 +609,9 @@ lsh_status lsh_attn_device_check(void* stream) {
 }
 
 int lsh_attn_version(void) { return LSH_ATTN_VERSION; }
+
+unsigned long long lsh_attn_kernel_launches(void) {
+  return g_launches.load(std::memory_order_relaxed);
+}
 
 }  // extern "C"

@@ -197,10 +197,10 @@ cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes)))
       return e;
   }
-  sort_count_kernel<<<dim3(segs, T), kCountThreads, hist_bytes, st>>>(buckets, cnt, p.L, n_b, T);
-  sort_scan_kernel<<<segs, kScanThreads, hist_bytes, st>>>(cnt, counts, n_b, T);
+  sort_count_kernel<<<dim3(segs, T), kCountThreads, hist_bytes, st>>>(buckets, cnt, p.L, n_b, T); note_launch();
+  sort_scan_kernel<<<segs, kScanThreads, hist_bytes, st>>>(cnt, counts, n_b, T); note_launch();
   sort_scatter_kernel<<<dim3(segs, T), 32, hist_bytes, st>>>(buckets, cnt, perm, undo, p.L, n_b,
-                                                              T);
+                                                              T); note_launch();
   return cudaGetLastError();
 }
 
