@@ -9,11 +9,17 @@ combine) over one batch of the workload, with inputs resident in HBM.  The
 default workload is the long-text shape: batch 1 x 8 heads, L = 65536,
 d_k = 64, bf16, 8 hashes, 1024 buckets, chunks of 64, causal.  Inputs are
 seeded synthetic N(0, 1) data.  L2 is flushed (a 256 MiB write) before every
-timed step; each step is timed with CUDA events on the launching stream.
+timed step; each step is timed with CUDA events on the launching stream.  At
+one GPU the line also carries `per_workload`: every named workload timed the
+same way (tokens/s, stage times, roofline fractions).
 
-Multi-GPU: one process per GPU (torchrun), each rank runs the same workload on
-its own GPU -- (batch, head) pairs are independent, so there is no collective
-on the data path ("scaling": "weak"); the time is the max over ranks.
+Multi-GPU: `--gpus N` (N > 1) started without torchrun re-launches itself
+under torch.distributed.run with N local ranks, one per GPU.  The job is an
+N-times larger batch of (batch, head) problems: rank r owns the r-th slice of
+batch*heads pairs (the headline workload's shape, its own seeded inputs).
+Hashing, sorting, the windows and the combine never cross heads, so there is
+no collective on the data path ("scaling": "weak"); the NCCL process group
+carries only the barriers and the max-over-ranks of the timings.
 
 Prints ONE JSON line on rank 0.
 """
@@ -42,6 +48,9 @@ METRIC = "LSH-attention fwd tokens/s at L=65536, 8 hashes; % of HBM/tensor roofl
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (HGX: 8 TB/s HBM3e, 2.25 PFLOP/s dense bf16); every
+# fraction is also reported against these.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 KERNEL_SOURCES = {
     "hash": ["hash_tc.cu", "hash_portable.cu"],
     "sort": ["sort.cu"],
@@ -202,6 +211,19 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------ distributed --
+def launch_ranks(args, argv):
+    """`--gpus N` without torchrun: run this script under torch.distributed.run
+    with N local ranks (rendezvous on 127.0.0.1) and return its exit code."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={args.gpus}", "--master-addr=127.0.0.1",
+           f"--master-port={port}", os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd)
+
+
 def dist_setup():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -209,9 +231,22 @@ def dist_setup():
     if world > 1:
         import torch.distributed as dist
         torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     return rank, world, local
+
+
+def rank_inputs(wl, rank, world, kmeans=False):
+    """Host inputs of this rank's (batch, head) slice: the headline shape,
+    seeded per rank (rank 0 gets the workload's own seed)."""
+    from lsh_bucketed_sparse_b200 import sharding
+    a, b = sharding.head_range(wl.batch * world, wl.heads, rank, world)
+    assert b - a == wl.batch * wl.heads
+    seed = wl.seed + 7919 * rank
+    qk, v, rot = W.make_inputs(wl, seed=seed)
+    if kmeans:
+        rot = W.make_centroids(wl, seed=wl.seed)
+    return qk, v, rot
 
 
 def barrier(world):
@@ -422,8 +457,121 @@ def run_one_stage(args, wl):
     return 0
 
 
+# -------------------------------------------------------------- measuring --
+def step_fn(wl, qk, v, rot, dev, args):
+    """One fused forward (lsh_attn_forward) over device inputs, outputs and
+    workspace allocated here."""
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup,
+                         bucket_mask=args.bucket_mask, kmeans=args.kmeans)
+    ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
+    out = torch.empty_like(qk)
+    lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
+
+    def step():
+        lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
+                             workspace=ws, out=out, lse=lse, dedup=args.dedup,
+                             bucket_mask=args.bucket_mask, kmeans=args.kmeans)
+    return step, shp
+
+
+def stage_times(wl, qk, v, rot, stream, flush, n, args):
+    """Device time of each stage through the four stage calls (the same
+    kernels as the fused call), averaged over n passes after two warm-ups."""
+    stage_ms = {k: 0.0 for k in ("hash", "sort", "chunked_attention", "combine")}
+    for it in range(n + 2):
+        flush.fill_(2.0)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes, kmeans=args.kmeans)
+        ev[1].record(stream)
+        perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=args.dedup)
+        ev[2].record(stream)
+        if args.dedup or args.bucket_mask:
+            o_r, l_r = lsh.lsh_attn_chunked_fwd_ex(
+                qk, v, inv, perm, wl.chunk_len, wl.causal, undo=undo if args.dedup else None,
+                buckets=b if args.bucket_mask else None, n_buckets=wl.n_buckets)
+        else:
+            o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                                n_buckets=wl.n_buckets)
+        ev[3].record(stream)
+        lsh.lsh_attn_combine(o_r, l_r)
+        ev[4].record(stream)
+        torch.cuda.synchronize()
+        if it >= 2:
+            for j, k in enumerate(stage_ms):
+                stage_ms[k] += ev[j].elapsed_time(ev[j + 1]) / n
+        del b, inv, perm, undo, o_r, l_r
+    return stage_ms
+
+
+def roofline_of(wl, stage_ms, ms_per_step, pk):
+    """Roofline of the dominant stage (its algorithmic bytes or FLOPs over its
+    device time, against the measured or fallback peak and the nominal one)
+    and of the whole pass (max of bytes / HBM peak and FLOPs / tensor peak)."""
+    model = stage_model(wl)
+    dom = max(stage_ms, key=stage_ms.get)
+    sec = stage_ms[dom] / 1e3
+    m = model[dom]
+    if m["flops"] / (pk["bf16_tflops_sustained"] * 1e12) > m["bytes"] / (pk["hbm_gbs"] * 1e9):
+        achieved, peak, nominal, unit, bound = m["flops"] / sec / 1e12, \
+            pk["bf16_tflops_sustained"], NOMINAL_PEAKS["bf16_tflops"], "TFLOP/s", "tensor"
+    else:
+        achieved, peak, nominal, unit, bound = m["bytes"] / sec / 1e9, pk["hbm_gbs"], \
+            NOMINAL_PEAKS["hbm_gbs"], "GB/s", "hbm"
+    r = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
+         "frac": achieved / peak, "peak_source": pk["source"],
+         "peak_nominal": nominal, "frac_nominal": achieved / nominal,
+         "algorithmic_bytes": m["bytes"], "algorithmic_flops": m["flops"],
+         "stage_ms": stage_ms}
+    total_bytes = sum(x["bytes"] for x in model.values())
+    total_flops = sum(x["flops"] for x in model.values())
+    t_roof = max(total_bytes / (pk["hbm_gbs"] * 1e9), total_flops / (pk["bf16_tflops"] * 1e12))
+    t_nom = max(total_bytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9),
+                total_flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12))
+    r["pass_roofline_ms"] = t_roof * 1e3
+    r["pass_frac"] = t_roof * 1e3 / ms_per_step
+    r["pass_roofline_ms_nominal"] = t_nom * 1e3
+    r["pass_frac_nominal"] = t_nom * 1e3 / ms_per_step
+    return r
+
+
+def per_workload(dev, stream, flush, steps, args, pk):
+    """Every named workload on this GPU: the fused pass timed as the headline
+    (L2 flushed before each step, CUDA events), tokens/s, stage times and the
+    roofline fractions."""
+    rows = []
+    for wl in W.WORKLOADS:
+        qk_h, v_h, rot_h = W.make_inputs(wl)
+        qk, v = qk_h.to(dev), v_h.to(dev)
+        rot = rot_h.to(dev) if rot_h is not None else None
+        step, _ = step_fn(wl, qk, v, rot, dev, args)
+        for _ in range(3):
+            flush.fill_(1.0)
+            step()
+        ms = 0.0
+        for k in range(steps):
+            flush.fill_(float(k))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms += e0.elapsed_time(e1)
+        ms /= steps
+        st = stage_times(wl, qk, v, rot, stream, flush, min(steps, 5), args)
+        lsh.lsh_attn_device_check()
+        roof = roofline_of(wl, st, ms, pk)
+        rows.append({"workload": wl.name, "value": wl.tokens / (ms / 1e3), "unit": UNIT,
+                     "ms_per_step": ms, "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32",
+                     "config": wl.describe(), "roofline": roof})
+        del qk, v, rot, step
+    return rows
+
+
 # ----------------------------------------------------------------- main --
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=100)
@@ -436,6 +584,8 @@ def main(argv=None):
                     help="(batch, head) pairs the CPU baseline times (about 10 s on 16 "
                          "threads for the long-text workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the per-workload table of the one-GPU line")
     ap.add_argument("--dedup", action="store_true",
                     help="the pass with the duplicate-count correction; a separate "
                          "measurement, not the headline")
@@ -460,29 +610,25 @@ def main(argv=None):
         return run_backward(args, wl)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        return launch_ranks(args, argv)
+    if world_env is not None and int(world_env) != args.gpus:
+        print(f"bench.py: WORLD_SIZE={world_env} but --gpus {args.gpus}", file=sys.stderr)
+        return 2
 
     rank, world, local = dist_setup()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
-    qk_h, v_h, rot_h = W.make_inputs(wl)
-    if args.kmeans:
-        rot_h = W.make_centroids(wl)
+    qk_h, v_h, rot_h = rank_inputs(wl, rank, world, kmeans=args.kmeans)
     qk, v = qk_h.to(dev), v_h.to(dev)
     rot = rot_h.to(dev) if rot_h is not None else None
-    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
-                         wl.chunk_len, wl.causal, wl.dtype, dedup=args.dedup,
-                         bucket_mask=args.bucket_mask, kmeans=args.kmeans)
-    ws = torch.empty(lsh.lsh_attn_forward_workspace_size(shp), dtype=torch.uint8, device=dev)
-    out = torch.empty_like(qk)
-    lse = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32, device=dev)
+    step, shp = step_fn(wl, qk, v, rot, dev, args)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
-
-    def step():
-        lsh.lsh_attn_forward(qk, v, rot, wl.n_hashes, wl.n_buckets, wl.chunk_len, wl.causal,
-                             workspace=ws, out=out, lse=lse, dedup=args.dedup,
-                             bucket_mask=args.bucket_mask, kmeans=args.kmeans)
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -493,6 +639,7 @@ def main(argv=None):
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     barrier(world)
     torch.cuda.synchronize()
+    launches0 = lsh.lsh_attn_kernel_launches()
     with ClockSampler(local) as clocks:
         clocks.start()
         for k in range(args.steps):
@@ -502,6 +649,7 @@ def main(argv=None):
             ends[k].record(stream)
         torch.cuda.synchronize()
         clocks.stop()
+    launches = lsh.lsh_attn_kernel_launches() - launches0
     barrier(world)
     lsh.lsh_attn_device_check()
     ms_local = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
@@ -509,32 +657,7 @@ def main(argv=None):
     ms_per_step = ms_total / args.steps
     value = world * wl.tokens * args.steps / (ms_total / 1e3)
 
-    # Per-stage device time: the same kernels through the four stage calls.
-    stage_ms = {k: 0.0 for k in ("hash", "sort", "chunked_attention", "combine")}
-    n_stage = min(args.steps, 10)
-    for it in range(n_stage + 2):
-        flush.fill_(2.0)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
-        ev[0].record(stream)
-        b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes, kmeans=args.kmeans)
-        ev[1].record(stream)
-        perm, undo, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=args.dedup)
-        ev[2].record(stream)
-        if args.dedup or args.bucket_mask:
-            o_r, l_r = lsh.lsh_attn_chunked_fwd_ex(
-                qk, v, inv, perm, wl.chunk_len, wl.causal, undo=undo if args.dedup else None,
-                buckets=b if args.bucket_mask else None, n_buckets=wl.n_buckets)
-        else:
-            o_r, l_r = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
-                                                n_buckets=wl.n_buckets)
-        ev[3].record(stream)
-        lsh.lsh_attn_combine(o_r, l_r)
-        ev[4].record(stream)
-        torch.cuda.synchronize()
-        if it >= 2:
-            for j, k in enumerate(stage_ms):
-                stage_ms[k] += ev[j].elapsed_time(ev[j + 1]) / n_stage
-        del b, inv, perm, undo, o_r, l_r
+    stage_ms = stage_times(wl, qk, v, rot, stream, flush, min(args.steps, 10), args)
 
     # End to end through the host-buffer entry point: copies in and out timed.
     pin = [t.pin_memory() if t is not None else None for t in (qk_h, v_h, rot_h)]
@@ -555,31 +678,18 @@ def main(argv=None):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in pin if t is not None)
     d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
+    del pin, out_h, lse_h, dbuf
 
-    # Roofline of the dominant kernel.
     pk = peaks()
-    model = stage_model(wl)
-    dom = max(stage_ms, key=stage_ms.get)
-    sec = stage_ms[dom] / 1e3
-    m = model[dom]
-    if m["flops"] / (pk["bf16_tflops_sustained"] * 1e12) > m["bytes"] / (pk["hbm_gbs"] * 1e9):
-        achieved, peak, unit, bound = m["flops"] / sec / 1e12, pk["bf16_tflops_sustained"], \
-            "TFLOP/s", "tensor"
-    else:
-        achieved, peak, unit, bound = m["bytes"] / sec / 1e9, pk["hbm_gbs"], "GB/s", "hbm"
-    roofline = {"kernel": dom, "bound": bound, "achieved": achieved, "peak": peak, "unit": unit,
-                "frac": achieved / peak, "traffic": traffic_for(dom, wl.name),
-                "peak_source": pk["source"],
-                "algorithmic_bytes": m["bytes"], "algorithmic_flops": m["flops"],
-                "stage_ms": stage_ms}
-    total_bytes = sum(s["bytes"] for s in model.values())
-    total_flops = sum(s["flops"] for s in model.values())
-    t_roof = max(total_bytes / (pk["hbm_gbs"] * 1e9), total_flops / (pk["bf16_tflops"] * 1e12))
-    roofline["pass_roofline_ms"] = t_roof * 1e3
-    roofline["pass_frac"] = t_roof * 1e3 / ms_per_step
+    roofline = roofline_of(wl, stage_ms, ms_per_step, pk)
+    roofline["traffic"] = traffic_for(roofline["kernel"], wl.name)
 
-    cpu = None
     variant = args.dedup or args.bucket_mask or args.kmeans
+    table = None
+    if rank == 0 and world == 1 and not variant and not args.no_per_workload:
+        del qk, v, rot, step
+        table = per_workload(dev, stream, flush, min(args.steps, 20), args, pk)
+    cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and not variant:
         cpu = cpu_baseline(wl, args.cpu_rounds, args.cpu_heads)
 
@@ -590,7 +700,9 @@ def main(argv=None):
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16" if wl.dtype == torch.bfloat16 else "f32", "data": "synthetic",
             "config": dict(wl.describe(), l2="flushed before every timed step (256 MiB write)",
-                           parallelism=f"independent (batch, head) problems, 1 per GPU x{world}",
+                           parallelism=(f"{world} GPU(s): rank r owns the r-th slice of "
+                                        f"{wl.batch * world}x{wl.heads} (batch, head) problems; "
+                                        "no collective on the data path"),
                            **({"variant": " + ".join(
                                (["duplicate-count correction (LSH_FLAG_DEDUP)"] if args.dedup
                                 else []) +
@@ -603,11 +715,13 @@ def main(argv=None):
             "e2e": {"value": world * wl.tokens / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "ms_per_step": e2e_ms},
-            # per forward: hash 1, sort 3 (count, scan, scatter), attention 1, combine 1
-            "gpu_launches": 6 * args.steps,
+            # kernels this library launched during the timed steps (host count)
+            "gpu_launches": launches,
             "roofline": roofline,
             "cpu_baseline": cpu,
         }
+        if table is not None:
+            line["per_workload"] = table
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

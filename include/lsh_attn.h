@@ -19,10 +19,11 @@
  *  - All tensor arguments are DEVICE pointers (cudaMalloc'd or equivalent)
  *    unless the name ends in _host.  The caller owns every buffer, including
  *    the workspace, and the library keeps no pointer after a call returns.
- *    The library allocates nothing for the caller's data; the three places
- *    where it holds device resources of its own are stated at their calls:
- *    lsh_attn_sort's scratch pool, lsh_attn_forward_host's streams and
- *    events, and lsh_attn_forward_noalloc's built-in scratch.
+ *    The library allocates nothing: the stage calls and the fused call take
+ *    their temporary memory from caller workspaces (sized by the
+ *    *_workspace_size queries).  The two places where it holds device
+ *    resources of its own are stated at their calls: lsh_attn_forward_host's
+ *    streams and events, and lsh_attn_forward_noalloc's built-in scratch.
  *  - Every device pointer must be 16-byte aligned.  Tensors are dense,
  *    row-major, last dimension fastest.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
@@ -151,17 +152,20 @@ LSH_ATTN_API lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, co
  *   perm    [B, H, n_h, L]  int32 out: perm[.., s] = position at sorted slot s.
  *   undo    [B, H, n_h, L]  int32 out, may be NULL: undo[.., perm[.., s]] = s.
  *   counts  [B, H, n_h, n_b] int32 out, may be NULL: tokens per bucket.
+ *   workspace  device memory of at least lsh_attn_sort_workspace_size()
+ *              bytes (n_h * B * H * ceil(L / 2048) * n_b * 4: the per-tile
+ *              bucket counts); 16-byte aligned; contents on entry ignored.
  * Bucket ids outside [0, n_b) are undefined behaviour (stage 1 never makes
  * them); the kernels do not read or write out of bounds for them.
- * The call takes n_h * B * H * ceil(L / 2048) * n_b * 4 bytes of temporary
- * device memory, stream-ordered on `stream` from a memory pool the library
- * creates on first use on each device and keeps (cudaMallocFromPoolAsync /
- * cudaFreeAsync; the pool's blocks stay with it for reuse until the process
- * exits); a failed allocation returns LSH_ERR_CUDA.  The fused calls take it
- * from their workspace instead.
+ * A workspace smaller than the query's answer returns LSH_ERR_WORKSPACE.
+ * The per-bucket counts come out of this stage, not out of stage 1: the
+ * sort counts every tile of keys anyway (its first kernel), so the hash
+ * needs no histogram of its own.
  * ---------------------------------------------------------------------- */
+LSH_ATTN_API lsh_status lsh_attn_sort_workspace_size(const lsh_shape* shape, size_t* bytes);
 LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
-                         int32_t* undo, int32_t* counts, void* stream);
+                         int32_t* undo, int32_t* counts, void* workspace,
+                         size_t workspace_bytes, void* stream);
 
 /* ---------------------------------------------------------------------- *
  * Stage 3: chunked attention of every round, results stored at ORIGINAL
@@ -326,6 +330,18 @@ LSH_ATTN_API int lsh_attn_version(void);
  * A diagnostic for benchmarks that report how many of their kernels ran in a
  * timed region: read it before and after.  Thread-safe; never reset. */
 LSH_ATTN_API unsigned long long lsh_attn_kernel_launches(void);
+
+/* Test hook for the failure-detection path.  Every wait inside this
+ * library's tensor-core kernels is bounded (2 s); when one runs out the
+ * kernel records an error word, every role of the CTA leaves its loop, work
+ * already in flight is drained and the kernel returns, and
+ * lsh_attn_device_check reports LSH_ERR_DEVICE_TIMEOUT.  This call sets the
+ * limit, in ns, of the first wait of the tensor-core hash's MMA thread (for
+ * the input tile of every CTA) for the hash launches that follow: 0 makes
+ * that wait give up at once, so a test can exercise the path without any
+ * fault or hang.  Returns the previous limit; pass it back to restore the
+ * normal behaviour.  Process-wide; not for use while other threads launch. */
+LSH_ATTN_API unsigned long long lsh_attn_test_hash_first_wait(unsigned long long ns);
 
 #ifdef __cplusplus
 }

@@ -21,6 +21,7 @@ import torch
 
 __all__ = [
     "LshError", "Shape", "lib", "make_shape", "lsh_attn_hash", "lsh_attn_sort",
+    "lsh_attn_sort_workspace_size",
     "lsh_attn_chunked_fwd", "lsh_attn_chunked_fwd_ex", "lsh_attn_combine", "lsh_attn_forward",
     "lsh_attn_forward_workspace_size", "lsh_attn_forward_host",
     "lsh_attn_forward_host_device_bytes", "lsh_attn_device_check", "lsh_attn_forward_noalloc",
@@ -63,7 +64,8 @@ _SZ = ctypes.c_size_t
 _SHP = ctypes.POINTER(Shape)
 _SIGS = {
     "lsh_attn_hash": [_SHP, _P, _P, _P, _P, _P],
-    "lsh_attn_sort": [_SHP, _P, _P, _P, _P, _P],
+    "lsh_attn_sort_workspace_size": [_SHP, ctypes.POINTER(_SZ)],
+    "lsh_attn_sort": [_SHP, _P, _P, _P, _P, _P, _SZ, _P],
     "lsh_attn_chunked_fwd": [_SHP, _P, _P, _P, _P, _P, _P, _P],
     "lsh_attn_chunked_fwd_ex": [_SHP, _P, _P, _P, _P, _P, _P, _P, _P, _P],
     "lsh_attn_combine": [_SHP, _P, _P, _P, _P, _P],
@@ -79,6 +81,7 @@ _SIGS = {
     "lsh_attn_device_check": [_P],
     "lsh_attn_version": [],
     "lsh_attn_kernel_launches": [],
+    "lsh_attn_test_hash_first_wait": [ctypes.c_ulonglong],
 }
 
 
@@ -97,6 +100,7 @@ def lib() -> ctypes.CDLL:
         L.lsh_attn_status_string.restype = ctypes.c_char_p
         L.lsh_attn_last_error.restype = ctypes.c_char_p
         L.lsh_attn_kernel_launches.restype = ctypes.c_ulonglong
+        L.lsh_attn_test_hash_first_wait.restype = ctypes.c_ulonglong
         _lib = L
     return _lib
 
@@ -228,9 +232,17 @@ def lsh_attn_sort(buckets, n_buckets, *, want_undo=True, want_counts=False, stre
     undo = torch.empty_like(perm) if want_undo else None
     counts = torch.empty(B, H, n_h, n_buckets, dtype=torch.int32, device=buckets.device) \
         if want_counts else None
+    ws = torch.empty(lsh_attn_sort_workspace_size(shp), dtype=torch.uint8, device=buckets.device)
     _check(lib().lsh_attn_sort(ctypes.byref(shp), _ptr(buckets), _ptr(perm), _ptr(undo),
-                               _ptr(counts), _stream(stream)))
+                               _ptr(counts), _ptr(ws), ws.numel(), _stream(stream)))
     return perm, undo, counts
+
+
+def lsh_attn_sort_workspace_size(shape: Shape) -> int:
+    """Bytes of workspace lsh_attn_sort needs for `shape` (per-tile counts)."""
+    n = _SZ()
+    _check(lib().lsh_attn_sort_workspace_size(ctypes.byref(shape), ctypes.byref(n)))
+    return n.value
 
 
 def _stage3_args(qk, v, inv_norm, perm):

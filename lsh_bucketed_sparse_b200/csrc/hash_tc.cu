@@ -26,6 +26,7 @@
 // among maximal entries.
 #include <algorithm>
 #include <climits>
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -50,6 +51,7 @@ struct Params {
   int16_t* buckets;          // [BH, n_h, L]
   float* inv_norm;           // [BH, L]
   unsigned int* err;
+  unsigned long long first_wait_ns;  // limit of the MMA thread's first wait
   int BH, L, d, n_h, P;
   int gr;                    // rounds per group
   int G;                     // CTAs per group
@@ -220,7 +222,11 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
       bool ok = true, issued = false;
       for (int tile = g; ok && tile < p.n_tiles; tile += p.G, ++it) {
         const int s = it % p.stages;
-        if (!mbar_wait(&x_full[s], (it / p.stages) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_for(&x_full[s], (it / p.stages) & 1, abort_flag,
+                           it == 0 ? p.first_wait_ns : kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
         tc_fence_after_sync();
         const uint32_t xa = smem_u32(x_smem + (size_t)s * x_stage_bytes);
         for (int pc = 0; pc < p.n_pieces; ++pc, ++gp) {
@@ -469,6 +475,10 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
 }
 
 // ---------------------------------------------------------------- host side
+// Limit of the MMA thread's first wait (normally the 2 s of every bounded
+// wait); lsh_attn_test_hash_first_wait sets it to exercise the timeout path.
+std::atomic<unsigned long long> g_first_wait_ns{kWaitLimitNs};
+
 struct Plan {
   int gr, n_groups, G, piece_w, n_pieces, stages;
   int np;  // pairs of chunks per piece for the fixed-position epilogue, 0 = general
@@ -546,6 +556,7 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (cr != CUDA_SUCCESS) return cudaErrorInvalidValue;
   Params p;
+  p.first_wait_ns = g_first_wait_ns.load(std::memory_order_relaxed);
   p.rot = static_cast<const __nv_bfloat16*>(rot);
   p.buckets = buckets;
   p.inv_norm = inv_norm;
@@ -582,6 +593,10 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   if (e != cudaSuccess) return e;
   kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p); note_launch();
   return cudaGetLastError();
+}
+
+unsigned long long set_hash_first_wait_ns(unsigned long long ns) {
+  return g_first_wait_ns.exchange(ns);
 }
 
 }  // namespace lsh

@@ -63,6 +63,9 @@ unsigned int* device_error_word();
 cudaError_t launch_hash_portable(const Problem& p, const void* qk, const void* rot,
                                  int16_t* buckets, float* inv_norm, cudaStream_t st);
 bool hash_tc_supported(const Problem& p);
+// Sets the limit of the tensor-core hash's first MMA wait (test hook); returns
+// the previous limit.
+unsigned long long set_hash_first_wait_ns(unsigned long long ns);
 cudaError_t launch_hash_tc(const Problem& p, const void* qk, const void* rot, int16_t* buckets,
                            float* inv_norm, cudaStream_t st);
 

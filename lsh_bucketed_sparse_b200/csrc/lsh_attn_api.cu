@@ -268,29 +268,6 @@ HostPipe* host_pipe(int dev) {
   return g_pipe[dev].ok ? &g_pipe[dev] : nullptr;
 }
 
-// A memory pool per device for the stage calls' temporary scratch; its
-// release threshold is unlimited, so freed blocks stay with the pool.
-cudaMemPool_t g_pool[kMaxDevices];
-std::once_flag g_pool_once[kMaxDevices];
-
-cudaMemPool_t scratch_pool(int dev) {
-  std::call_once(g_pool_once[dev], [dev] {
-    cudaMemPoolProps props = {};
-    props.allocType = cudaMemAllocationTypePinned;
-    props.location.type = cudaMemLocationTypeDevice;
-    props.location.id = dev;
-    cudaMemPool_t pool = nullptr;
-    if (cudaMemPoolCreate(&pool, &props) != cudaSuccess) return;
-    uint64_t keep = ~0ull;
-    if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep) != cudaSuccess) {
-      cudaMemPoolDestroy(pool);
-      return;
-    }
-    g_pool[dev] = pool;
-  });
-  return g_pool[dev];
-}
-
 // Queues every group's copy-in, forward pass and copy-out on the pipe's
 // streams (host_pipe's comment gives the overlap).
 lsh_status host_groups(const Problem& p, const HostStaging& h, HostPipe* hp, int G,
@@ -383,32 +360,28 @@ lsh_status lsh_attn_hash(const lsh_shape* shape, const void* qk, const void* rot
   return run_hash(p, qk, rotations, buckets, inv_norm, static_cast<cudaStream_t>(stream));
 }
 
+lsh_status lsh_attn_sort_workspace_size(const lsh_shape* shape, size_t* bytes) {
+  Problem p;
+  CHECK(to_problem(shape, &p));
+  if (!bytes) return fail(LSH_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = sort_scratch_bytes(p);
+  return LSH_OK;
+}
+
 lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buckets, int32_t* perm,
-                         int32_t* undo, int32_t* counts, void* stream) {
+                         int32_t* undo, int32_t* counts, void* workspace, size_t workspace_bytes,
+                         void* stream) {
   Problem p;
   CHECK(to_problem(shape, &p));
   CHECK(check_ptr(buckets, "buckets"));
   CHECK(check_ptr(perm, "perm"));
   CHECK(check_ptr(undo, "undo", true));
   CHECK(check_ptr(counts, "counts", true));
-  // The per-tile counts live in stream-ordered scratch from the library's
-  // own memory pool on this device (it keeps its memory, so after the first
-  // call the allocation is a reuse), released on the same stream once the
-  // sort has used them.
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(LSH_ERR_UNSUPPORTED, "device %d", dev);
-  cudaMemPool_t pool = scratch_pool(dev);
-  if (!pool) return fail(LSH_ERR_CUDA, "could not create the scratch memory pool");
-  void* scratch = nullptr;
-  e = cudaMallocFromPoolAsync(&scratch, sort_scratch_bytes(p), pool, st);
-  if (e != cudaSuccess) return cuda_fail(e, "sort scratch");
-  const lsh_status r = run_sort(p, buckets, perm, undo, counts, scratch, st);
-  e = cudaFreeAsync(scratch, st);
-  if (r != LSH_OK) return r;
-  return e == cudaSuccess ? LSH_OK : cuda_fail(e, "sort scratch release");
+  CHECK(check_ptr(workspace, "workspace"));
+  const size_t need = sort_scratch_bytes(p);
+  if (workspace_bytes < need)
+    return fail(LSH_ERR_WORKSPACE, "sort workspace of %zu bytes, need %zu", workspace_bytes, need);
+  return run_sort(p, buckets, perm, undo, counts, workspace, static_cast<cudaStream_t>(stream));
 }
 
 lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,
@@ -609,6 +582,10 @@ lsh_status lsh_attn_device_check(void* stream) {
 }
 
 int lsh_attn_version(void) { return LSH_ATTN_VERSION; }
+
+unsigned long long lsh_attn_test_hash_first_wait(unsigned long long ns) {
+  return set_hash_first_wait_ns(ns);
+}
 
 unsigned long long lsh_attn_kernel_launches(void) {
   return g_launches.load(std::memory_order_relaxed);

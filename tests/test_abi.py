@@ -102,7 +102,15 @@ def test_unknown_flag_rejected(L):
 def test_stage_calls_validate(L):
     shp = shape()
     assert L.lsh_attn_hash(ctypes.byref(shp), FAKE, FAKE, None, FAKE, STREAM) == 1
-    assert L.lsh_attn_sort(ctypes.byref(shp), FAKE, None, None, None, STREAM) == 1
+    assert L.lsh_attn_sort(ctypes.byref(shp), FAKE, None, None, None, FAKE, 1 << 30, STREAM) == 1
+    # no workspace, or one that is too small
+    assert L.lsh_attn_sort(ctypes.byref(shp), FAKE, FAKE, None, None, None, 1 << 30, STREAM) == 1
+    need = ctypes.c_size_t()
+    assert L.lsh_attn_sort_workspace_size(ctypes.byref(shp), ctypes.byref(need)) == 0
+    assert need.value > 0
+    assert L.lsh_attn_sort(ctypes.byref(shp), FAKE, FAKE, None, None, FAKE, need.value - 16,
+                           STREAM) == 3  # LSH_ERR_WORKSPACE
+    assert b"sort workspace" in L.lsh_attn_last_error()
     assert L.lsh_attn_chunked_fwd(ctypes.byref(shp), FAKE, FAKE, FAKE, MISALIGNED, FAKE, FAKE,
                                   STREAM) == 1
     assert L.lsh_attn_combine(ctypes.byref(shp), FAKE, FAKE, FAKE, None, STREAM) == 1

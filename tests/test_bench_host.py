@@ -29,3 +29,47 @@ def test_window_pairs_counts_every_query_key_pair(L, c):
         lo = (k - 1) * c if k > 0 else 0
         brute += min((k + 1) * c, L) - lo
     assert bench.window_pairs(wl) == brute * 3 * 2
+
+
+def test_gpus_without_torchrun_relaunches_under_torch_distributed_run(monkeypatch):
+    calls = []
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "call", lambda cmd: calls.append(cmd) or 0)
+    assert bench.main(["--gpus", "4", "--steps", "2", "--warmup", "3"]) == 0
+    (cmd,) = calls
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert cmd[-6:] == [bench.os.path.abspath(bench.__file__), "--gpus", "4", "--steps", "2",
+                        "--warmup", "3"][-6:]
+
+
+def test_world_size_must_match_gpus(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--gpus", "4", "--warmup", "3"]) == 2
+
+
+def test_rank_inputs_are_the_headline_shape_with_per_rank_seeds():
+    wl = W.small("ranks", batch=1, heads=2, seq_len=128, n_hashes=2, n_buckets=8)
+    a = bench.rank_inputs(wl, 0, 2)
+    b = bench.rank_inputs(wl, 1, 2)
+    assert a[0].shape == b[0].shape == (1, 2, 128, 64)
+    assert not bool((a[0] == b[0]).all())
+    same = W.make_inputs(wl)
+    assert bool((a[0] == same[0]).all()) and bool((a[1] == same[1]).all())
+
+
+def test_roofline_of_uses_the_dominant_stage_and_both_peak_sets():
+    wl = W.HEADLINE
+    stage_ms = {"hash": 0.2, "sort": 0.05, "chunked_attention": 0.5, "combine": 0.1}
+    pk = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1400.0,
+          "source": "test"}
+    r = bench.roofline_of(wl, stage_ms, 0.85, pk)
+    m = bench.stage_model(wl)["chunked_attention"]
+    assert r["kernel"] == "chunked_attention" and r["bound"] == "hbm"
+    assert r["achieved"] == pytest.approx(m["bytes"] / 0.5e-3 / 1e9)
+    assert r["frac"] == pytest.approx(r["achieved"] / 6000.0)
+    assert r["frac_nominal"] == pytest.approx(r["achieved"] / 8000.0)
+    total = sum(x["bytes"] for x in bench.stage_model(wl).values())
+    assert r["pass_roofline_ms"] == pytest.approx(total / 6000e9 * 1e3)
+    assert r["pass_frac"] == pytest.approx(r["pass_roofline_ms"] / 0.85)
+    assert r["pass_frac_nominal"] < r["pass_frac"]
