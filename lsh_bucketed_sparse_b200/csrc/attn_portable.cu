@@ -4,7 +4,8 @@
 // "Implementation" and "Masking").
 //
 // Used for float32 inputs and shapes the tensor-core kernel does not take.
-// One CTA per (b*h, round, chunk), flattened into grid.x; one warp per query.  Keys of the window
+// One CTA per (b*h, round, chunk, group of kWarps queries of the chunk),
+// flattened into grid.x; one warp per query.  Keys of the window
 // (chunk k-1 when k > 0, and chunk k, in sorted order) are visited 32 at a
 // time, one key per lane for the score, with an online softmax; the value
 // accumulation gives each lane the output dimensions lane, lane + 32, ...
@@ -36,9 +37,12 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                      float scale) {
   extern __shared__ float q_all[];  // [kWarps][d]
   const int n_c = (L + c - 1) / c;  // the last chunk may be short
-  const int k = (int)(blockIdx.x % n_c);
-  const int r = (int)((blockIdx.x / n_c) % n_h);
-  const size_t bh = blockIdx.x / ((size_t)n_c * n_h);
+  const int qparts = (c + kWarps - 1) / kWarps;
+  const int qp = (int)(blockIdx.x % qparts);
+  const size_t chunk_id = blockIdx.x / qparts;
+  const int k = (int)(chunk_id % n_c);
+  const int r = (int)((chunk_id / n_c) % n_h);
+  const size_t bh = chunk_id / ((size_t)n_c * n_h);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int32_t* P = perm + (bh * n_h + r) * (size_t)L;
   const T* X = qk + bh * (size_t)L * d;
@@ -50,7 +54,8 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
   const int k0 = k > 0 ? (k - 1) * c : 0, k1 = min((k + 1) * c, L);
   constexpr int kPer = kMaxD / 32;
 
-  for (int qslot = k * c + warp; qslot < k1; qslot += kWarps) {
+  const int q_end = min(k * c + (qp + 1) * kWarps, k1);
+  for (int qslot = k * c + qp * kWarps + warp; qslot < q_end; qslot += kWarps) {
     const int i = P[qslot];
     for (int e = lane; e < d; e += 32) qs[e] = to_f32(X[(size_t)i * d + e]);
     __syncwarp();
@@ -124,7 +129,10 @@ cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v
   if (!p.dedup) undo = nullptr;
   if (!p.bucket_mask) buckets = nullptr;
   if (p.d > kMaxD) return cudaErrorInvalidValue;
-  const unsigned grid = (unsigned)((long long)p.n_chunks() * p.n_h * p.BH());
+  const long long qparts = (p.c + kWarps - 1) / kWarps;
+  const long long grid_ll = (long long)p.n_chunks() * p.n_h * p.BH() * qparts;
+  if (grid_ll > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const unsigned grid = (unsigned)grid_ll;
   const size_t smem = (size_t)kWarps * p.d * sizeof(float);
   const float scale = 1.0f / sqrtf((float)p.d);
   if (p.bf16)

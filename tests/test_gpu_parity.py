@@ -266,8 +266,9 @@ def test_host_buffer_entry_point_matches():
 def test_headline_workload_sampled():
     """L = 65536, 8 hashes, 1024 buckets (the long-text shape) at full size, in the
     configuration the benchmark times: buckets of one head in full and sampled
-    rows of the others against the oracle, the sort bit for bit everywhere, and
-    sampled tokens' per-round and combined outputs recomputed one by one."""
+    rows of the others against the oracle, the sort bit for bit everywhere,
+    head 0's per-round and combined outputs element by element, and sampled
+    tokens of the other heads recomputed one by one."""
     wl = W.HEADLINE
     qk, v, rot = W.make_inputs(wl)
     g = _stages(wl, qk, v, rot)
@@ -289,9 +290,27 @@ def test_headline_workload_sampled():
         perm, undo = O.sort_head(gb[0, h])
         np.testing.assert_array_equal(gp[0, h], perm)
         np.testing.assert_array_equal(gu[0, h], undo)
-    # attention + combine at sampled tokens (including the first, causal edge)
+    # attention + combine: head 0 in full, element by element (all 8 rounds,
+    # every token), and the median elementwise relative error of its output
     go_r, gl_r = g["o_rounds"], g["lse_rounds"]
-    for h in range(wl.heads):
+    o_r0 = np.empty((wl.n_hashes, wl.seq_len, wl.d_k))
+    l_r0 = np.empty((wl.n_hashes, wl.seq_len))
+    for r in range(wl.n_hashes):
+        o_r0[r], l_r0[r] = O.attend_round(x64[0, 0], v64[0, 0], gp[0, 0, r], wl.chunk_len,
+                                          wl.causal)
+    out0, lse0 = O.combine_head(o_r0, l_r0)
+    P.check_float(go_r[0, 0].cpu()[None], o_r0[None], bf16, "o_rounds(head 0)")
+    P.check_lse(gl_r[0, 0].cpu(), l_r0, bf16, "lse_rounds(head 0)")
+    P.check_float(g["f_out"][0, 0].cpu()[None, None], out0[None, None], bf16, "out(head 0)")
+    P.check_lse(g["f_lse"][0, 0].cpu(), lse0, bf16, "lse(head 0)")
+    go0 = P.np64(g["f_out"][0, 0])
+    big = np.abs(out0) > 1e-3 * np.abs(out0).max()
+    med = float(np.median(np.abs(go0 - out0)[big] / np.abs(out0)[big]))
+    print(f"headline out head 0: median elementwise relative error {med:.2e}")
+    assert med <= 5e-3, med  # bf16 rounding of the output alone is up to 2^-9 relative
+    # heads 1-7: sampled tokens (including the first, causal edge), each
+    # recomputed one by one through every round and the combine
+    for h in range(1, wl.heads):
         toks = np.concatenate([[0, 1, wl.seq_len - 1], rng.choice(wl.seq_len, 61, replace=False)])
         o_or, o_lr, o_out, o_lse = [], [], [], []
         for i in toks:
