@@ -120,6 +120,13 @@ SMALL = [
             n_buckets=128, chunk_len=128),
     W.small("tc-attn-c64-d64-noncausal", batch=2, heads=2, seq_len=1536, n_hashes=2,
             n_buckets=128, causal=False),
+    # L not a multiple of 4: every segment after the first starts off a
+    # 16-byte boundary of perm (position loads fall back to 4-byte loads)
+    W.small("odd-L1001-c64-d64", batch=2, heads=2, seq_len=1001, n_hashes=3, n_buckets=64),
+    W.small("odd-L999-c128-d64", heads=3, seq_len=999, n_hashes=2, n_buckets=64,
+            chunk_len=128, causal=False),
+    W.small("odd-L1003-c64-d128", heads=2, seq_len=1003, d_k=128, n_hashes=2,
+            n_buckets=128),
 ]
 
 
