@@ -50,6 +50,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "step_split.cuh"
 
 namespace lsh {
 namespace {
@@ -88,10 +89,7 @@ struct Params {
   const int32_t* undo;     // [BH, n_h, L] every round's undo for the duplicate correction
   unsigned int* err;
   int L, n_h, causal;
-  int steps;          // ceil(L / 128) per segment
-  int strip;          // steps per unit
-  int n_strips;
-  int n_units;
+  StepSplit split;    // the CTAs' share of the steps (ceil(L / 128) per segment)
   float ksc;          // log2 e / sqrt(d)
 };
 
@@ -159,43 +157,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
   return idesc_bf16_f32(M, N) | (1u << 16);
 }
 
-// A strip of steps [s0, s1) of segment (bh, r).
-struct Unit {
-  int bh, r, s0, s1;
-};
-
-__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
-  Unit x;
-  const int strip = u % p.n_strips;
-  const int seg = u / p.n_strips;
-  x.r = (int)(seg % p.n_h);
-  x.bh = (int)(seg / p.n_h);
-  x.s0 = strip * p.strip;
-  x.s1 = min(p.steps, x.s0 + p.strip);
-  return x;
-}
-
 // The CTA's sequence of blocks to load: for each of its units, the look-back
 // block (if s0 > 0) and then blocks s0 .. s1-1.
 struct Cursor {
-  int u;
+  int k;  // piece index
   Unit U;
   int b;
   bool valid;
 };
 
-__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, int u) {
-  c.u = u;
-  c.valid = u < p.n_units;
-  if (c.valid) {
-    c.U = unit_of(p, u);
-    c.b = c.U.s0 > 0 ? c.U.s0 - 1 : c.U.s0;
-  }
+__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, int k) {
+  int got;
+  while ((got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, c.U)) == kPieceEmpty) ++k;
+  c.k = k;
+  c.valid = got == kPieceRun;
+  if (c.valid) c.b = c.U.s0 > 0 ? c.U.s0 - 1 : c.U.s0;
 }
 
-__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, int u_step) {
+__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p) {
   if (!c.valid) return;
-  if (++c.b >= c.U.s1) cursor_start(c, p, c.u + u_step);
+  if (++c.b >= c.U.s1) cursor_start(c, p, c.k + 1);
 }
 
 // Positions of sorted slots sl .. sl+3 of a segment (INT_MAX past its end).
@@ -364,7 +345,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const int u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (warp == 0) {
     // ================================================================ qk producer
@@ -372,11 +352,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     // blocks ahead and norms one block ahead, so neither waits in line.
     if (lane == 0) tma_prefetch_desc(&qmap);
     Cursor c0, c1, c2;
-    cursor_start(c0, p, u_begin);
+    cursor_start(c0, p, 0);
     c1 = c0;
-    cursor_next(c1, p, u_step);
+    cursor_next(c1, p);
     c2 = c1;
-    cursor_next(c2, p, u_step);
+    cursor_next(c2, p);
     int pos0[4], pos1[4];
     float in0[4];
     int bk0[4];
@@ -445,7 +425,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       }
       c0 = c1;
       c1 = c2;
-      cursor_next(c2, p, u_step);
+      cursor_next(c2, p);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitProducer);
@@ -455,9 +435,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     // ================================================================ v producer
     if (lane == 0) tma_prefetch_desc(&vmap);
     Cursor c0, c1;
-    cursor_start(c0, p, u_begin);
+    cursor_start(c0, p, 0);
     c1 = c0;
-    cursor_next(c1, p, u_step);
+    cursor_next(c1, p);
     int pos0[4];
     cursor_positions(c0, p, lane, pos0);
     int li = 0;
@@ -480,7 +460,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
 #pragma unroll
       for (int k = 0; k < 4; ++k) pos0[k] = pos1[k];
       c0 = c1;
-      cursor_next(c1, p, u_step);
+      cursor_next(c1, p);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitProducer);
@@ -556,8 +536,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
         return true;
       };
-      for (int u = u_begin; ok && u < p.n_units; u += u_step) {
-        const Unit U = unit_of(p, u);
+      for (int k = 0; ok; ++k) {
+        Unit U;
+        const int got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, U);
+        if (got == kPieceEnd) break;
+        if (got == kPieceEmpty) continue;
         const int first = li;
         li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
         // S of the next step is computed while the softmax works on this one.
@@ -829,8 +812,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     };
 
     int li = 0, t = 0;
-    for (int u = u_begin; ok && u < p.n_units; u += u_step) {
-      const Unit U = unit_of(p, u);
+    for (int k = 0; ok; ++k) {
+      Unit U;
+      const int got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, U);
+      if (got == kPieceEnd) break;
+      if (got == kPieceEmpty) continue;
       const int first = li;
       li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
       RowState cur, next;
@@ -879,15 +865,8 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   p.L = pr.L;
   p.n_h = pr.n_h;
   p.causal = pr.causal ? 1 : 0;
-  p.steps = (pr.L + kQ - 1) / kQ;
-  const long long segs = (long long)pr.BH() * pr.n_h;
-  const long long total = segs * p.steps;
-  // About six strips per SM, each at least two steps.
-  int strip = (int)std::max<long long>(2, total / (148LL * 6));
-  strip = std::min(strip, p.steps);
-  p.strip = strip;
-  p.n_strips = (p.steps + strip - 1) / strip;
-  p.n_units = (int)(segs * p.n_strips);
+  int grid = 0;
+  p.split = make_step_split((long long)pr.BH() * pr.n_h, (pr.L + kQ - 1) / kQ, sm_count(), grid);
   p.ksc = kLog2e / sqrtf((float)pr.d);
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -921,8 +900,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   cudaError_t e = cudaFuncSetAttribute(kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)std::min<long long>(148, p.n_units);
-  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], p); note_launch();
+  kernel<<<(unsigned)grid, kThreads, smem, st>>>(maps[0], maps[1], p); note_launch();
   return cudaGetLastError();
 }
 

@@ -47,6 +47,7 @@
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
+#include "step_split.cuh"
 
 namespace lsh {
 namespace {
@@ -94,7 +95,7 @@ struct Params {
   const int32_t* undo;     // [BH, n_h, L] every round's undo for the duplicate correction
   unsigned int* err;
   int L, n_h, causal;
-  int steps, strip, n_strips, n_units;
+  StepSplit split;  // the CTAs' share of the steps
   float ksc;  // log2 e / sqrt(d)
 };
 
@@ -174,42 +175,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32_bmn(int M, int N) {
 // addresses stay below 2^18, so adding a byte offset / 16 never carries out.
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
-struct Unit {
-  int bh, r, s0, s1;
-};
-
-__device__ __forceinline__ Unit unit_of(const Params& p, int u) {
-  Unit x;
-  const int strip = u % p.n_strips;
-  const int seg = u / p.n_strips;
-  x.r = seg % p.n_h;
-  x.bh = seg / p.n_h;
-  x.s0 = strip * p.strip;
-  x.s1 = min(p.steps, x.s0 + p.strip);
-  return x;
-}
-
 // The CTA's sequence of blocks to load: for each of its units, the look-back
 // block (if s0 > 0) and then blocks s0 .. s1-1.
 struct Cursor {
-  int u;
+  int k;  // piece index
   Unit U;
   int b;
   bool valid;
 };
 
-__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, int u) {
-  c.u = u;
-  c.valid = u < p.n_units;
-  if (c.valid) {
-    c.U = unit_of(p, u);
-    c.b = c.U.s0 > 0 ? c.U.s0 - 1 : c.U.s0;
-  }
+__device__ __forceinline__ void cursor_start(Cursor& c, const Params& p, int k) {
+  int got;
+  while ((got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, c.U)) == kPieceEmpty) ++k;
+  c.k = k;
+  c.valid = got == kPieceRun;
+  if (c.valid) c.b = c.U.s0 > 0 ? c.U.s0 - 1 : c.U.s0;
 }
 
-__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p, int u_step) {
+__device__ __forceinline__ void cursor_next(Cursor& c, const Params& p) {
   if (!c.valid) return;
-  if (++c.b >= c.U.s1) cursor_start(c, p, c.u + u_step);
+  if (++c.b >= c.U.s1) cursor_start(c, p, c.k + 1);
 }
 
 // Positions of rows r0 .. r0+3 of the cursor's block (INT_MAX past the
@@ -340,7 +325,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem_base = *tmem_slot;
-  const int u_begin = blockIdx.x, u_step = gridDim.x;
 
   if (warp < kSoftBase) {
   if (warp < kQW) {
@@ -351,11 +335,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     const int r0 = kRowsQW * warp + 4 * lane;
     if (lane == 0) tma_prefetch_desc(&qmap);
     Cursor c0, c1, c2;
-    cursor_start(c0, p, u_begin);
+    cursor_start(c0, p, 0);
     c1 = c0;
-    cursor_next(c1, p, u_step);
+    cursor_next(c1, p);
     c2 = c1;
-    cursor_next(c2, p, u_step);
+    cursor_next(c2, p);
     int pos0[4], pos1[4];
     float in0[4];
     int bk0[4];
@@ -424,7 +408,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       }
       c0 = c1;
       c1 = c2;
-      cursor_next(c2, p, u_step);
+      cursor_next(c2, p);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitProducer);
@@ -447,11 +431,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     const int r0 = vrow0(w) + 4 * lane;
     if (lane == 0) tma_prefetch_desc(&vmap);
     Cursor c0, c1, c2;
-    cursor_start(c0, p, u_begin);
+    cursor_start(c0, p, 0);
     c1 = c0;
-    cursor_next(c1, p, u_step);
+    cursor_next(c1, p);
     c2 = c1;
-    cursor_next(c2, p, u_step);
+    cursor_next(c2, p);
     int pos0[4], pos1[4];
     cursor_positions(c0, p, r0, pos0);
     cursor_positions(c1, p, r0, pos1);
@@ -478,7 +462,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       }
       c0 = c1;
       c1 = c2;
-      cursor_next(c2, p, u_step);
+      cursor_next(c2, p);
     }
     if (!ok) {
       if (lane == 0) atomicOr(p.err, kErrWaitProducer);
@@ -567,8 +551,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
         return true;
       };
-      for (int u = u_begin; ok && u < p.n_units; u += u_step) {
-        const Unit U = unit_of(p, u);
+      for (int k = 0; ok; ++k) {
+        Unit U;
+        const int got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, U);
+        if (got == kPieceEnd) break;
+        if (got == kPieceEmpty) continue;
         const int first = li;
         li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
         // S of the next step is computed while the softmax works on this one.
@@ -834,8 +821,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     };
 
     int li = 0, t = 0;
-    for (int u = u_begin; ok && u < p.n_units; u += u_step) {
-      const Unit U = unit_of(p, u);
+    for (int k = 0; ok; ++k) {
+      Unit U;
+      const int got = split_piece(p.split, p.n_h, blockIdx.x, gridDim.x, k, U);
+      if (got == kPieceEnd) break;
+      if (got == kPieceEmpty) continue;
       const int first = li;
       li += (U.s1 - U.s0) + (U.s0 > 0 ? 1 : 0);
       RowState cur, next;
@@ -856,19 +846,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
   __syncthreads();
   tc_fence_after_sync();
   if (warp == kMmaWarp) tmem_dealloc(tmem_base, 512);
-}
-
-int sm_count() {
-  static int n = 0;
-  if (n == 0) {
-    int dev = 0, v = 0;
-    if (cudaGetDevice(&dev) == cudaSuccess &&
-        cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      n = v;
-    else
-      return 148;
-  }
-  return n;
 }
 
 }  // namespace
@@ -905,16 +882,9 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
   p.L = pr.L;
   p.n_h = pr.n_h;
   p.causal = pr.causal ? 1 : 0;
-  p.steps = (pr.L + kQ - 1) / kQ;
   const int sms = sm_count();
-  const long long segs = (long long)pr.BH() * pr.n_h;
-  const long long total = segs * p.steps;
-  // About six strips per SM, each at least two steps.
-  int strip = (int)std::max<long long>(2, total / ((long long)sms * 6));
-  strip = std::min(strip, p.steps);
-  p.strip = strip;
-  p.n_strips = (p.steps + strip - 1) / strip;
-  p.n_units = (int)(segs * p.n_strips);
+  int grid = 0;
+  p.split = make_step_split((long long)pr.BH() * pr.n_h, (pr.L + kQ - 1) / kQ, sms, grid);
   p.ksc = kLog2e / sqrtf((float)pr.d);
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
@@ -944,8 +914,7 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
   cudaError_t e;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)std::min<long long>(sms, p.n_units);
-  kernel<<<grid, kThreads, smem, st>>>(maps[0], maps[1], p);
+  kernel<<<(unsigned)grid, kThreads, smem, st>>>(maps[0], maps[1], p);
   note_launch();
   return cudaGetLastError();
 }

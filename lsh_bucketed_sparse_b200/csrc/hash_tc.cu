@@ -513,7 +513,7 @@ bool make_plan(const Problem& pr, Plan* out) {
       if (L.total + 1024 > (uint32_t)kSmemLimit) continue;
       out->gr = gr;
       out->n_groups = pr.n_h / gr;
-      out->G = (int)std::max(1LL, std::min<long long>(148 / out->n_groups, n_tiles));
+      out->G = (int)std::max(1LL, std::min<long long>(sm_count() / out->n_groups, n_tiles));
       out->piece_w = piece_w;
       out->n_pieces = (n_cols + piece_w - 1) / piece_w;
       out->stages = stages;

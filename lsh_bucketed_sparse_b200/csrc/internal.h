@@ -55,6 +55,10 @@ cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
 // after its <<<...>>>); read through lsh_attn_kernel_launches().
 void note_launch();
 
+// Streaming multiprocessors of the current device (148 on B200; 148 if the
+// query fails), cached per device.
+int sm_count();
+
 // Address of the device word that kernels set when a bounded wait runs out.
 // Resolved for the current device (cudaGetSymbolAddress); nullptr on error.
 unsigned int* device_error_word();

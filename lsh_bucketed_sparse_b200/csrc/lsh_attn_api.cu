@@ -41,6 +41,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 std::once_flag g_word_once[kMaxDevices];
 unsigned int* g_word_ptr[kMaxDevices];
+std::atomic<int> g_sm_count[kMaxDevices];
 
 }  // namespace
 
@@ -331,6 +332,17 @@ cudaError_t join_pipe(HostPipe* hp, cudaStream_t st) {
 }
 
 }  // namespace
+
+int sm_count() {
+  int dev = 0, v = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = g_sm_count[dev].load(std::memory_order_relaxed);
+  if (n > 0) return n;
+  if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+    return 148;
+  g_sm_count[dev].store(v, std::memory_order_relaxed);
+  return v;
+}
 
 unsigned int* device_error_word() {
   int dev = 0;
