@@ -18,9 +18,11 @@
 //               one of the two accumulator buffers;
 //   warps 2..9  epilogue: two warps per TMEM lane quadrant (32 token rows),
 //               splitting each round's 32-column chunks between them; each
-//               keeps, per row, the first chunk that holds its largest |p|
-//               and resolves the exact index at the end of the round; the
-//               two halves' candidates meet through shared memory.
+//               keeps, per row, the 8-column group that holds its largest
+//               |p| (a copy in shared memory, stored only by the lanes whose
+//               candidate changes) and resolves the exact index at the end
+//               of the round; the two halves' candidates meet through shared
+//               memory.
 // Argmax order: larger |p| first; among equal |p| the smaller index of
 // [xR; -xR] (p_j >= 0 gives index j, else n_b/2 + j), i.e. the lowest index
 // among maximal entries.
@@ -41,6 +43,7 @@ using namespace sm100;
 constexpr int kRows = 128;          // tokens per tile = MMA M = TMEM lanes
 constexpr int kPieceMax = 256;      // columns per accumulator buffer = MMA N max
 constexpr int kChunk = 32;          // columns per tcgen05.ld
+constexpr int kGroup = 8;           // columns of a chunk saved as a candidate
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int kRBudget = 128 * 1024;
@@ -71,7 +74,7 @@ __host__ __device__ inline Smem smem_layout(int n_cols, int d, int stages) {
   uint32_t off = 0;
   s.r = off;    off += (uint32_t)n_cols * d * 2;
   s.x = off;    off += (uint32_t)stages * kRows * d * 2;
-  s.save = off; off += kEpiWarps * 32 * kChunk * 4;   // one 128-byte row per epilogue thread
+  s.save = off; off += kEpiWarps * 32 * kGroup * 4;   // 32 bytes per epilogue thread
   s.bars = off; off += (uint32_t)(2 * stages + 4 + 4 + 1) * 8;
   s.xch = off;  off += 2 * kRows * 8;
   s.misc = off; off += 16;
@@ -90,30 +93,20 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// Largest |p| of a 32-column chunk: a depth-4 tree of 17 max instructions.
-__device__ __forceinline__ float chunk_max_abs(const uint32_t* u) {
-  float v[11];
+// Largest |p| (hash) or p (assignment) of each 8-column group of a
+// 32-column chunk: four max instructions per group.
+template <bool ABS>
+__device__ __forceinline__ void group_maxima(const uint32_t* u, float* g) {
 #pragma unroll
-  for (int t = 0; t < 10; ++t)
-    v[t] = max3f(fabsf(__uint_as_float(u[3 * t])), fabsf(__uint_as_float(u[3 * t + 1])),
-                 fabsf(__uint_as_float(u[3 * t + 2])));
-  v[10] = fmaxf(fabsf(__uint_as_float(u[30])), fabsf(__uint_as_float(u[31])));
-  const float w0 = max3f(v[0], v[1], v[2]), w1 = max3f(v[3], v[4], v[5]);
-  const float w2 = max3f(v[6], v[7], v[8]), w3 = fmaxf(v[9], v[10]);
-  return fmaxf(max3f(w0, w1, w2), w3);
-}
-
-// Largest signed p of a 32-column chunk (the routing-style assignment).
-__device__ __forceinline__ float chunk_max_signed(const uint32_t* u) {
-  float v[11];
+  for (int k = 0; k < 4; ++k) {
+    float v[8];
 #pragma unroll
-  for (int t = 0; t < 10; ++t)
-    v[t] = max3f(__uint_as_float(u[3 * t]), __uint_as_float(u[3 * t + 1]),
-                 __uint_as_float(u[3 * t + 2]));
-  v[10] = fmaxf(__uint_as_float(u[30]), __uint_as_float(u[31]));
-  const float w0 = max3f(v[0], v[1], v[2]), w1 = max3f(v[3], v[4], v[5]);
-  const float w2 = max3f(v[6], v[7], v[8]), w3 = fmaxf(v[9], v[10]);
-  return fmaxf(max3f(w0, w1, w2), w3);
+    for (int t = 0; t < 8; ++t) {
+      const float x = __uint_as_float(u[8 * k + t]);
+      v[t] = ABS ? fabsf(x) : x;
+    }
+    g[k] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+  }
 }
 
 // KM: the routing-style assignment (argmax over the n_b columns of given
@@ -269,46 +262,35 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     const int half = ew >> 2;            // which alternate 32-column chunks
     const int row = quad * 32 + lane;    // token row inside the tile
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    // This thread's copy of the chunk that holds its row's largest |p| so
-    // far: a private 128-byte row, 16-byte pieces rotated by (lane & 7) so
-    // that neighbouring lanes hit different banks.
-    uint8_t* my_save = save_smem + (size_t)(ew * 32 + lane) * (kChunk * 4);
-    const int sx = lane & 7;
-    // Predicated stores: no branch, so the warp stays converged.
-    auto save_chunk_if = [&](bool take, const uint32_t* u) {
+    // This thread's copy of the 8-column group that holds its row's largest
+    // |p| so far: two 16-byte slots, swapped on every other group of four
+    // lanes so that the eight lanes of a quarter warp hit different banks.
+    uint8_t* my_save = save_smem + (size_t)(ew * 32 + lane) * (kGroup * 4);
+    const int sx = (lane >> 2) & 1;
+    // Group k of the chunk u when `take` and k == grp: predicated stores, so
+    // that the warp stays converged and each lane writes at most 32 bytes.
+    auto save_group_if = [&](bool take, int grp, const uint32_t* u) {
       const uint32_t base = smem_u32(my_save);
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
-          "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
-          "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t"
-          "@p st.shared.v4.b32 [%11], {%12, %13, %14, %15};\n\t"
-          "@p st.shared.v4.b32 [%16], {%17, %18, %19, %20};\n\t}" ::"r"((uint32_t)take),
-          "r"(base + (uint32_t)((0 ^ sx) << 4)), "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]),
-          "r"(base + (uint32_t)((1 ^ sx) << 4)), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]),
-          "r"(base + (uint32_t)((2 ^ sx) << 4)), "r"(u[8]), "r"(u[9]), "r"(u[10]), "r"(u[11]),
-          "r"(base + (uint32_t)((3 ^ sx) << 4)), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
-          : "memory");
-      asm volatile(
-          "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
-          "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
-          "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t"
-          "@p st.shared.v4.b32 [%11], {%12, %13, %14, %15};\n\t"
-          "@p st.shared.v4.b32 [%16], {%17, %18, %19, %20};\n\t}" ::"r"((uint32_t)take),
-          "r"(base + (uint32_t)((4 ^ sx) << 4)), "r"(u[16]), "r"(u[17]), "r"(u[18]), "r"(u[19]),
-          "r"(base + (uint32_t)((5 ^ sx) << 4)), "r"(u[20]), "r"(u[21]), "r"(u[22]), "r"(u[23]),
-          "r"(base + (uint32_t)((6 ^ sx) << 4)), "r"(u[24]), "r"(u[25]), "r"(u[26]), "r"(u[27]),
-          "r"(base + (uint32_t)((7 ^ sx) << 4)), "r"(u[28]), "r"(u[29]), "r"(u[30]), "r"(u[31])
-          : "memory");
+      const uint32_t a0 = base + (uint32_t)(sx << 4), a1 = base + (uint32_t)((sx ^ 1) << 4);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t* w = u + 8 * k;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+            "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
+            "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t}" ::"r"((uint32_t)(take && grp == k)),
+            "r"(a0), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]),
+            "r"(a1), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
+            : "memory");
+      }
     };
     auto load_saved = [&](float* sv) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint4 w = *reinterpret_cast<const uint4*>(my_save + ((q ^ sx) << 4));
-        sv[4 * q] = __uint_as_float(w.x);
-        sv[4 * q + 1] = __uint_as_float(w.y);
-        sv[4 * q + 2] = __uint_as_float(w.z);
-        sv[4 * q + 3] = __uint_as_float(w.w);
-      }
+      const uint4 w0 = *reinterpret_cast<const uint4*>(my_save + (sx << 4));
+      const uint4 w1 = *reinterpret_cast<const uint4*>(my_save + ((sx ^ 1) << 4));
+      sv[0] = __uint_as_float(w0.x); sv[1] = __uint_as_float(w0.y);
+      sv[2] = __uint_as_float(w0.z); sv[3] = __uint_as_float(w0.w);
+      sv[4] = __uint_as_float(w1.x); sv[5] = __uint_as_float(w1.y);
+      sv[6] = __uint_as_float(w1.z); sv[7] = __uint_as_float(w1.w);
     };
     int it = 0, gp = 0, ex = 0;
     bool ok = true;
@@ -317,29 +299,46 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     float best_a = kNone;
     int best_j0 = 0;
 
-    // One 32-column chunk starting at round column j0: keep it when it holds
-    // a larger |p| (hash) or p (assignment) than every earlier chunk of the
-    // round; on equal values the earlier chunk stays, except for the hash's
-    // positive-entry rule below.
+    // One 32-column chunk starting at round column j0: keep its group that
+    // holds the largest |p| (hash) or p (assignment) when that beats every
+    // earlier chunk of the round.  Equal values keep the earliest entry,
+    // except for the hash's rule that a positive entry wins over negative ones
+    // (handled on the rare path below, for ties inside the chunk and with the
+    // saved group).
     auto take_chunk = [&](const uint32_t* u, int j0) {
-      const float cm = KM ? chunk_max_signed(u) : chunk_max_abs(u);
+      float g[4];
+      group_maxima<!KM>(u, g);
+      const float cm = fmaxf(max3f(g[0], g[1], g[2]), g[3]);
+      int grp = g[2] == cm ? 2 : 3;
+      grp = g[1] == cm ? 1 : grp;
+      grp = g[0] == cm ? 0 : grp;
       bool take = cm > best_a;
-      if (!KM && __any_sync(0xffffffffu, cm == best_a)) {
-        // Equal largest |p| in an earlier chunk (rare): a positive entry
-        // wins over negative ones, and the earlier chunk wins otherwise.
-        float sv[kChunk];
-        load_saved(sv);
-        bool pos_saved = false, pos_new = false;
+      if (!KM) {
+        const int n_eq = (g[0] == cm) + (g[1] == cm) + (g[2] == cm) + (g[3] == cm);
+        if (__any_sync(0xffffffffu, n_eq > 1 || cm == best_a)) {
+          // The lowest group holding +cm, if any, carries the chunk's candidate.
+          int gpos = -1;
 #pragma unroll
-        for (int t = 0; t < kChunk; ++t) {
-          pos_saved |= (sv[t] == best_a);
-          pos_new |= (__uint_as_float(u[t]) == cm);
+          for (int k = 3; k >= 0; --k) {
+            bool hp = false;
+#pragma unroll
+            for (int t = 0; t < kGroup; ++t) hp |= (__uint_as_float(u[8 * k + t]) == cm);
+            if (hp) gpos = k;
+          }
+          if (gpos >= 0) grp = gpos;
+          if (cm == best_a) {
+            float sv[kGroup];
+            load_saved(sv);
+            bool pos_saved = false;
+#pragma unroll
+            for (int t = 0; t < kGroup; ++t) pos_saved |= (sv[t] == best_a);
+            take = !pos_saved && gpos >= 0;
+          }
         }
-        if (cm == best_a) take = !pos_saved && pos_new;
       }
       best_a = take ? cm : best_a;
-      best_j0 = take ? j0 : best_j0;
-      save_chunk_if(take, u);
+      best_j0 = take ? j0 + kGroup * grp : best_j0;
+      save_group_if(take, grp, u);
     };
 
     // End of round r0 + rr: this half's candidate, then the two halves meet
@@ -348,11 +347,11 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
       int z = INT_MAX;
       const float a = best_a;
       if (best_a > kNone) {
-        float sv[kChunk];
+        float sv[kGroup];
         load_saved(sv);
         int tp = -1, tn = 0;
 #pragma unroll
-        for (int t = kChunk - 1; t >= 0; --t) {
+        for (int t = kGroup - 1; t >= 0; --t) {
           if (sv[t] == best_a) tp = t;
           if (!KM && sv[t] == -best_a) tn = t;
         }
