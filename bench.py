@@ -54,7 +54,7 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 KERNEL_SOURCES = {
     "hash": ["hash_tc.cu", "hash_portable.cu"],
     "sort": ["sort.cu"],
-    "chunked_attention": ["attn_tc.cu", "attn_tc64.cu", "attn_portable.cu"],
+    "chunked_attention": ["attn_tc.cu", "attn_tc64.cu", "attn_portable.cu", "step_split.cuh"],
     "combine": ["combine.cu"],
 }
 
