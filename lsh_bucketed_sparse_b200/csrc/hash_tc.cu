@@ -18,7 +18,7 @@
 //               one of the two accumulator buffers;
 //   warps 2..9  epilogue: two warps per TMEM lane quadrant (32 token rows),
 //               splitting each round's 32-column chunks between them; each
-//               keeps, per row, the 8-column group that holds its largest
+//               keeps, per row, the 16-column group that holds its largest
 //               |p| (a copy in shared memory, stored only by the lanes whose
 //               candidate changes) and resolves the exact index at the end
 //               of the round; the two halves' candidates meet through shared
@@ -43,7 +43,13 @@ using namespace sm100;
 constexpr int kRows = 128;          // tokens per tile = MMA M = TMEM lanes
 constexpr int kPieceMax = 256;      // columns per accumulator buffer = MMA N max
 constexpr int kChunk = 32;          // columns per tcgen05.ld
-constexpr int kGroup = 8;           // columns of a chunk saved as a candidate
+// Columns of a chunk saved as a candidate.  Measured on the long-text
+// workload: groups of 8 0.520 ms, of 16 0.512 ms, whole 32-column chunks
+// 0.551 ms (more shared-memory wavefronts per save).
+constexpr int kGroup = 16;
+constexpr int kGroups = kChunk / kGroup;  // groups per chunk
+constexpr int kSlots = kGroup / 4;        // 16-byte slots of a saved group
+static_assert(kGroup == 8 || kGroup == 16, "group of 8 or 16 columns");
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = (2 + kEpiWarps) * 32;
 constexpr int kRBudget = 128 * 1024;
@@ -74,7 +80,7 @@ __host__ __device__ inline Smem smem_layout(int n_cols, int d, int stages) {
   uint32_t off = 0;
   s.r = off;    off += (uint32_t)n_cols * d * 2;
   s.x = off;    off += (uint32_t)stages * kRows * d * 2;
-  s.save = off; off += kEpiWarps * 32 * kGroup * 4;   // 32 bytes per epilogue thread
+  s.save = off; off += kEpiWarps * 32 * kGroup * 4;   // one saved group per epilogue thread
   s.bars = off; off += (uint32_t)(2 * stages + 4 + 4 + 1) * 8;
   s.xch = off;  off += 2 * kRows * 8;
   s.misc = off; off += 16;
@@ -93,19 +99,26 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return r;
 }
 
-// Largest |p| (hash) or p (assignment) of each 8-column group of a
-// 32-column chunk: four max instructions per group.
+// Largest |p| (hash) or p (assignment) of each group of a 32-column chunk:
+// a tree of three-input max instructions (four per 8 columns, eight per 16).
 template <bool ABS>
 __device__ __forceinline__ void group_maxima(const uint32_t* u, float* g) {
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    float v[8];
+  for (int k = 0; k < kGroups; ++k) {
+    float v[kGroup];
 #pragma unroll
-    for (int t = 0; t < 8; ++t) {
-      const float x = __uint_as_float(u[8 * k + t]);
+    for (int t = 0; t < kGroup; ++t) {
+      const float x = __uint_as_float(u[kGroup * k + t]);
       v[t] = ABS ? fabsf(x) : x;
     }
-    g[k] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+    if constexpr (kGroup == 8) {
+      g[k] = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]), fmaxf(v[6], v[7]));
+    } else {
+      const float a = max3f(max3f(v[0], v[1], v[2]), max3f(v[3], v[4], v[5]),
+                            max3f(v[6], v[7], v[8]));
+      const float b = max3f(max3f(v[9], v[10], v[11]), max3f(v[12], v[13], v[14]), v[15]);
+      g[k] = fmaxf(a, b);
+    }
   }
 }
 
@@ -262,35 +275,38 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     const int half = ew >> 2;            // which alternate 32-column chunks
     const int row = quad * 32 + lane;    // token row inside the tile
     const uint32_t lane_addr = tmem_base + ((uint32_t)(quad * 32) << 16);
-    // This thread's copy of the 8-column group that holds its row's largest
-    // |p| so far: two 16-byte slots, swapped on every other group of four
-    // lanes so that the eight lanes of a quarter warp hit different banks.
+    // This thread's copy of the group that holds its row's largest |p| so
+    // far: kSlots 16-byte slots, their order permuted per lane so that the
+    // eight lanes of a quarter warp hit different banks.
     uint8_t* my_save = save_smem + (size_t)(ew * 32 + lane) * (kGroup * 4);
-    const int sx = (lane >> 2) & 1;
+    const int sx = kGroup == 8 ? ((lane >> 2) & 1) : ((lane >> 1) & 3);
+    auto slot_addr = [&](int q) { return smem_u32(my_save) + (uint32_t)((q ^ sx) << 4); };
     // Group k of the chunk u when `take` and k == grp: predicated stores, so
-    // that the warp stays converged and each lane writes at most 32 bytes.
+    // that the warp stays converged and each lane writes one group at most.
     auto save_group_if = [&](bool take, int grp, const uint32_t* u) {
-      const uint32_t base = smem_u32(my_save);
-      const uint32_t a0 = base + (uint32_t)(sx << 4), a1 = base + (uint32_t)((sx ^ 1) << 4);
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t* w = u + 8 * k;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
-            "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t"
-            "@p st.shared.v4.b32 [%6], {%7, %8, %9, %10};\n\t}" ::"r"((uint32_t)(take && grp == k)),
-            "r"(a0), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]),
-            "r"(a1), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7])
-            : "memory");
+      for (int k = 0; k < kGroups; ++k) {
+        const uint32_t on = (uint32_t)(take && grp == k);
+#pragma unroll
+        for (int q = 0; q < kSlots; ++q) {
+          const uint32_t* w = u + kGroup * k + 4 * q;
+          asm volatile(
+              "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
+              "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"(on),
+              "r"(slot_addr(q)), "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3])
+              : "memory");
+        }
       }
     };
     auto load_saved = [&](float* sv) {
-      const uint4 w0 = *reinterpret_cast<const uint4*>(my_save + (sx << 4));
-      const uint4 w1 = *reinterpret_cast<const uint4*>(my_save + ((sx ^ 1) << 4));
-      sv[0] = __uint_as_float(w0.x); sv[1] = __uint_as_float(w0.y);
-      sv[2] = __uint_as_float(w0.z); sv[3] = __uint_as_float(w0.w);
-      sv[4] = __uint_as_float(w1.x); sv[5] = __uint_as_float(w1.y);
-      sv[6] = __uint_as_float(w1.z); sv[7] = __uint_as_float(w1.w);
+#pragma unroll
+      for (int q = 0; q < kSlots; ++q) {
+        const uint4 w = *reinterpret_cast<const uint4*>(my_save + ((q ^ sx) << 4));
+        sv[4 * q] = __uint_as_float(w.x);
+        sv[4 * q + 1] = __uint_as_float(w.y);
+        sv[4 * q + 2] = __uint_as_float(w.z);
+        sv[4 * q + 3] = __uint_as_float(w.w);
+      }
     };
     int it = 0, gp = 0, ex = 0;
     bool ok = true;
@@ -306,23 +322,31 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     // (handled on the rare path below, for ties inside the chunk and with the
     // saved group).
     auto take_chunk = [&](const uint32_t* u, int j0) {
-      float g[4];
+      float g[kGroups];
       group_maxima<!KM>(u, g);
-      const float cm = fmaxf(max3f(g[0], g[1], g[2]), g[3]);
-      int grp = g[2] == cm ? 2 : 3;
-      grp = g[1] == cm ? 1 : grp;
-      grp = g[0] == cm ? 0 : grp;
+      float cm;
+      int grp, n_eq;
+      if constexpr (kGroups == 4) {
+        cm = fmaxf(max3f(g[0], g[1], g[2]), g[3]);
+        grp = g[2] == cm ? 2 : 3;
+        grp = g[1] == cm ? 1 : grp;
+        grp = g[0] == cm ? 0 : grp;
+        n_eq = (g[0] == cm) + (g[1] == cm) + (g[2] == cm) + (g[3] == cm);
+      } else {
+        cm = fmaxf(g[0], g[1]);
+        grp = g[0] == cm ? 0 : 1;
+        n_eq = g[0] == g[1] ? 2 : 1;
+      }
       bool take = cm > best_a;
       if (!KM) {
-        const int n_eq = (g[0] == cm) + (g[1] == cm) + (g[2] == cm) + (g[3] == cm);
         if (__any_sync(0xffffffffu, n_eq > 1 || cm == best_a)) {
           // The lowest group holding +cm, if any, carries the chunk's candidate.
           int gpos = -1;
 #pragma unroll
-          for (int k = 3; k >= 0; --k) {
+          for (int k = kGroups - 1; k >= 0; --k) {
             bool hp = false;
 #pragma unroll
-            for (int t = 0; t < kGroup; ++t) hp |= (__uint_as_float(u[8 * k + t]) == cm);
+            for (int t = 0; t < kGroup; ++t) hp |= (__uint_as_float(u[kGroup * k + t]) == cm);
             if (hp) gpos = k;
           }
           if (gpos >= 0) grp = gpos;
