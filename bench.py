@@ -659,26 +659,47 @@ def main(argv=None):
 
     stage_ms = stage_times(wl, qk, v, rot, stream, flush, min(args.steps, 10), args)
 
-    # End to end through the host-buffer entry point: copies in and out timed.
+    # End to end through the host-buffer entry point: every step copies its
+    # inputs in from pinned host memory and its outputs back, inside the
+    # timed region.  Steps alternate between two caller streams, each with
+    # its own device buffer and host output buffers (as a caller streaming
+    # batches would), so one step's copies in may start while the previous
+    # step's last heads are still computed and copied out.
     pin = [t.pin_memory() if t is not None else None for t in (qk_h, v_h, rot_h)]
-    out_h = torch.empty_like(qk_h).pin_memory()
-    lse_h = torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32).pin_memory()
-    dbuf = torch.empty(lsh.lsh_attn_forward_host_device_bytes(shp), dtype=torch.uint8, device=dev)
-    for _ in range(3):
-        lsh.lsh_attn_forward_host(shp, pin[0], pin[1], pin[2], out_h, lse_h, dbuf)
+    n_dev = lsh.lsh_attn_forward_host_device_bytes(shp)
+    lanes = []
+    for _ in range(2):
+        lanes.append({
+            "stream": torch.cuda.Stream(device=dev),
+            "out": torch.empty_like(qk_h).pin_memory(),
+            "lse": torch.empty(wl.batch, wl.heads, wl.seq_len, dtype=torch.float32).pin_memory(),
+            "dbuf": torch.empty(n_dev, dtype=torch.uint8, device=dev),
+        })
+
+    def e2e_step(k):
+        ln = lanes[k % 2]
+        lsh.lsh_attn_forward_host(shp, pin[0], pin[1], pin[2], ln["out"], ln["lse"], ln["dbuf"],
+                                  stream=ln["stream"])
+
+    for k in range(4):
+        e2e_step(k)
     e2e_steps = min(args.steps, 10)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
     e0.record(stream)
-    for _ in range(e2e_steps):
-        lsh.lsh_attn_forward_host(shp, pin[0], pin[1], pin[2], out_h, lse_h, dbuf)
+    for ln in lanes:
+        ln["stream"].wait_stream(stream)
+    for k in range(e2e_steps):
+        e2e_step(k)
+    for ln in lanes:
+        stream.wait_stream(ln["stream"])
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world) / e2e_steps
     h2d = sum(t.numel() * t.element_size() for t in pin if t is not None)
-    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * 4
-    del pin, out_h, lse_h, dbuf
+    d2h = lanes[0]["out"].numel() * lanes[0]["out"].element_size() + lanes[0]["lse"].numel() * 4
+    del pin, lanes
 
     pk = peaks()
     roofline = roofline_of(wl, stage_ms, ms_per_step, pk)
