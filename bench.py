@@ -51,11 +51,17 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # B200 datasheet figures (HGX: 8 TB/s HBM3e, 2.25 PFLOP/s dense bf16); every
 # fraction is also reported against these.
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+# The files each stage's captured kernel is built from (its source and the
+# headers it includes, paths from the repository root): a DRAM-traffic record
+# in profiles/traffic.json holds only while their hash is unchanged.
+CSRC = "lsh_bucketed_sparse_b200/csrc/"
+_HEADERS = [CSRC + "common.cuh", CSRC + "internal.h", "include/lsh_attn.h"]
 KERNEL_SOURCES = {
-    "hash": ["hash_tc.cu", "hash_portable.cu"],
-    "sort": ["sort.cu"],
-    "chunked_attention": ["attn_tc.cu", "attn_tc64.cu", "attn_portable.cu", "step_split.cuh"],
-    "combine": ["combine.cu"],
+    "hash": [CSRC + "hash_tc.cu", CSRC + "sm100.cuh"] + _HEADERS,
+    "sort": [CSRC + "sort.cu"] + _HEADERS,
+    "chunked_attention": [CSRC + "attn_tc64.cu", CSRC + "sm100.cuh",
+                          CSRC + "step_split.cuh"] + _HEADERS,
+    "combine": [CSRC + "combine.cu"] + _HEADERS,
 }
 
 
@@ -112,7 +118,7 @@ def stage_model(wl):
 def source_sha(stage):
     h = hashlib.sha256()
     for name in KERNEL_SOURCES[stage]:
-        with open(os.path.join(ROOT, "lsh_bucketed_sparse_b200", "csrc", name), "rb") as f:
+        with open(os.path.join(ROOT, name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
