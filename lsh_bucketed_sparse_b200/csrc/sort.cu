@@ -18,8 +18,9 @@
 //      of shared memory, the rows are turned into each warp's first slot per
 //      bucket (base + tile prefix + the counts of the warps before it), and
 //      each warp then walks its keys in order, 32 at a time, ranking equal
-//      keys inside the warp with __match_any_sync: equal buckets keep
-//      position order (stability) without global atomics.  Above 192
+//      keys inside the warp (equal-key lane masks built from one ballot per
+//      bit of the bucket id): equal buckets keep position order (stability)
+//      without global atomics.  Above 192
 //      buckets (where eight rows of counts cost more than they save) one
 //      warp walks the whole tile instead.
 #include "common.cuh"
@@ -41,6 +42,20 @@ constexpr int kSubKeys = kTileKeys / kScatterWarps;  // keys per scatter warp
 // n_b = 64: 31.7 -> 21.5; 192: 33.8 -> 27.6; 256: 29.7 -> 35.8; 1024:
 // 60.4 -> 87.0.  So eight warps up to n_b = 192, one warp above.
 constexpr int kScatterWideMaxBuckets = 192;
+
+// Lanes of the warp holding the same key as this lane: built from one ballot
+// per bit of the key (keys below 2^bits; invalid lanes form their own
+// group).  Cheaper than __match_any_sync for the ten bits of 1024 buckets.
+__device__ __forceinline__ unsigned same_key(bool valid, int b, int bits) {
+  const unsigned v = __ballot_sync(0xffffffffu, valid);
+  unsigned m = valid ? v : ~v;
+  for (int k = 0; k < bits; ++k) {
+    const bool bit = valid && ((b >> k) & 1);
+    const unsigned x = __ballot_sync(0xffffffffu, bit);
+    m &= bit ? x : ~x;
+  }
+  return m;
+}
 
 __global__ void __launch_bounds__(kCountThreads)
 sort_count_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ cnt, int L,
@@ -148,7 +163,9 @@ sort_scatter8_kernel(const int16_t* __restrict__ buckets, const int32_t* __restr
   const int beg = tile * kTileKeys + warp * kSubKeys;
   const int end = min(L, min(tile * kTileKeys + kTileKeys, beg + kSubKeys));
   constexpr int kRowsW = kSubKeys / 32;
+  const int bits = 32 - __clz(max(n_b - 1, 1));
   int kb[kRowsW];
+  unsigned peers[kRowsW];
 #pragma unroll
   for (int i = 0; i < kRowsW; ++i) {
     const int e = beg + 32 * i + lane;
@@ -160,8 +177,8 @@ sort_scatter8_kernel(const int16_t* __restrict__ buckets, const int32_t* __restr
     const int e = beg + 32 * i + lane;
     const int b = kb[i];
     const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
-    const unsigned peers = __match_any_sync(0xffffffffu, b);
-    if (valid && lane == 31 - __clz(peers)) mine[b] += __popc(peers);
+    peers[i] = same_key(valid, b, bits);
+    if (valid && lane == 31 - __clz(peers[i])) mine[b] += __popc(peers[i]);
     __syncwarp();
   }
   __syncthreads();
@@ -184,15 +201,14 @@ sort_scatter8_kernel(const int16_t* __restrict__ buckets, const int32_t* __restr
     const int e = beg + 32 * i + lane;
     const int b = kb[i];
     const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
-    const unsigned peers = __match_any_sync(0xffffffffu, b);
-    const int rank = __popc(peers & ((1u << lane) - 1u));
+    const int rank = __popc(peers[i] & ((1u << lane) - 1u));
     int slot = 0;
     if (valid) slot = mine[b] + rank;
     __syncwarp();
     if (valid) {
       P[slot] = e;
       if (U) U[e] = slot;
-      if (lane == 31 - __clz(peers)) mine[b] += __popc(peers);
+      if (lane == 31 - __clz(peers[i])) mine[b] += __popc(peers[i]);
     }
     __syncwarp();
   }
@@ -212,6 +228,7 @@ sort_scatter_kernel(const int16_t* __restrict__ buckets, const int32_t* __restri
   int32_t* P = perm + (size_t)seg * L;
   int32_t* U = undo ? undo + (size_t)seg * L : nullptr;
   const int beg = tile * kTileKeys, end = min(L, beg + kTileKeys);
+  const int bits = 32 - __clz(max(n_b - 1, 1));
   for (int base0 = beg; base0 < end; base0 += 32 * kBatch) {
     int kb[kBatch];
 #pragma unroll
@@ -224,7 +241,7 @@ sort_scatter_kernel(const int16_t* __restrict__ buckets, const int32_t* __restri
       const int e = base0 + 32 * i + lane;
       const int b = kb[i];
       const bool valid = (e < end) && (unsigned)b < (unsigned)n_b;
-      const unsigned peers = __match_any_sync(0xffffffffu, b);
+      const unsigned peers = same_key(valid, b, bits);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       int slot = 0;
       if (valid) slot = off[b] + rank;
