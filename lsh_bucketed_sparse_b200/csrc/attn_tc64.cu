@@ -25,22 +25,29 @@
 //               ||x|| * log2 e / sqrt(d) into the metadata ring;
 //   warp 2      v producer: the block's 128 rows of v into the value ring;
 //   warp 3      MMA issuer (one thread): S = Q K^T (look-back keys and the
-//               block's own keys are two MMAs per k-step), then O = P V;
+//               block's own keys are two MMAs per k-step), then O = P V and
+//               the row sums of P (P times a block of ones, N = 16);
 //   warps 4-11  softmax: two warps per TMEM lane quadrant (32 query rows),
 //               each taking alternate 32-key chunks of the row.  Keys are
 //               unit vectors, so a score never exceeds ||q|| / sqrt(d):
 //               that bound is the exponent's reference (p = 2^(s' - ref)
-//               <= 1) and the two warps only add partial sums; a row whose
-//               sum underflows is redone against its exact maximum.  Masks:
-//               window, causal (key position above the query's), self (the
-//               key j == i is left out; a row with no other key outputs v_i
-//               with lse -1e5, the value the -1e5 self score gives).  The
-//               output: each warp scales its half of the row's O columns by
-//               1/l and stores them at the row's original position.
-// TMEM: two buffers of 256 columns, S in [0, 192) (P written over the first
-// half of each 32-column chunk once read) and O in [192, 256); step t uses
-// buffer t & 1.  The softmax of step t+1 runs before the output of step t,
-// so P V of step t overlaps it.
+//               <= 1), and a term is then at least 2^(-2 ref), so the two
+//               warps need not exchange anything: each writes its P chunks
+//               as it goes and the tensor cores add the row.  Rows whose
+//               bound is so large that every term could flush to zero take
+//               their exact maximum as the reference instead (the quadrant's
+//               two warps exchange their halves' maxima).  Masks: window,
+//               causal (key position above the query's), self (the key
+//               j == i is left out; a row with no other key, i.e. a zero
+//               row sum, outputs v_i with lse -1e5, the value the -1e5 self
+//               score gives).  The output: each warp scales its half of the
+//               row's O columns by 1/l and stores them at the row's original
+//               position.
+// TMEM: S in two buffers of 192 columns (P written over the first half of
+// each 32-column chunk once read; step t uses buffer t & 1), then one O
+// buffer of 64 columns and the row sums.  The softmax of step t+1 runs
+// before the output of step t, so P V of step t overlaps it, and P V of step
+// t+1 waits only for that output to be read.
 #include <algorithm>
 #include <climits>
 
@@ -57,10 +64,11 @@ using namespace sm100;
 constexpr int kQ = 128;                 // queries per step = MMA M
 constexpr int kC = 64;                  // chunk length
 constexpr int kD = 64;                  // d_k
-constexpr int kNk = kC + kQ;            // key columns per step
+constexpr int kNk = kC + kQ;            // key columns per step = TMEM columns of an S buffer
 constexpr int kTile = kQ * kD * 2;      // one 128-row bf16 tile (128B-swizzled)
-constexpr int kBufCols = 256;           // TMEM columns per buffer
-constexpr int kOCol = kNk;              // O inside a buffer
+constexpr int kOCol = 2 * kNk;          // O (one buffer) after the two S buffers
+constexpr int kSumCol = kOCol + kD;     // P's row sums (16 equal columns)
+constexpr int kOnesBytes = 16 * 128;    // 16 rows of bf16 ones: B of the row-sum MMA
 constexpr int kQW = 2;                  // qk producer warps
 constexpr int kRowsQW = kQ / kQW;       // rows of a block per qk producer warp
 constexpr int kMmaWarp = 3;
@@ -74,7 +82,10 @@ constexpr int kMetaSlots = 8;
 constexpr int kMaxRounds = 8;  // rounds the duplicate correction carries per row
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-constexpr float kTinySum = 1e-20f;  // a row summing below this is redone with its max
+// A row's terms are 2^(s' - ref) >= 2^(-2 ref) with the bound as reference
+// (and >= 2^(-2 ref - 3) with the duplicate correction), so below this bound
+// no term can flush to zero; a row above it takes its exact maximum instead.
+constexpr float kBigRef = 58.f;
 
 static_assert(kRowsQW % 4 == 0, "gather4 moves four rows");
 
@@ -100,13 +111,13 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, pos, ksc, qref, bkt, chk, xch, bars, misc, total;
+  uint32_t qk, v, ones, pos, ksc, qref, bkt, chk, xch, bars, misc, total;
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
-  // rings; s_full, p_full, o_full, o_free (2 each); exchange (2 x 4); redo
-  // (4); done
-  return 2 * nq + 2 * nv + 2 * kMetaSlots + 8 + 8 + 4 + 1;
+  // rings; s_full, p_full, o_full, o_free (2 each); exact-max exchange (4);
+  // done
+  return 2 * nq + 2 * nv + 2 * kMetaSlots + 8 + 4 + 1;
 }
 
 template <bool BM, bool DD>
@@ -115,12 +126,13 @@ __host__ __device__ constexpr Layout layout(int nq, int nv) {
   uint32_t off = 0;
   l.qk = off;   off += nq * kTile;
   l.v = off;    off += nv * kTile;
+  l.ones = off; off += kOnesBytes;
   l.pos = off;  off += kMetaSlots * kQ * 4;
   l.ksc = off;  off += kMetaSlots * kQ * 4;
   l.qref = off; off += kMetaSlots * kQ * 4;
   l.bkt = off;  off += BM ? kMetaSlots * kQ * 4 : 0;
   l.chk = off;  off += DD ? kMetaSlots * kQ * kMaxRounds * 4 : 0;
-  l.xch = off;  off += (2 * 2 + 2 + 2) * kQ * 4;  // partial sums [2][2], maxima [2], redo sums [2]
+  l.xch = off;  off += 2 * 2 * kQ * 4;  // exact maxima [2 phases][2 halves]
   l.bars = off; off += n_barriers(nq, nv) * 8;
   l.misc = off; off += 16;
   l.total = off;
@@ -227,10 +239,15 @@ __device__ __forceinline__ int gather_row(int rowbase, int pos) {
 
 struct RowState {
   int qpos;   // original position (INT_MAX: no such query)
-  bool any;   // some key other than itself was visible
-  float lt;   // sum of 2^(s' - ref) over the row
   float ref;  // exponent reference, log2 units
 };
+
+// One column of 32 TMEM lanes: thread t reads lane (base + t).
+__device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+  return r;
+}
 
 // log2 of the number of rounds whose window of the query (chunk indices
 // `cq`) holds the key (chunk indices at `ck`).
@@ -269,9 +286,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
   float* qref_s = reinterpret_cast<float*>(smem + Ly.qref);
   int* bkt_s = reinterpret_cast<int*>(smem + Ly.bkt);
   int* chk_s = reinterpret_cast<int*>(smem + Ly.chk);  // [NM * kQ][kMaxRounds]
-  float* xl = reinterpret_cast<float*>(smem + Ly.xch);  // [2 buf][2 half][kQ]
-  float* xm = xl + 4 * kQ;                              // [2 half][kQ]
-  float* xl2 = xm + 2 * kQ;                             // [2 half][kQ]
+  float* xm = reinterpret_cast<float*>(smem + Ly.xch);  // [2 phases][2 half][kQ]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bars);
   uint64_t* qk_full = bars;            // [NQ] TMA bytes + one arrival per qk producer warp
   uint64_t* qk_empty = qk_full + NQ;   // [NQ] MMA: keys consumed
@@ -283,8 +298,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
   uint64_t* p_full = s_full + 2;       // [2] P in TMEM (softmax warps)
   uint64_t* o_full = p_full + 2;       // [2] O in TMEM; P (and with it S's buffer) consumed
   uint64_t* o_free = o_full + 2;       // [2] O read (softmax warps)
-  uint64_t* xbar = o_free + 2;         // [2][4] partial sums, the two warps of a quadrant
-  uint64_t* rbar = xbar + 8;           // [4] redo exchange
+  uint64_t* rbar = o_free + 2;         // [4] exact-max exchange, the two warps of a quadrant
   uint64_t* done = rbar + 4;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Ly.misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Ly.misc + 4);
@@ -308,9 +322,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       mbar_init(&p_full[b], kSoftWarps);
       mbar_init(&o_full[b], 1);
       mbar_init(&o_free[b], kSoftWarps);
-      for (int q = 0; q < 4; ++q) {
-        mbar_init(&xbar[b * 4 + q], 2);
-      }
     }
     for (int q = 0; q < 4; ++q) mbar_init(&rbar[q], 2);
     mbar_init(done, 1);
@@ -321,6 +332,10 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  // bf16 ones (every byte pair 0x3F80): the B operand of the row-sum MMA
+  for (int i = tid; i < kOnesBytes / 4; i += kThreads)
+    reinterpret_cast<uint32_t*>(smem + Ly.ones)[i] = 0x3F803F80u;
+  fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -485,7 +500,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       constexpr uint32_t idesc_prev = idesc_bf16_f32(kQ, kC);
       constexpr uint32_t idesc_cur = idesc_bf16_f32(kQ, kQ);
       constexpr uint32_t idesc_pv = idesc_bf16_f32_bmn(kQ, kD);
+      constexpr uint32_t idesc_sum = idesc_bf16_f32(kQ, 16);
       const uint32_t qk_base = smem_u32(qk_s), v_base = smem_u32(v_s);
+      // every byte pair of the tile is bf16 1.0, so one K-major descriptor
+      // (16 rows of N) serves every K step of the row-sum MMA
+      const uint64_t ones_desc = sdesc_kmajor_sw128(smem_u32(smem + Ly.ones));
       // S(s) = Q K^T into buffer ts & 1, once P V of step ts - 2 (which read
       // P from that buffer) is done.
       auto issue_qk = [&](const Unit& U, int first, int s, int ts) -> bool {
@@ -501,7 +520,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
             !mbar_wait_spin(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
-        const uint32_t s_tmem = tmem_base + b * kBufCols;
+        const uint32_t s_tmem = tmem_base + b * kNk;
         const uint64_t a0 = sdesc_kmajor_sw128(qk_base + cs * kTile);
         const uint64_t bp0 = sdesc_kmajor_sw128(qk_base + ps * kTile + (kQ - kC) * 128);
 #pragma unroll
@@ -523,15 +542,18 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         const int cs = ci % NV, ps = (pi + NV) % NV;
         const int b = ts & 1;
         if (!mbar_wait_spin(&p_full[b], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
-        if (!mbar_wait_spin(&o_free[b], (uint32_t)(((ts >> 1) & 1) ^ 1), abort_flag))
+        // one O buffer: the output pass of step ts - 1 must have read it
+        if (ts >= 1 && !mbar_wait_spin(&o_free[(ts - 1) & 1], (uint32_t)(((ts - 1) >> 1) & 1),
+                                       abort_flag))
           return false;
         if (!mbar_wait_spin(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
         if (has_prev && s == U.s0 &&
             !mbar_wait_spin(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
           return false;
         tc_fence_after_sync();
-        const uint32_t p_tmem = tmem_base + b * kBufCols;
-        const uint32_t o_tmem = p_tmem + kOCol;
+        const uint32_t p_tmem = tmem_base + b * kNk;
+        const uint32_t o_tmem = tmem_base + kOCol;
+        const uint32_t sum_tmem = tmem_base + kSumCol;
         const uint64_t dprev =
             sdesc_mnmajor_sw128(v_base + ps * kTile + (kQ - kC) * 128, kTile, 1024);
         const uint64_t dcur = sdesc_mnmajor_sw128(v_base + cs * kTile, kTile, 1024);
@@ -546,6 +568,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
           mma_bf16_ts(o_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
                       desc_add(dcur, (kk - kC / 16) * 16 * 128), idesc_pv,
                       (has_prev || kk > kC / 16) ? 1u : 0u);
+        // the row sums of P: P times a column block of ones (N = 16)
+        for (int kk = has_prev ? 0 : kC / 16; kk < kNk / 16; ++kk)
+          mma_bf16_ts(sum_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+                      desc_add(ones_desc, (kk & 3) * 32), idesc_sum,
+                      kk > (has_prev ? 0 : kC / 16) ? 1u : 0u);
         mma_commit(&o_full[b]);
         if (has_prev) mma_commit(&v_empty[ps]);
         if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
@@ -603,7 +630,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       const bool has_prev = s > 0;
       const int cs = ci % NM, ps = (pi + NM) % NM;
       const int b = ts & 1;
-      const uint32_t s_tmem = tmem_base + lane_off + b * kBufCols;
+      const uint32_t s_tmem = tmem_base + lane_off + b * kNk;
       if (!mbar_wait_spin(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
       if (has_prev && s == U.s0 &&
           !mbar_wait_spin(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
@@ -622,73 +649,12 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       const int lo = has_prev ? win_lo : max(win_lo, kC);
       // metadata row of key column j0 (a multiple of 32, all in one block)
       auto kbase = [&](int j0) { return j0 < kC ? ps * kQ + (kQ - kC) + j0 : cs * kQ + (j0 - kC); };
-      bool any = false;
-      float la[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pk[2][16];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) {
-        const int j0 = 32 * half + 64 * (kv0 + i);
-        if (j0 >= lo) {
-          uint32_t sv[32];
-          __syncwarp();
-          tmem_ld_32x32b_x32(s_tmem + j0, sv);
-          tmem_ld_wait(sv);
-          const int kb = kbase(j0);
-          // Causal: a key is visible iff its position is below the query's
-          // (one comparison, which also leaves the query itself out), and
-          // the row sees some key iff the chunk's smallest position does.
-          if (CAUSAL && !BMASK) any |= __reduce_min_sync(0xffffffffu, pos_s[kb + lane]) < qpos;
-#pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
-            const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
-            const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
-            const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
-            int kba[4] = {0, 0, 0, 0};
-            if (BMASK) {
-              const int4 kbv = *reinterpret_cast<const int4*>(bkt_s + kb + e);
-              kba[0] = kbv.x; kba[1] = kbv.y; kba[2] = kbv.z; kba[3] = kbv.w;
-            }
-            float pr[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              bool valid;
-              if (CAUSAL) {
-                valid = kpa[h] < qpos;
-              } else {
-                valid = kpa[h] <= qlim && kpa[h] != qpos;
-              }
-              if (BMASK) valid = valid && kba[h] == qb;
-              if (!CAUSAL || BMASK) any |= valid;
-              float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -qref);
-              if (DEDUP && valid) x -= DUP_LOG2(kb + e + h);
-              pr[h] = valid ? ex2(x) : 0.f;
-              la[h] += pr[h];
-            }
-            pk[i][e / 2] = pack_bf16(pr[0], pr[1]);
-            pk[i][e / 2 + 1] = pack_bf16(pr[2], pr[3]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 16; ++e) pk[i][e] = 0u;
-        }
-      }
-      const float l = (la[0] + la[1]) + (la[2] + la[3]);
-      // The two warps of the quadrant add their partial sums (a row that saw
-      // no key is carried as -1).
-      const int xb = ts & 1;
-      xl[(xb * 2 + half) * kQ + m] = any ? l : -1.f;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&xbar[xb * 4 + quad]);
-      if (!mbar_wait_spin(&xbar[xb * 4 + quad], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
-      const float other = xl[(xb * 2 + (half ^ 1)) * kQ + m];
-      any = any || other >= 0.f;
-      float lt = l + fmaxf(other, 0.f);
+      // The exponent reference is the row's bound ||q|| log2 e / sqrt(d)
+      // (every term <= 1), except in rows whose bound is so large that all
+      // their terms could flush to zero: those take their exact maximum over
+      // the visible keys (the two warps of the quadrant exchange halves).
       float ref = qref;
-      // Every term underflowed against the bound: redo the row against its
-      // exact maximum (S is still intact: P is written below).
-      const bool need = any && !(lt >= kTinySum);
-      if (__any_sync(0xffffffffu, need)) {
+      if (__any_sync(0xffffffffu, qref > kBigRef)) {
         float mx = -INFINITY;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -705,55 +671,66 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
               mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e] - DUP_LOG2(kb + e));
           }
         }
-        xm[half * kQ + m] = mx;
+        float* xmp = xm + rph * 2 * kQ;  // two phases: the other warp may still read the last
+        xmp[half * kQ + m] = mx;
         __syncwarp();
         if (lane == 0) mbar_arrive(&rbar[quad]);
         if (!mbar_wait_spin(&rbar[quad], rph, abort_flag)) return false;
         rph ^= 1;
-        const float gmax = fmaxf(mx, xm[(half ^ 1) * kQ + m]);
-        float l2 = 0.f;
+        const float gmax = fmaxf(mx, xmp[(half ^ 1) * kQ + m]);
+        if (qref > kBigRef && gmax > -INFINITY) ref = gmax;
+      }
+      // P (bf16) over the first 16 columns of each of this warp's 32-key
+      // chunks of S, zeros where the row's window does not reach; the row
+      // sums come from the tensor cores (P times ones) with P V.
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int j0 = 32 * half + 64 * (kv0 + i);
-          if (j0 < lo) continue;
+      for (int i = 0; i < 2; ++i) {
+        const int j0 = 32 * half + 64 * (kv0 + i);
+        uint32_t pk[16];
+        if (j0 >= lo) {
           uint32_t sv[32];
           __syncwarp();
           tmem_ld_32x32b_x32(s_tmem + j0, sv);
           tmem_ld_wait(sv);
-          if (!need) continue;
           const int kb = kbase(j0);
 #pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pr[2];
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-              const int kp = pos_s[kb + e + g];
-              const bool valid =
-                  kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e + g] == qb);
-              pr[g] = valid ? ex2(fmaf(__uint_as_float(sv[e + g]), ksc_s[kb + e + g], -gmax) -
-                                  DUP_LOG2(kb + e + g))
-                            : 0.f;
-              l2 += pr[g];
+          for (int e = 0; e < 32; e += 4) {
+            const int4 kp = *reinterpret_cast<const int4*>(pos_s + kb + e);
+            const float4 ks = *reinterpret_cast<const float4*>(ksc_s + kb + e);
+            const int kpa[4] = {kp.x, kp.y, kp.z, kp.w};
+            const float ksa[4] = {ks.x, ks.y, ks.z, ks.w};
+            int kba[4] = {0, 0, 0, 0};
+            if (BMASK) {
+              const int4 kbv = *reinterpret_cast<const int4*>(bkt_s + kb + e);
+              kba[0] = kbv.x; kba[1] = kbv.y; kba[2] = kbv.z; kba[3] = kbv.w;
             }
-            pk[i][e / 2] = pack_bf16(pr[0], pr[1]);
+            float pr[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              // Causal: a key is visible iff its position is below the
+              // query's (one comparison, which also leaves the query out).
+              bool valid;
+              if (CAUSAL) {
+                valid = kpa[h] < qpos;
+              } else {
+                valid = kpa[h] <= qlim && kpa[h] != qpos;
+              }
+              if (BMASK) valid = valid && kba[h] == qb;
+              float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -ref);
+              if (DEDUP && valid) x -= DUP_LOG2(kb + e + h);
+              pr[h] = valid ? ex2(x) : 0.f;
+            }
+            pk[e / 2] = pack_bf16(pr[0], pr[1]);
+            pk[e / 2 + 1] = pack_bf16(pr[2], pr[3]);
           }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) pk[e] = 0u;
         }
-        xl2[half * kQ + m] = l2;
         __syncwarp();
-        if (lane == 0) mbar_arrive(&rbar[quad]);
-        if (!mbar_wait_spin(&rbar[quad], rph, abort_flag)) return false;
-        rph ^= 1;
-        if (need) {
-          lt = l2 + xl2[(half ^ 1) * kQ + m];
-          ref = gmax;
-        }
+        tmem_st_32x32b_x16(s_tmem + j0, pk);
       }
 #undef DUP_LOG2
-      // P over the first 16 columns of each chunk's S; zeros where the row's
-      // window does not reach.
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < 2; ++i) tmem_st_32x32b_x16(s_tmem + 32 * half + 64 * (kv0 + i), pk[i]);
       tmem_st_32x32b_x16(s_tmem + 32 * half + 64 * kz, zeros);
       tmem_st_wait();
       tc_fence_before_sync();
@@ -766,8 +743,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         if (s == U.s1 - 1) mbar_arrive(&m_empty[cs]);
       }
       st.qpos = qpos;
-      st.any = any;
-      st.lt = lt;
       st.ref = ref;
       return true;
     };
@@ -782,13 +757,19 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       tc_fence_after_sync();
       uint32_t ov[32];
       __syncwarp();
-      tmem_ld_32x32b_x32(tmem_base + lane_off + b * kBufCols + kOCol + 32 * half, ov);
+      tmem_ld_32x32b_x32(tmem_base + lane_off + kOCol + 32 * half, ov);
+      uint32_t lsum = tmem_ld_32x32b_x1(tmem_base + lane_off + kSumCol);
       tmem_ld_wait(ov);
+      asm volatile("" : "+r"(lsum));  // not read before the wait above
+      const float lt = __uint_as_float(lsum);
       tc_fence_before_sync();
       __syncwarp();
       if (lane == 0) mbar_arrive(&o_free[b]);
       const bool q_valid = st.qpos != INT_MAX;
-      const float inv_l = st.any ? 1.f / st.lt : 0.f;
+      // every visible key adds a positive term (no term flushes to zero, see
+      // kBigRef), so the row saw a key other than itself iff its sum is > 0
+      const bool any = lt > 0.f;
+      const float inv_l = any ? 1.f / lt : 0.f;
       uint4 w[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -801,7 +782,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         w[q].w = pack_bf16(__uint_as_float(ov[8 * q + 6]) * inv_l,
                            __uint_as_float(ov[8 * q + 7]) * inv_l);
       }
-      const bool self_only = q_valid && !st.any;
+      const bool self_only = q_valid && !any;
       if (__any_sync(0xffffffffu, self_only)) {
         // nothing but itself to attend to: the -1e5 self score makes it v_i
         const __nv_bfloat16* vrow = p.v + ((size_t)U.bh * p.L + (q_valid ? st.qpos : 0)) * kD;
@@ -816,7 +797,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       }
       const size_t seg_row = ((size_t)U.bh * p.n_h + U.r) * p.L;
       if (half == 0 && q_valid)
-        p.lse_rounds[seg_row + st.qpos] = st.any ? st.ref * kLn2 + logf(st.lt) : kSelfScore;
+        p.lse_rounds[seg_row + st.qpos] = any ? st.ref * kLn2 + logf(lt) : kSelfScore;
       return true;
     };
 
