@@ -42,7 +42,9 @@
 //               row sum, outputs v_i with lse -1e5, the value the -1e5 self
 //               score gives).  The output: each warp scales its half of the
 //               row's O columns by 1/l and stores them at the row's original
-//               position.
+//               position as two 32-byte stores (o_rounds 32-byte aligned):
+//               a warp's store touches 32 rows, so its number of stores
+//               sets the load/store unit's work.
 // TMEM: S in two buffers of 192 columns (P written over the first half of
 // each 32-column chunk once read; step t uses buffer t & 1), then one O
 // buffer of 64 columns and the row sums.  The softmax of step t+1 runs
@@ -241,6 +243,13 @@ struct RowState {
   int qpos;   // original position (INT_MAX: no such query)
   float ref;  // exponent reference, log2 units
 };
+
+// 32 bytes to global memory in one store (the address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a.x),
+               "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
 
 // One column of 32 TMEM lanes: thread t reads lane (base + t).
 __device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
@@ -791,9 +800,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
           if (self_only) w[q] = reinterpret_cast<const uint4*>(vrow + 32 * half)[q];
       }
       if (q_valid) {
-        uint4* orow = reinterpret_cast<uint4*>(p.o_rounds + (((size_t)U.bh * p.n_h + U.r) * p.L + st.qpos) * kD + 32 * half);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) orow[q] = w[q];
+        // the half row (64 bytes, 32-byte aligned) as two 32-byte stores
+        __nv_bfloat16* orow =
+            p.o_rounds + (((size_t)U.bh * p.n_h + U.r) * p.L + st.qpos) * kD + 32 * half;
+        st_global_v8(orow, w[0], w[1]);
+        st_global_v8(orow + 16, w[2], w[3]);
       }
       const size_t seg_row = ((size_t)U.bh * p.n_h + U.r) * p.L;
       if (half == 0 && q_valid)

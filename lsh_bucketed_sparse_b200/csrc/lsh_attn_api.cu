@@ -131,7 +131,8 @@ lsh_status run_attn(const Problem& p, const void* qk, const void* v, const float
                     const int32_t* perm, const int32_t* undo, const int16_t* buckets,
                     void* o_r, float* lse_r, cudaStream_t st) {
   cudaError_t e = cudaErrorNotSupported;
-  if (!p.portable && attn_tc64_supported(p))
+  // (the chunk-64 kernel writes o_rounds in 32-byte stores)
+  if (!p.portable && attn_tc64_supported(p) && reinterpret_cast<uintptr_t>(o_r) % 32 == 0)
     e = launch_attn_tc64(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st);
   else if (!p.portable && attn_tc_supported(p) && !(p.dedup && (p.bucket_mask || p.n_h > 8)))
     e = launch_attn_tc(p, qk, v, inv_norm, perm, buckets, undo, o_r, lse_r, st);

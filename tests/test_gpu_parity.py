@@ -633,3 +633,29 @@ def test_binding_rejects_mismatched_device_tensors():
         with pytest.raises((ValueError, TypeError)):
             call()
     lsh.lsh_attn_device_check()
+
+
+def test_o_rounds_only_16_byte_aligned_gives_the_same_result():
+    # The chunk-64 kernel stores o_rounds in 32-byte pieces; an o_rounds that
+    # is 16-byte aligned but not 32 (allowed by the boundary) takes the
+    # general kernel instead, with the same result up to its own rounding.
+    wl = W.small("align16", heads=2, seq_len=1024, n_hashes=2, n_buckets=64)
+    qk, v, rot = [t.to(DEV) for t in W.make_inputs(wl)]
+    b, inv = lsh.lsh_attn_hash(qk, rot, wl.n_buckets, wl.n_hashes)
+    perm, _, _ = lsh.lsh_attn_sort(b, wl.n_buckets, want_undo=False)
+    o_ref, l_ref = lsh.lsh_attn_chunked_fwd(qk, v, inv, perm, wl.chunk_len, wl.causal,
+                                            n_buckets=wl.n_buckets)
+    n = o_ref.numel()
+    raw = torch.empty(n + 64, dtype=qk.dtype, device=DEV)
+    shift = (-(raw.data_ptr() // 2) % 16) + 8   # 16 bytes past a 32-byte boundary
+    o_mis = raw[shift:shift + n].view_as(o_ref)
+    assert o_mis.data_ptr() % 32 == 16
+    l_mis = torch.empty_like(l_ref)
+    shp = lsh.make_shape(wl.batch, wl.heads, wl.seq_len, wl.d_k, wl.n_hashes, wl.n_buckets,
+                         wl.chunk_len, wl.causal, wl.dtype)
+    lsh._check(lsh.lib().lsh_attn_chunked_fwd(
+        ctypes.byref(shp), lsh._ptr(qk), lsh._ptr(v), lsh._ptr(inv), lsh._ptr(perm),
+        lsh._ptr(o_mis), lsh._ptr(l_mis), lsh._stream(None)))
+    torch.cuda.synchronize()
+    P.check_float(o_mis.cpu(), o_ref.cpu(), True, "o_rounds (16-byte aligned)", 3)
+    P.check_lse(l_mis.cpu(), l_ref.cpu(), True, "lse_rounds (16-byte aligned)")
