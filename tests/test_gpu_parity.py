@@ -245,6 +245,26 @@ def test_large_norms_take_the_exact_max_path(chunk, d):
     print(wl.name, report)
 
 
+@pytest.mark.parametrize("chunk,d", [(64, 64), (128, 128)])
+@pytest.mark.parametrize("causal", [True, False])
+def test_mixed_norms_in_one_warp(chunk, d, causal):
+    # Every third token scaled by 256 (exact in bf16): in most warps some rows
+    # take their exact maximum as the exponent reference and the rest keep
+    # the bound, inside the same pass (and a large-norm query's keys are
+    # mostly ordinary ones, and the reverse).
+    wl = W.small(f"mixed-norm-{chunk}-{d}-{int(causal)}", heads=2, seq_len=1536, d_k=d,
+                 n_hashes=2, n_buckets=64, chunk_len=chunk, causal=causal)
+
+    def scale(qk):
+        f = torch.ones(qk.shape[-2], 1, dtype=qk.dtype)
+        f[::3] = 256
+        return qk * f
+
+    report, g = _full_check(wl, qk_override=scale)
+    assert torch.isfinite(g["out"].float()).all()
+    print(wl.name, report)
+
+
 def test_deterministic():
     wl = W.small("det", heads=2, seq_len=1024, n_hashes=2, n_buckets=64)
     qk, v, rot = [t.to(DEV) if t is not None else None for t in W.make_inputs(wl)]
