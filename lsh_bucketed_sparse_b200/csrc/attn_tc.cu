@@ -91,11 +91,19 @@ struct Params {
   int L, n_h, causal;
   StepSplit split;    // the CTAs' share of the steps (ceil(L / 128) per segment)
   float ksc;          // log2 e / sqrt(d)
+  int o32;            // o_rounds is 32-byte aligned: 32-byte stores
 };
 
 struct Layout {
   uint32_t qk, v, p, pos, ksc, qref, bkt, chk, xch, bars, misc, total;
 };
+
+// 32 bytes to global memory in one store (the address 32-byte aligned).
+__device__ __forceinline__ void st_global_v8(void* ptr, const uint4& a, const uint4& b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr), "r"(a.x),
+               "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
   // rings; S/O/P full/free pairs (2 x 6); exchange (2 x 4); redo (4); done
@@ -799,8 +807,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
           }
         }
         if (q_valid) {
+          if (p.o32) {
+            // two 32-byte stores: each store of the warp touches 32 rows
+            st_global_v8(orow + d0, w[0], w[1]);
+            st_global_v8(orow + d0 + 16, w[2], w[3]);
+          } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
+            for (int q = 0; q < 4; ++q) reinterpret_cast<uint4*>(orow + d0)[q] = w[q];
+          }
         }
       }
       if (half == 0 && q_valid)
@@ -868,6 +882,7 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   int grid = 0;
   p.split = make_step_split((long long)pr.BH() * pr.n_h, (pr.L + kQ - 1) / kQ, sm_count(), grid);
   p.ksc = kLog2e / sqrtf((float)pr.d);
+  p.o32 = reinterpret_cast<uintptr_t>(o_rounds) % 32 == 0 ? 1 : 0;
   auto encode = tensor_map_encoder();
   if (!encode) return cudaErrorNotSupported;
   // [B*H*L, d] views of qk and v: boxes of one row of 64 elements (128 B),
