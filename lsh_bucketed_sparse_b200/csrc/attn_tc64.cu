@@ -81,12 +81,11 @@ constexpr int kThreads = (kSoftBase + kSoftWarps) * 32;  // 3 warps per schedule
 
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kMetaSlots = 8;
-constexpr int kMaxRounds = 8;  // rounds the duplicate correction carries per row
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
-// A row's terms are 2^(s' - ref) >= 2^(-2 ref) with the bound as reference
-// (and >= 2^(-2 ref - 3) with the duplicate correction), so below this bound
-// no term can flush to zero; a row above it takes its exact maximum instead.
+// A row's terms are 2^(s' - ref) >= 2^(-2 ref) with the bound as reference,
+// so below this bound no term can flush to zero; a row above it takes its
+// exact maximum instead.
 constexpr float kBigRef = 58.f;
 
 static_assert(kRowsQW % 4 == 0, "gather4 moves four rows");
@@ -105,7 +104,6 @@ struct Params {
   __nv_bfloat16* o_rounds;
   float* lse_rounds;
   const int16_t* buckets;  // [BH, n_h, L] for the bucket-equality mask, else null
-  const int32_t* undo;     // [BH, n_h, L] every round's undo for the duplicate correction
   unsigned int* err;
   int L, n_h, causal;
   StepSplit split;  // the CTAs' share of the steps
@@ -113,7 +111,7 @@ struct Params {
 };
 
 struct Layout {
-  uint32_t qk, v, ones, pos, ksc, qref, bkt, chk, xch, bars, misc, total;
+  uint32_t qk, v, ones, pos, ksc, qref, bkt, xch, bars, misc, total;
 };
 
 __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
@@ -122,7 +120,7 @@ __host__ __device__ constexpr uint32_t n_barriers(int nq, int nv) {
   return 2 * nq + 2 * nv + 2 * kMetaSlots + 8 + 4 + 1;
 }
 
-template <bool BM, bool DD>
+template <bool BM>
 __host__ __device__ constexpr Layout layout(int nq, int nv) {
   Layout l{};
   uint32_t off = 0;
@@ -133,7 +131,6 @@ __host__ __device__ constexpr Layout layout(int nq, int nv) {
   l.ksc = off;  off += kMetaSlots * kQ * 4;
   l.qref = off; off += kMetaSlots * kQ * 4;
   l.bkt = off;  off += BM ? kMetaSlots * kQ * 4 : 0;
-  l.chk = off;  off += DD ? kMetaSlots * kQ * kMaxRounds * 4 : 0;
   l.xch = off;  off += 2 * 2 * kQ * 4;  // exact maxima [2 phases][2 halves]
   l.bars = off; off += n_barriers(nq, nv) * 8;
   l.misc = off; off += 16;
@@ -149,16 +146,16 @@ struct Plan {
 
 // Ring depths that fit: key tiles first (a block is live for two steps as
 // queries and look-back keys), at most six of each.
-template <bool BM, bool DD>
+template <bool BM>
 __host__ __device__ constexpr Plan make_plan() {
   constexpr uint32_t limit = kSmemLimit - 1024;  // 1024 for aligning the base
-  const uint32_t fixed = layout<BM, DD>(0, 0).total + n_barriers(6, 6) * 8;
+  const uint32_t fixed = layout<BM>(0, 0).total + n_barriers(6, 6) * 8;
   if (fixed >= limit) return Plan{0, 0, 0, false};
   const int tiles = (int)((limit - fixed) / kTile);
   if (tiles < 5) return Plan{0, 0, 0, false};
   const int q = (tiles + 1) / 2 < 6 ? (tiles + 1) / 2 : 6;
   const int v = tiles - q < 6 ? tiles - q : 6;
-  const uint32_t smem = layout<BM, DD>(q, v).total + 1024;
+  const uint32_t smem = layout<BM>(q, v).total + 1024;
   return Plan{q, v, smem, smem <= (uint32_t)kSmemLimit};
 }
 
@@ -258,43 +255,25 @@ __device__ __forceinline__ uint32_t tmem_ld_32x32b_x1(uint32_t taddr) {
   return r;
 }
 
-// log2 of the number of rounds whose window of the query (chunk indices
-// `cq`) holds the key (chunk indices at `ck`).
-__device__ __forceinline__ float dup_log2(const int* ck, const int (&cq)[kMaxRounds], int n_h) {
-  const int4 a = *reinterpret_cast<const int4*>(ck);
-  const int4 b = *reinterpret_cast<const int4*>(ck + 4);
-  const int k8[kMaxRounds] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-  int n = 0;
-#pragma unroll
-  for (int rr = 0; rr < kMaxRounds; ++rr)
-    n += (rr < n_h && (unsigned)(cq[rr] - k8[rr]) <= 1u) ? 1 : 0;
-  float l;
-  asm("lg2.approx.f32 %0, %1;" : "=f"(l) : "f"((float)max(n, 1)));
-  return l;
-}
-
 // BMASK: the bucket-equality mask (section 2: a query attends only to
-// targets in its own bucket).  DEDUP: the duplicate-count correction
-// (Appendix A "Duplicate handling"): a visible key's exponent loses
-// log2 N_ij, N_ij = the rounds r' (at most kMaxRounds) with
-// chunk_r'(i) - chunk_r'(j) in {0, 1}.
-template <bool CAUSAL, bool BMASK, bool DEDUP>
+// targets in its own bucket).  The duplicate-count correction runs on the
+// general kernel (attn_tc.cu), which measured faster for it.
+template <bool CAUSAL, bool BMASK>
 __global__ void __launch_bounds__(kThreads, 1)
 attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap vmap,
               const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  constexpr Plan PL = make_plan<BMASK, DEDUP>();
+  constexpr Plan PL = make_plan<BMASK>();
   constexpr int NQ = PL.nq, NV = PL.nv, NM = kMetaSlots;
-  constexpr Layout Ly = layout<BMASK, DEDUP>(NQ, NV);
+  constexpr Layout Ly = layout<BMASK>(NQ, NV);
   uint8_t* qk_s = smem + Ly.qk;
   uint8_t* v_s = smem + Ly.v;
   int* pos_s = reinterpret_cast<int*>(smem + Ly.pos);
   float* ksc_s = reinterpret_cast<float*>(smem + Ly.ksc);
   float* qref_s = reinterpret_cast<float*>(smem + Ly.qref);
   int* bkt_s = reinterpret_cast<int*>(smem + Ly.bkt);
-  int* chk_s = reinterpret_cast<int*>(smem + Ly.chk);  // [NM * kQ][kMaxRounds]
   float* xm = reinterpret_cast<float*>(smem + Ly.xch);  // [2 phases][2 half][kQ]
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Ly.bars);
   uint64_t* qk_full = bars;            // [NQ] TMA bytes + one arrival per qk producer warp
@@ -411,14 +390,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
           ksc_s[row] = in0[k] * p.ksc;
           qref_s[row] = in0[k] > 0.f ? p.ksc / in0[k] : 0.f;
           if (BMASK) bkt_s[row] = bk0[k];
-          if (DEDUP) {
-            const size_t ub = (size_t)c0.U.bh * p.n_h * p.L;
-#pragma unroll
-            for (int rr = 0; rr < kMaxRounds; ++rr)
-              chk_s[row * kMaxRounds + rr] =
-                  (rr < p.n_h && pos0[k] != INT_MAX) ? p.undo[ub + (size_t)rr * p.L + pos0[k]] / kC
-                                                     : -2;
-          }
         }
       }
       __syncwarp();
@@ -649,11 +620,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
       const int qb = BMASK ? bkt_s[cs * kQ + m] : 0;
-      int cq[kMaxRounds];
-#pragma unroll
-      for (int rr = 0; rr < kMaxRounds; ++rr)
-        cq[rr] = DEDUP ? chk_s[(cs * kQ + m) * kMaxRounds + rr] : 0;
-#define DUP_LOG2(kr) (DEDUP ? dup_log2(chk_s + (kr) * kMaxRounds, cq, p.n_h) : 0.f)
       const int qlim = p.causal ? qpos : INT_MAX - 1;
       const int lo = has_prev ? win_lo : max(win_lo, kC);
       // metadata row of key column j0 (a multiple of 32, all in one block)
@@ -677,7 +643,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
           for (int e = 0; e < 32; ++e) {
             const int kp = pos_s[kb + e];
             if (kp <= qlim && kp != qpos && (!BMASK || bkt_s[kb + e] == qb))
-              mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e] - DUP_LOG2(kb + e));
+              mx = fmaxf(mx, __uint_as_float(sv[e]) * ksc_s[kb + e]);
           }
         }
         float* xmp = xm + rph * 2 * kQ;  // two phases: the other warp may still read the last
@@ -725,8 +691,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
                 valid = kpa[h] <= qlim && kpa[h] != qpos;
               }
               if (BMASK) valid = valid && kba[h] == qb;
-              float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -ref);
-              if (DEDUP && valid) x -= DUP_LOG2(kb + e + h);
+              const float x = fmaf(__uint_as_float(sv[e + h]), ksa[h], -ref);
               pr[h] = valid ? ex2(x) : 0.f;
             }
             pk[e / 2] = pack_bf16(pr[0], pr[1]);
@@ -739,7 +704,6 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         __syncwarp();
         tmem_st_32x32b_x16(s_tmem + j0, pk);
       }
-#undef DUP_LOG2
       tmem_st_32x32b_x16(s_tmem + 32 * half + 64 * kz, zeros);
       tmem_st_wait();
       tc_fence_before_sync();
@@ -843,8 +807,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
 }  // namespace
 
 bool attn_tc64_supported(const Problem& p) {
-  return p.bf16 && p.d == kD && p.c == kC && !(p.bucket_mask && p.dedup) &&
-         !(p.dedup && p.n_h > kMaxRounds) &&
+  return p.bf16 && p.d == kD && p.c == kC && !p.dedup &&
          (long long)p.BH() * p.n_h * p.L < (1LL << 31) - 1 &&
          sm100::tensor_map_encoder() != nullptr;
 }
@@ -854,12 +817,11 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
                              const int32_t* undo, void* o_rounds, float* lse_rounds,
                              cudaStream_t st) {
   if (!pr.bucket_mask) buckets = nullptr;
-  if (!pr.dedup) undo = nullptr;
-  if (buckets && undo) return cudaErrorNotSupported;
-  constexpr Plan PL = make_plan<false, false>();
-  constexpr Plan PLM = make_plan<true, false>();
-  constexpr Plan PLD = make_plan<false, true>();
-  static_assert(PL.ok && PLM.ok && PLD.ok, "no shared-memory plan");
+  (void)undo;  // the duplicate correction runs on the general kernel
+  if (pr.dedup) return cudaErrorNotSupported;
+  constexpr Plan PL = make_plan<false>();
+  constexpr Plan PLM = make_plan<true>();
+  static_assert(PL.ok && PLM.ok, "no shared-memory plan");
   unsigned int* err = device_error_word();
   if (!err) return cudaErrorUnknown;
   Params p;
@@ -869,7 +831,6 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
   p.o_rounds = static_cast<__nv_bfloat16*>(o_rounds);
   p.lse_rounds = lse_rounds;
   p.buckets = buckets;
-  p.undo = undo;
   p.err = err;
   p.L = pr.L;
   p.n_h = pr.n_h;
@@ -895,14 +856,10 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
         CUDA_SUCCESS)
       return cudaErrorInvalidValue;
   }
-  const bool bmask = buckets != nullptr, dedup = undo != nullptr;
-  const size_t smem = dedup ? PLD.smem : (bmask ? PLM.smem : PL.smem);
-  auto kernel = pr.causal ? (dedup ? attn64_kernel<true, false, true>
-                                   : (bmask ? attn64_kernel<true, true, false>
-                                            : attn64_kernel<true, false, false>))
-                          : (dedup ? attn64_kernel<false, false, true>
-                                   : (bmask ? attn64_kernel<false, true, false>
-                                            : attn64_kernel<false, false, false>));
+  const bool bmask = buckets != nullptr;
+  const size_t smem = bmask ? PLM.smem : PL.smem;
+  auto kernel = pr.causal ? (bmask ? attn64_kernel<true, true> : attn64_kernel<true, false>)
+                          : (bmask ? attn64_kernel<false, true> : attn64_kernel<false, false>);
   cudaError_t e;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
