@@ -179,6 +179,9 @@ LSH_ATTN_API lsh_status lsh_attn_sort(const lsh_shape* shape, const int16_t* buc
  *   inv_norm    [B, H, L]         float32 (from stage 1).
  *   perm        [B, H, n_h, L]    int32 (from stage 2).
  *   o_rounds    [B, H, n_h, L, d] dtype out: softmax-weighted v per round.
+ *               16-byte alignment suffices; with 32-byte alignment (every
+ *               cudaMalloc'd buffer) the bf16 kernels write it in 32-byte
+ *               stores, which is faster.
  *   lse_rounds  [B, H, n_h, L]    float32 out: log-sum-exp of the scores.
  * ---------------------------------------------------------------------- */
 LSH_ATTN_API lsh_status lsh_attn_chunked_fwd(const lsh_shape* shape, const void* qk, const void* v,
