@@ -488,12 +488,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const bool has_prev = s > 0;
         const int cs = (int)(ci % NQ), ps = (int)(((pi % NQ) + NQ) % NQ);
         const int buf = (int)(ts % K::kNbuf);
-        if (!mbar_wait_spin(&s_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
-          return false;
-        if (!mbar_wait_spin(&qk_full[cs], (uint32_t)((ci / NQ) & 1), abort_flag)) return false;
-        if (has_prev && s == U.s0 &&
-            !mbar_wait_spin(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
-          return false;
+        // the free S buffer, this block's keys and, at a strip's first
+        // step, the look-back block's (tested together)
+        {
+          const uint32_t pc = (uint32_t)((ci / NQ) & 1);
+          const bool back = has_prev && s == U.s0;
+          if (!mbar_wait4_spin(&s_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1),
+                               &qk_full[cs], pc, back ? &qk_full[ps] : &qk_full[cs],
+                               back ? (uint32_t)((pi / NQ) & 1) : pc, &qk_full[cs], pc,
+                               abort_flag))
+            return false;
+        }
         tc_fence_after_sync();
         const uint32_t s_tmem = tmem_base + buf * K::kBufCols;
         const uint32_t qa = smem_u32(qk_s + (size_t)cs * K::kTile);
@@ -517,13 +522,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
         const int cs = (int)(ci % NV), ps = (int)(((pi % NV) + NV) % NV);
         const int buf = (int)(ts % K::kNbuf);
         const int pb = (int)(ts % NP);
-        if (!mbar_wait_spin(&p_full[pb], (uint32_t)((ts / NP) & 1), abort_flag)) return false;
-        if (!mbar_wait_spin(&o_free[buf], (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), abort_flag))
-          return false;
-        if (!mbar_wait_spin(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
-        if (has_prev && s == U.s0 &&
-            !mbar_wait_spin(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
-          return false;
+        // P of this step, a free O buffer, this block's values and, at a
+        // strip's first step, the look-back block's (tested together)
+        {
+          const uint32_t vc = (uint32_t)((ci / NV) & 1);
+          const bool back = has_prev && s == U.s0;
+          if (!mbar_wait4_spin(&p_full[pb], (uint32_t)((ts / NP) & 1), &o_free[buf],
+                               (uint32_t)(((ts / K::kNbuf) & 1) ^ 1), &v_full[cs], vc,
+                               back ? &v_full[ps] : &v_full[cs],
+                               back ? (uint32_t)((pi / NV) & 1) : vc, abort_flag))
+            return false;
+        }
         tc_fence_after_sync();
         const uint32_t o_tmem = tmem_base + buf * K::kBufCols + K::kNk;
         const uint32_t pbase = smem_u32(p_s + (size_t)pb * K::kPBytes);
@@ -593,11 +602,17 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int buf = (int)(ts % K::kNbuf);
       const int pb = (int)(ts % NP);
       const uint32_t s_tmem = tmem_base + lane_off + buf * K::kBufCols;
-      if (!mbar_wait_spin(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
-      if (has_prev && s == U.s0 &&
-          !mbar_wait_spin(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
-        return false;
-      if (!mbar_wait_spin(&s_full[buf], (uint32_t)((ts / K::kNbuf) & 1), abort_flag)) return false;
+      // S of this step, the step's metadata (and, at a strip's first step,
+      // the look-back block's) and a free P buffer, tested together
+      {
+        const uint32_t mc = (uint32_t)((ci / NM) & 1);
+        const bool back = has_prev && s == U.s0;
+        if (!mbar_wait4_warp(&s_full[buf], (uint32_t)((ts / K::kNbuf) & 1), &m_full[cs], mc,
+                             back ? &m_full[ps] : &m_full[cs],
+                             back ? (uint32_t)((pi / NM) & 1) : mc, &p_empty[pb],
+                             (uint32_t)(((ts / NP) & 1) ^ 1), abort_flag))
+          return false;
+      }
       tc_fence_after_sync();
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
@@ -612,7 +627,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
       const int lo = has_prev ? win_lo : max(win_lo, C);
       // metadata row of key column j0 (a multiple of 32, all in one block)
       auto kbase = [&](int j0) { return j0 < C ? ps * kQ + (kQ - C) + j0 : cs * kQ + (j0 - C); };
-      if (!mbar_wait_spin(&p_empty[pb], (uint32_t)(((ts / NP) & 1) ^ 1), abort_flag)) return false;
       uint8_t* prow = p_s + (size_t)pb * K::kPBytes;
       bool any = false;
       float la[4] = {0.f, 0.f, 0.f, 0.f};

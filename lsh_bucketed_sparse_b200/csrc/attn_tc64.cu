@@ -24,9 +24,10 @@
 //               scale 1/||x|| * log2 e / sqrt(d) and query reference
 //               ||x|| * log2 e / sqrt(d) into the metadata ring;
 //   warp 2      v producer: the block's 128 rows of v into the value ring;
-//   warp 3      MMA issuer (one thread): S = Q K^T (look-back keys and the
-//               block's own keys are two MMAs per k-step), then O = P V and
-//               the row sums of P (P times a block of ones, N = 16);
+//   warp 3      MMA issuer (the warp waits, one elected lane issues):
+//               S = Q K^T (look-back keys and the block's own keys are two
+//               MMAs per k-step), then O = P V and the row sums of P (P
+//               times a block of ones, N = 16);
 //   warps 4-11  softmax: two warps per TMEM lane quadrant (32 query rows),
 //               each taking alternate 32-key chunks of the row.  Keys are
 //               unit vectors, so a score never exceeds ||q|| / sqrt(d):
@@ -162,6 +163,12 @@ __host__ __device__ constexpr Plan make_plan() {
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -474,7 +481,13 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     }
   } else if (warp == kMmaWarp) {
     // ============================================================== MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the loop and one elected lane issues, and a step's
+    // barriers are tested together (their round trips overlap): on the
+    // long-text workload 0.47 ms a launch against 0.50 with the loop in lane
+    // 0 alone and one barrier at a time, on the causal 4x8x4096 one 0.078
+    // against 0.092 (the general kernel and the hash measured slower with
+    // the warp-wide loop and keep the lone lane).
+    {
       int li = 0, t = 0;  // blocks consumed, steps issued
       bool ok = true, issued = false;
       constexpr uint32_t idesc_prev = idesc_bf16_f32(kQ, kC);
@@ -492,26 +505,32 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         const bool has_prev = s > 0;
         const int cs = ci % NQ, ps = (pi + NQ) % NQ;
         const int b = ts & 1;
-        if (ts >= 2 &&
-            !mbar_wait_spin(&o_full[b], (uint32_t)(((ts >> 1) - 1) & 1), abort_flag))
-          return false;
-        if (!mbar_wait_spin(&qk_full[cs], (uint32_t)((ci / NQ) & 1), abort_flag)) return false;
-        if (has_prev && s == U.s0 &&
-            !mbar_wait_spin(&qk_full[ps], (uint32_t)((pi / NQ) & 1), abort_flag))
+        // the buffer's last P V (step ts - 2), this block's keys and, at a
+        // strip's first step, the look-back block's
+        const uint32_t pc = (uint32_t)((ci / NQ) & 1);
+        const bool old = ts >= 2, back = has_prev && s == U.s0;
+        if (!mbar_wait4_warp(&qk_full[cs], pc,
+                             old ? &o_full[b] : &qk_full[cs],
+                             old ? (uint32_t)(((ts >> 1) - 1) & 1) : pc,
+                             back ? &qk_full[ps] : &qk_full[cs],
+                             back ? (uint32_t)((pi / NQ) & 1) : pc, &qk_full[cs], pc, abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t s_tmem = tmem_base + b * kNk;
         const uint64_t a0 = sdesc_kmajor_sw128(qk_base + cs * kTile);
         const uint64_t bp0 = sdesc_kmajor_sw128(qk_base + ps * kTile + (kQ - kC) * 128);
+        if (elect_one_sync()) {
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          const uint64_t a = desc_add(a0, kk * 32);
-          if (has_prev) mma_bf16_ss(s_tmem, a, desc_add(bp0, kk * 32), idesc_prev, kk > 0);
-          mma_bf16_ss(s_tmem + kC, a, a, idesc_cur, kk > 0);
+          for (int kk = 0; kk < kD / 16; ++kk) {
+            const uint64_t a = desc_add(a0, kk * 32);
+            if (has_prev) mma_bf16_ss(s_tmem, a, desc_add(bp0, kk * 32), idesc_prev, kk > 0);
+            mma_bf16_ss(s_tmem + kC, a, a, idesc_cur, kk > 0);
+          }
+          mma_commit(&s_full[b]);
+          if (has_prev) mma_commit(&qk_empty[ps]);
+          if (s == U.s1 - 1) mma_commit(&qk_empty[cs]);
         }
-        mma_commit(&s_full[b]);
-        if (has_prev) mma_commit(&qk_empty[ps]);
-        if (s == U.s1 - 1) mma_commit(&qk_empty[cs]);
+        __syncwarp();
         return true;
       };
       // O(s) = P(s) V, P read from tensor memory: keys [16 kk, 16 kk + 16)
@@ -521,14 +540,16 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         const bool has_prev = s > 0;
         const int cs = ci % NV, ps = (pi + NV) % NV;
         const int b = ts & 1;
-        if (!mbar_wait_spin(&p_full[b], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
-        // one O buffer: the output pass of step ts - 1 must have read it
-        if (ts >= 1 && !mbar_wait_spin(&o_free[(ts - 1) & 1], (uint32_t)(((ts - 1) >> 1) & 1),
-                                       abort_flag))
-          return false;
-        if (!mbar_wait_spin(&v_full[cs], (uint32_t)((ci / NV) & 1), abort_flag)) return false;
-        if (has_prev && s == U.s0 &&
-            !mbar_wait_spin(&v_full[ps], (uint32_t)((pi / NV) & 1), abort_flag))
+        // P of this step, the one O buffer read by the output pass of step
+        // ts - 1, this block's values and, at a strip's first step, the
+        // look-back block's
+        const uint32_t pp = (uint32_t)((ts >> 1) & 1), vc = (uint32_t)((ci / NV) & 1);
+        const bool back = has_prev && s == U.s0;
+        if (!mbar_wait4_warp(&p_full[b], pp,
+                             ts >= 1 ? &o_free[(ts - 1) & 1] : &p_full[b],
+                             ts >= 1 ? (uint32_t)(((ts - 1) >> 1) & 1) : pp, &v_full[cs], vc,
+                             back ? &v_full[ps] : &v_full[cs],
+                             back ? (uint32_t)((pi / NV) & 1) : vc, abort_flag))
           return false;
         tc_fence_after_sync();
         const uint32_t p_tmem = tmem_base + b * kNk;
@@ -537,25 +558,28 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         const uint64_t dprev =
             sdesc_mnmajor_sw128(v_base + ps * kTile + (kQ - kC) * 128, kTile, 1024);
         const uint64_t dcur = sdesc_mnmajor_sw128(v_base + cs * kTile, kTile, 1024);
-        if (has_prev) {
+        if (elect_one_sync()) {
+          if (has_prev) {
 #pragma unroll
-          for (int kk = 0; kk < kC / 16; ++kk)
+            for (int kk = 0; kk < kC / 16; ++kk)
+              mma_bf16_ts(o_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+                          desc_add(dprev, kk * 16 * 128), idesc_pv, kk > 0);
+          }
+#pragma unroll
+          for (int kk = kC / 16; kk < kNk / 16; ++kk)
             mma_bf16_ts(o_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                        desc_add(dprev, kk * 16 * 128), idesc_pv, kk > 0);
+                        desc_add(dcur, (kk - kC / 16) * 16 * 128), idesc_pv,
+                        (has_prev || kk > kC / 16) ? 1u : 0u);
+          // the row sums of P: P times a column block of ones (N = 16)
+          for (int kk = has_prev ? 0 : kC / 16; kk < kNk / 16; ++kk)
+            mma_bf16_ts(sum_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
+                        desc_add(ones_desc, (kk & 3) * 32), idesc_sum,
+                        kk > (has_prev ? 0 : kC / 16) ? 1u : 0u);
+          mma_commit(&o_full[b]);
+          if (has_prev) mma_commit(&v_empty[ps]);
+          if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
         }
-#pragma unroll
-        for (int kk = kC / 16; kk < kNk / 16; ++kk)
-          mma_bf16_ts(o_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                      desc_add(dcur, (kk - kC / 16) * 16 * 128), idesc_pv,
-                      (has_prev || kk > kC / 16) ? 1u : 0u);
-        // the row sums of P: P times a column block of ones (N = 16)
-        for (int kk = has_prev ? 0 : kC / 16; kk < kNk / 16; ++kk)
-          mma_bf16_ts(sum_tmem, p_tmem + 32 * (kk >> 1) + 8 * (kk & 1),
-                      desc_add(ones_desc, (kk & 3) * 32), idesc_sum,
-                      kk > (has_prev ? 0 : kC / 16) ? 1u : 0u);
-        mma_commit(&o_full[b]);
-        if (has_prev) mma_commit(&v_empty[ps]);
-        if (s == U.s1 - 1) mma_commit(&v_empty[cs]);
+        __syncwarp();
         return true;
       };
       for (int k = 0; ok; ++k) {
@@ -573,11 +597,11 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
           if (!issue_pv(U, first, s, t)) { ok = false; break; }
         }
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         atomicOr(p.err, kErrWaitMma);
         *abort_flag = 1;
       }
-      if (issued) {
+      if (issued && elect_one_sync()) {
         mma_commit(done);
         const unsigned long long t0 = globaltimer();
         while (!mbar_try_wait(done, 0)) {
@@ -611,11 +635,14 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       const int cs = ci % NM, ps = (pi + NM) % NM;
       const int b = ts & 1;
       const uint32_t s_tmem = tmem_base + lane_off + b * kNk;
-      if (!mbar_wait_spin(&m_full[cs], (uint32_t)((ci / NM) & 1), abort_flag)) return false;
-      if (has_prev && s == U.s0 &&
-          !mbar_wait_spin(&m_full[ps], (uint32_t)((pi / NM) & 1), abort_flag))
-        return false;
-      if (!mbar_wait_spin(&s_full[b], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
+      {
+        const uint32_t mc = (uint32_t)((ci / NM) & 1), sp = (uint32_t)((ts >> 1) & 1);
+        const bool back = has_prev && s == U.s0;
+        if (!mbar_wait4_warp(&s_full[b], sp, &m_full[cs], mc,
+                             back ? &m_full[ps] : &m_full[cs],
+                             back ? (uint32_t)((pi / NM) & 1) : mc, &s_full[b], sp, abort_flag))
+          return false;
+      }
       tc_fence_after_sync();
       const int qpos = pos_s[cs * kQ + m];
       const float qref = qref_s[cs * kQ + m];
@@ -721,9 +748,9 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     };
 
     // Output of step s: the two warps of a quadrant each take half of the D
-    // columns of its 32 rows, scale by 1/l, and stage them in shared memory
-    // (16-byte pieces XOR-swizzled by the row); then each warp writes 16
-    // whole rows to their original positions, eight lanes per 128-byte row.
+    // columns of its 32 rows, scale them by 1/l, and each lane writes its
+    // row's half (64 bytes) to the row's original position as two 32-byte
+    // stores; the half-0 warp also writes the row's log-sum-exp.
     auto o_pass = [&](const Unit& U, int ts, int s, const RowState& st) -> bool {
       const int b = ts & 1;
       if (!mbar_wait_spin(&o_full[b], (uint32_t)((ts >> 1) & 1), abort_flag)) return false;
@@ -771,8 +798,9 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         st_global_v8(orow + 16, w[2], w[3]);
       }
       const size_t seg_row = ((size_t)U.bh * p.n_h + U.r) * p.L;
-      if (half == 0 && q_valid)
-        p.lse_rounds[seg_row + st.qpos] = any ? st.ref * kLn2 + logf(lt) : kSelfScore;
+      // the two warps of the quadrant take turns (a step each)
+      if (half == (ts & 1) && q_valid)
+        p.lse_rounds[seg_row + st.qpos] = any ? (st.ref + lg2(lt)) * kLn2 : kSelfScore;
       return true;
     };
 

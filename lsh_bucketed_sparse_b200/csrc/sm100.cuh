@@ -146,6 +146,57 @@ __device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity,
   }
 }
 
+// Spins, as a whole converged warp, until the phases of all four barriers
+// have completed (repeat a barrier to wait on fewer).  The four tests of a
+// pass are independent, so their shared-memory round trips overlap instead of
+// adding up; a warp vote gives every lane the same verdict.  A completed
+// phase cannot complete again before the caller acts, so a lane that saw it
+// early loses nothing by waiting for the vote.  Same abort flag and time
+// limit as mbar_wait_spin.
+__device__ __forceinline__ bool mbar_wait4_warp(uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                                uint32_t p1, uint64_t* b2, uint32_t p2,
+                                                uint64_t* b3, uint32_t p3,
+                                                const volatile int* abort) {
+  unsigned long long t0 = 0;
+  for (uint32_t n = 0;; ++n) {
+    const bool d = mbar_test(b0, p0) & mbar_test(b1, p1) & mbar_test(b2, p2) & mbar_test(b3, p3);
+    if (__all_sync(0xffffffffu, d)) return true;
+    if (n == 0) t0 = globaltimer();
+    if ((n & 1023u) == 1023u) {
+      const bool stop = *abort || globaltimer() - t0 > kWaitLimitNs;
+      if (__any_sync(0xffffffffu, stop)) return false;
+    }
+  }
+}
+
+// mbar_wait_spin over four barriers at once for a single thread (repeat a
+// barrier to wait on fewer): the four tests of a pass are independent, so
+// their round trips overlap.
+__device__ __forceinline__ bool mbar_wait4_spin(uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                                uint32_t p1, uint64_t* b2, uint32_t p2,
+                                                uint64_t* b3, uint32_t p3,
+                                                const volatile int* abort) {
+  unsigned long long t0 = 0;
+  for (uint32_t n = 0;; ++n) {
+    if (mbar_test(b0, p0) & mbar_test(b1, p1) & mbar_test(b2, p2) & mbar_test(b3, p3))
+      return true;
+    if (n == 0) t0 = globaltimer();
+    if ((n & 1023u) == 1023u && (*abort || globaltimer() - t0 > kWaitLimitNs)) return false;
+  }
+}
+
+// True in exactly one active lane of a converged warp.
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, %1;\n\t"
+      "selp.b32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred)
+      : "r"(0xffffffffu));
+  return pred != 0;
+}
+
 // ---- fences -------------------------------------------------------------------
 // Generic-proxy writes to shared memory -> visible to the async proxy (TMA,
 // tensor core).
