@@ -172,6 +172,7 @@ __device__ __forceinline__ float lg2(float x) {
   return y;
 }
 
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
@@ -378,8 +379,8 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         bk1[k] = bucket_of(c1, pos1[k]);
       }
       const int qs = li % NQ, ms = li % NM;
-      if (!mbar_wait_spin(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
-      if (!mbar_wait_spin(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&qk_empty[qs], (uint32_t)(((li / NQ) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&m_empty[ms], (uint32_t)(((li / NM) & 1) ^ 1), abort_flag)) { ok = false; break; }
       if (lane == 0) mbar_expect_tx(&qk_full[qs], kRowsQW * kD * 2);
       __syncwarp();
       const int rowbase = c0.U.bh * p.L;
@@ -447,7 +448,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
       int pos2[4];
       cursor_positions(c2, p, r0, pos2);
       const int vs = li % NV;
-      if (!mbar_wait_spin(&v_empty[vs], (uint32_t)(((li / NV) & 1) ^ 1), abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&v_empty[vs], (uint32_t)(((li / NV) & 1) ^ 1), abort_flag)) { ok = false; break; }
       if (lane == 0) mbar_expect_tx(&v_full[vs], vrows(w) * kD * 2);
       __syncwarp();
       const int rowbase = c0.U.bh * p.L;
@@ -481,12 +482,13 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
     }
   } else if (warp == kMmaWarp) {
     // ============================================================== MMA issuer
-    // The whole warp runs the loop and one elected lane issues, and a step's
-    // barriers are tested together (their round trips overlap): on the
+    // The whole warp runs the loop and one elected lane issues (on the
     // long-text workload 0.47 ms a launch against 0.50 with the loop in lane
-    // 0 alone and one barrier at a time, on the causal 4x8x4096 one 0.078
-    // against 0.092 (the general kernel and the hash measured slower with
-    // the warp-wide loop and keep the lone lane).
+    // 0 alone; the general kernel and the hash measured slower that way and
+    // keep the lone lane).  Its waits sleep in try_wait instead of polling,
+    // as the producers' do: a polling warp takes issue slots and shared-
+    // memory round trips from the two softmax warps of its scheduler, which
+    // then finish their P pass last (0.441 against 0.469 ms).
     {
       int li = 0, t = 0;  // blocks consumed, steps issued
       bool ok = true, issued = false;
@@ -509,7 +511,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         // strip's first step, the look-back block's
         const uint32_t pc = (uint32_t)((ci / NQ) & 1);
         const bool old = ts >= 2, back = has_prev && s == U.s0;
-        if (!mbar_wait4_warp(&qk_full[cs], pc,
+        if (!mbar_wait4_sleep(&qk_full[cs], pc,
                              old ? &o_full[b] : &qk_full[cs],
                              old ? (uint32_t)(((ts >> 1) - 1) & 1) : pc,
                              back ? &qk_full[ps] : &qk_full[cs],
@@ -545,7 +547,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
         // look-back block's
         const uint32_t pp = (uint32_t)((ts >> 1) & 1), vc = (uint32_t)((ci / NV) & 1);
         const bool back = has_prev && s == U.s0;
-        if (!mbar_wait4_warp(&p_full[b], pp,
+        if (!mbar_wait4_sleep(&p_full[b], pp,
                              ts >= 1 ? &o_free[(ts - 1) & 1] : &p_full[b],
                              ts >= 1 ? (uint32_t)(((ts - 1) >> 1) & 1) : pp, &v_full[cs], vc,
                              back ? &v_full[ps] : &v_full[cs],

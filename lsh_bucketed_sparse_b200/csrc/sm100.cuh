@@ -169,6 +169,18 @@ __device__ __forceinline__ bool mbar_wait4_warp(uint64_t* b0, uint32_t p0, uint6
   }
 }
 
+// mbar_wait on four barriers in turn for a converged warp (repeat a barrier
+// to wait on fewer): the warp sleeps instead of polling, and a vote gives
+// every lane the same verdict.
+__device__ __forceinline__ bool mbar_wait4_sleep(uint64_t* b0, uint32_t p0, uint64_t* b1,
+                                                 uint32_t p1, uint64_t* b2, uint32_t p2,
+                                                 uint64_t* b3, uint32_t p3,
+                                                 const volatile int* abort) {
+  const bool ok = mbar_wait(b0, p0, abort) && mbar_wait(b1, p1, abort) &&
+                  mbar_wait(b2, p2, abort) && mbar_wait(b3, p3, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // mbar_wait_spin over four barriers at once for a single thread (repeat a
 // barrier to wait on fewer): the four tests of a pass are independent, so
 // their round trips overlap.
