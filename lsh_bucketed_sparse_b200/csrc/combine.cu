@@ -61,7 +61,9 @@ combine_kernel(const T* __restrict__ o_rounds, const float* __restrict__ lse_rou
   using V = Vec16<T>;
   const int n_h = NH > 0 ? NH : n_h_rt;
   const int per_row = d / V::N;
-  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  // blocks run in roughly increasing index order: the last rows first, since
+  // the attention wrote the last heads' rounds last and they may still be in L2
+  const long long tid = (long long)(gridDim.x - 1 - blockIdx.x) * blockDim.x + threadIdx.x;
   const long long row = tid / per_row;
   const int part = (int)(tid % per_row);
   if (row >= rows) return;
