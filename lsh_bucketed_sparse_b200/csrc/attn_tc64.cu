@@ -15,8 +15,11 @@
 //     (no P ring in shared memory, no P stores through the LSU);
 //   - the key gathers of a block are issued by two TMA warps (a warp's
 //     tile::gather4 operations are serialised: about 66 cycles each);
-//   - the MMA thread issues from descriptors computed once per step plus
-//     compile-time offsets.
+//   - the MMA issuer is a whole warp (one elected lane issues) working from
+//     descriptors computed once per step plus compile-time offsets;
+//   - the warps that are not on the critical path (MMA issuer, producers)
+//     sleep in try_wait; the softmax warps poll all of a step's barriers in
+//     one pass.
 //
 // Warp roles (12 warps, 168 registers each):
 //   warps 0-1   qk producers: rows [64 w, 64 w + 64) of every block: TMA
@@ -45,7 +48,8 @@
 //               row's O columns by 1/l and stores them at the row's original
 //               position as two 32-byte stores (o_rounds 32-byte aligned):
 //               a warp's store touches 32 rows, so its number of stores
-//               sets the load/store unit's work.
+//               sets the load/store unit's work; the two warps write the
+//               row's log-sum-exp on alternate steps.
 // TMEM: S in two buffers of 192 columns (P written over the first half of
 // each 32-column chunk once read; step t uses buffer t & 1), then one O
 // buffer of 64 columns and the row sums.  The softmax of step t+1 runs
