@@ -349,6 +349,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  wait_prior_grid();
   tc_fence_before_sync();
   __syncthreads();
   tc_fence_after_sync();
@@ -929,7 +930,9 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
   cudaError_t e = cudaFuncSetAttribute(kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kernel<<<(unsigned)grid, kThreads, smem, st>>>(maps[0], maps[1], p); note_launch();
+  e = launch_dependent(kernel, dim3((unsigned)grid), dim3(kThreads), smem, st, maps[0], maps[1], p);
+  note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

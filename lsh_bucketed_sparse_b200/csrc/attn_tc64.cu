@@ -335,6 +335,7 @@ attn64_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ 
   // bf16 ones (every byte pair 0x3F80): the B operand of the row-sum MMA
   for (int i = tid; i < kOnesBytes / 4; i += kThreads)
     reinterpret_cast<uint32_t*>(smem + Ly.ones)[i] = 0x3F803F80u;
+  wait_prior_grid();
   fence_proxy_async_smem();
   tc_fence_before_sync();
   __syncthreads();
@@ -897,8 +898,9 @@ cudaError_t launch_attn_tc64(const Problem& pr, const void* qk, const void* v,
   cudaError_t e;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  kernel<<<(unsigned)grid, kThreads, smem, st>>>(maps[0], maps[1], p);
+  e = launch_dependent(kernel, dim3((unsigned)grid), dim3(kThreads), smem, st, maps[0], maps[1], p);
   note_launch();
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -58,6 +58,7 @@ __global__ void __launch_bounds__(kThreads)
 combine_kernel(const T* __restrict__ o_rounds, const float* __restrict__ lse_rounds,
                T* __restrict__ out, float* __restrict__ lse, long long rows, int L, int d,
                int n_h_rt) {
+  wait_prior_grid();
   using V = Vec16<T>;
   const int n_h = NH > 0 ? NH : n_h_rt;
   const int per_row = d / V::N;
@@ -128,14 +129,22 @@ void launch_t(const Problem& p, const void* o_rounds, const float* lse_rounds, v
               float* lse, unsigned blocks, long long rows, cudaStream_t st) {
   const T* o = static_cast<const T*>(o_rounds);
   T* y = static_cast<T*>(out);
-  switch (p.n_h) {
-    case 1: combine_kernel<T, 1><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 1); note_launch(); break;
-    case 2: combine_kernel<T, 2><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 2); note_launch(); break;
-    case 4: combine_kernel<T, 4><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 4); note_launch(); break;
-    case 8: combine_kernel<T, 8><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, 8); note_launch(); break;
-    default:
-      combine_kernel<T, 0><<<blocks, kThreads, 0, st>>>(o, lse_rounds, y, lse, rows, p.L, p.d, p.n_h); note_launch();
+  // launch errors surface through the caller's cudaGetLastError
+  const int nh = p.n_h;
+  const dim3 g(blocks), b(kThreads);
+  switch (nh) {
+    case 1: (void)launch_dependent(combine_kernel<T, 1>, g, b, 0, st, o, lse_rounds, y, lse, rows,
+                                   p.L, p.d, 1); break;
+    case 2: (void)launch_dependent(combine_kernel<T, 2>, g, b, 0, st, o, lse_rounds, y, lse, rows,
+                                   p.L, p.d, 2); break;
+    case 4: (void)launch_dependent(combine_kernel<T, 4>, g, b, 0, st, o, lse_rounds, y, lse, rows,
+                                   p.L, p.d, 4); break;
+    case 8: (void)launch_dependent(combine_kernel<T, 8>, g, b, 0, st, o, lse_rounds, y, lse, rows,
+                                   p.L, p.d, 8); break;
+    default: (void)launch_dependent(combine_kernel<T, 0>, g, b, 0, st, o, lse_rounds, y, lse,
+                                    rows, p.L, p.d, nh);
   }
+  note_launch();
 }
 
 }  // namespace

@@ -22,6 +22,17 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
   return __float2bfloat16_rn(x);
 }
 
+// Programmatic dependent launch: the forward path's kernels are launched
+// so that one may be set up (launch, shared-memory and tensor-memory
+// allocation, barrier initialisation) while the kernel before it on the
+// stream finishes; every thread waits here for that kernel to complete,
+// with its writes visible, before it touches global memory.  No kernel
+// triggers its successor early: when the short kernels did, the next
+// kernel's CTAs sat beside them and the long-text pass got slower.
+__device__ __forceinline__ void wait_prior_grid() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

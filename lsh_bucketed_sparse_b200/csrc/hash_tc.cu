@@ -177,6 +177,7 @@ hash_tc_kernel(const __grid_constant__ CUtensorMap xmap, const Params p) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
+  wait_prior_grid();
   // Rotations of this group -> shared memory, K-major with 128B swizzle:
   // operand row n = column (rr * P + j) of the group, k = input dimension.
   for (int idx = tid; idx < p.n_cols * (p.d / 8); idx += kThreads) {
@@ -614,7 +615,10 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
   if (e != cudaSuccess) return e;
-  kernel<<<plan.n_groups * plan.G, kThreads, plan.smem, st>>>(map, p); note_launch();
+  cudaError_t le = launch_dependent(kernel, dim3(plan.n_groups * plan.G), dim3(kThreads),
+                                    plan.smem, st, map, p);
+  note_launch();
+  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 

@@ -55,6 +55,24 @@ cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
 // after its <<<...>>>); read through lsh_attn_kernel_launches().
 void note_launch();
 
+// Launch with programmatic stream serialisation allowed (the kernel calls
+// wait_prior_grid before its first global-memory access).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                             cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Streaming multiprocessors of the current device (148 on B200; 148 if the
 // query fails), cached per device.
 int sm_count();

@@ -63,6 +63,7 @@ sort_count_kernel(const int16_t* __restrict__ buckets, int32_t* __restrict__ cnt
   extern __shared__ int32_t hist[];  // [n_b]
   const int seg = blockIdx.x, tile = blockIdx.y;
   for (int b = threadIdx.x; b < n_b; b += blockDim.x) hist[b] = 0;
+  wait_prior_grid();
   __syncthreads();
   const int16_t* keys = buckets + (size_t)seg * L;
   const int beg = tile * kTileKeys, end = min(L, beg + kTileKeys);
@@ -125,6 +126,7 @@ sort_scan_kernel(int32_t* __restrict__ cnt, int32_t* __restrict__ counts,
   extern __shared__ int32_t base[];  // [n_b]
   const int seg = blockIdx.x;
   int32_t* c = cnt + (size_t)seg * T * n_b;
+  wait_prior_grid();
   // The tiles are walked kScanBatch at a time with all of a batch's loads
   // issued before any is used, so a thread waits on memory once per batch.
   for (int b = threadIdx.x; b < n_b; b += blockDim.x) {
@@ -156,6 +158,7 @@ sort_scatter8_kernel(const int16_t* __restrict__ buckets, const int32_t* __restr
                      int32_t* __restrict__ undo, int L, int n_b, int T) {
   extern __shared__ int32_t off[];  // [kScatterWarps][n_b]
   const int seg = blockIdx.x, tile = blockIdx.y;
+  wait_prior_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t* mine = off + (size_t)warp * n_b;
   for (int b = lane; b < n_b; b += 32) mine[b] = 0;
@@ -220,6 +223,7 @@ sort_scatter_kernel(const int16_t* __restrict__ buckets, const int32_t* __restri
                     int32_t* __restrict__ undo, int L, int n_b, int T) {
   extern __shared__ int32_t off[];  // [n_b]
   const int seg = blockIdx.x, tile = blockIdx.y, lane = threadIdx.x;
+  wait_prior_grid();
   const int32_t* c = cnt + ((size_t)seg * T + tile) * n_b;
   const int32_t* bs = base + (size_t)seg * n_b;
   for (int b = lane; b < n_b; b += 32) off[b] = c[b] + bs[b];
@@ -296,15 +300,25 @@ cudaError_t launch_sort(const Problem& p, const int16_t* buckets, int32_t* perm,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)hist_bytes)))
       return e;
   }
-  sort_count_kernel<<<dim3(segs, T), kCountThreads, hist_bytes, st>>>(buckets, cnt, p.L, n_b, T); note_launch();
-  sort_scan_kernel<<<segs, kScanThreads, hist_bytes, st>>>(cnt, counts, base, n_b, T); note_launch();
+  if ((e = launch_dependent(sort_count_kernel, dim3(segs, T), dim3(kCountThreads), hist_bytes, st,
+                            buckets, cnt, p.L, n_b, T)))
+    return e;
+  note_launch();
+  if ((e = launch_dependent(sort_scan_kernel, dim3(segs), dim3(kScanThreads), hist_bytes, st, cnt,
+                            counts, base, n_b, T)))
+    return e;
+  note_launch();
   if (wide) {
-    sort_scatter8_kernel<<<dim3(segs, T), kScatterWarps * 32, scatter8_bytes, st>>>(
-        buckets, cnt, base, perm, undo, p.L, n_b, T); note_launch();
+    e = launch_dependent(sort_scatter8_kernel, dim3(segs, T), dim3(kScatterWarps * 32),
+                         scatter8_bytes, st, buckets, static_cast<const int32_t*>(cnt),
+                         static_cast<const int32_t*>(base), perm, undo, p.L, n_b, T);
   } else {
-    sort_scatter_kernel<<<dim3(segs, T), 32, hist_bytes, st>>>(buckets, cnt, base, perm, undo,
-                                                                p.L, n_b, T); note_launch();
+    e = launch_dependent(sort_scatter_kernel, dim3(segs, T), dim3(32), hist_bytes, st, buckets,
+                         static_cast<const int32_t*>(cnt), static_cast<const int32_t*>(base),
+                         perm, undo, p.L, n_b, T);
   }
+  if (e) return e;
+  note_launch();
   return cudaGetLastError();
 }
 
