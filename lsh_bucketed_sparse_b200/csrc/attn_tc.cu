@@ -931,8 +931,8 @@ cudaError_t launch_cd(const Problem& pr, const void* qk, const void* v, const fl
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   e = launch_dependent(kernel, dim3((unsigned)grid), dim3(kThreads), smem, st, maps[0], maps[1], p);
-  note_launch();
   if (e != cudaSuccess) return e;
+  note_launch();
   return cudaGetLastError();
 }
 

@@ -615,10 +615,10 @@ cudaError_t launch_hash_tc(const Problem& pr, const void* qk, const void* rot, i
   cudaError_t e =
       cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)plan.smem);
   if (e != cudaSuccess) return e;
-  cudaError_t le = launch_dependent(kernel, dim3(plan.n_groups * plan.G), dim3(kThreads),
-                                    plan.smem, st, map, p);
+  e = launch_dependent(kernel, dim3(plan.n_groups * plan.G), dim3(kThreads), plan.smem, st, map,
+                       p);
+  if (e != cudaSuccess) return e;
   note_launch();
-  if (le != cudaSuccess) return le;
   return cudaGetLastError();
 }
 

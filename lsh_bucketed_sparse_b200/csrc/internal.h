@@ -52,7 +52,7 @@ cudaError_t launch_backward(const Problem& p, const void* qk, const void* v,
                             void* workspace, cudaStream_t st);
 
 // Counts one kernel launch of this library (every launch site calls it right
-// after its <<<...>>>); read through lsh_attn_kernel_launches().
+// after its launch); read through lsh_attn_kernel_launches().
 void note_launch();
 
 // Launch with programmatic stream serialisation allowed (the kernel calls
