@@ -44,6 +44,7 @@ attn_portable_kernel(const T* __restrict__ qk, const T* __restrict__ v,
                      T* __restrict__ o_rounds,
                      float* __restrict__ lse_rounds, int L, int d, int n_h, int c, int causal,
                      float scale) {
+  wait_prior_grid();
   extern __shared__ float smem[];
   float* ks = smem;                              // [kKB][d + 1]
   float* vs = ks + (size_t)kKB * (d + 1);        // [kKB][d]
@@ -179,14 +180,15 @@ cudaError_t launch_attn_portable(const Problem& p, const void* qk, const void* v
                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                 (int)smem);
   if (e != cudaSuccess) return e;
-  if (p.bf16)
-    attn_portable_kernel<__nv_bfloat16><<<grid, kWarps * 32, smem, st>>>(
-        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm, undo, buckets,
-        (__nv_bfloat16*)o_rounds, lse_rounds, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
-  else
-    attn_portable_kernel<float><<<grid, kWarps * 32, smem, st>>>(
-        (const float*)qk, (const float*)v, inv_norm, perm, undo, buckets, (float*)o_rounds, lse_rounds, p.L,
-        p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
+  const dim3 b(kWarps * 32);
+  e = p.bf16 ? launch_dependent(attn_portable_kernel<__nv_bfloat16>, grid, b, smem, st,
+                                (const __nv_bfloat16*)qk, (const __nv_bfloat16*)v, inv_norm, perm,
+                                undo, buckets, (__nv_bfloat16*)o_rounds, lse_rounds, p.L, p.d,
+                                p.n_h, p.c, p.causal ? 1 : 0, scale)
+             : launch_dependent(attn_portable_kernel<float>, grid, b, smem, st, (const float*)qk,
+                                (const float*)v, inv_norm, perm, undo, buckets, (float*)o_rounds,
+                                lse_rounds, p.L, p.d, p.n_h, p.c, p.causal ? 1 : 0, scale);
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }

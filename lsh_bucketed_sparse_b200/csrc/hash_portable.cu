@@ -26,6 +26,7 @@ hash_portable_kernel(const T* __restrict__ qk, const T* __restrict__ rot,
                      int16_t* __restrict__ buckets, float* __restrict__ inv_norm, int BH, int L,
                      int d, int n_h, int half, int n_cent) {
   extern __shared__ float xs_all[];  // [kWarps][d]
+  wait_prior_grid();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   float* xs = xs_all + warp * d;
   const long long rows = (long long)BH * L;
@@ -91,14 +92,16 @@ cudaError_t launch_hash_portable(const Problem& p, const void* qk, const void* r
   long long blocks = (rows + kWarps - 1) / kWarps;
   if (blocks > 148 * 16) blocks = 148 * 16;
   const size_t smem = (size_t)kWarps * p.d * sizeof(float);
-  if (p.bf16)
-    hash_portable_kernel<__nv_bfloat16><<<(unsigned)blocks, kWarps * 32, smem, st>>>(
-        (const __nv_bfloat16*)qk, (const __nv_bfloat16*)rot, buckets, inv_norm, p.BH(), p.L,
-        p.d, p.n_h, p.kmeans ? 0 : p.half(), p.kmeans ? p.n_b : 0);
-  else
-    hash_portable_kernel<float><<<(unsigned)blocks, kWarps * 32, smem, st>>>(
-        (const float*)qk, (const float*)rot, buckets, inv_norm, p.BH(), p.L, p.d, p.n_h,
-        p.kmeans ? 0 : p.half(), p.kmeans ? p.n_b : 0);
+  const dim3 g((unsigned)blocks), b(kWarps * 32);
+  const int half = p.kmeans ? 0 : p.half(), n_cent = p.kmeans ? p.n_b : 0;
+  const cudaError_t e =
+      p.bf16 ? launch_dependent(hash_portable_kernel<__nv_bfloat16>, g, b, smem, st,
+                                (const __nv_bfloat16*)qk, (const __nv_bfloat16*)rot, buckets,
+                                inv_norm, p.BH(), p.L, p.d, p.n_h, half, n_cent)
+             : launch_dependent(hash_portable_kernel<float>, g, b, smem, st, (const float*)qk,
+                                (const float*)rot, buckets, inv_norm, p.BH(), p.L, p.d, p.n_h,
+                                half, n_cent);
+  if (e != cudaSuccess) return e;
   note_launch();
   return cudaGetLastError();
 }
