@@ -137,15 +137,6 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 16-byte shared-memory store issued only where `pred` holds, without a branch.
-__device__ __forceinline__ void st_shared_if(bool pred, uint32_t addr, uint4 v) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %0, 0;\n\t"
-      "@p st.shared.v4.b32 [%1], {%2, %3, %4, %5};\n\t}" ::"r"((uint32_t)pred),
-      "r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-      : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&h);
